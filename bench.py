@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the HSTU jagged layer stack on B200 through the C ABI.
+
+One step = one forward pass of the 4-layer bf16 HSTU stack over one synthetic jagged batch
+(8 users, lengths U{2048..8192}, d_model 512, 8 heads of width 64, interleaved item/action
+tokens): per layer the f1 GEMM + SiLU, the jagged causal pointwise attention with relative
+position/time bias, LayerNorm(AV) ⊙ U and the f2 GEMM + residual.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch (a different seed of
+the same workload, weak scaling); no collective sits on the data path, only the timing barrier
+and the max-over-ranks reduction of the measured time.
+
+Prints one JSON line on rank 0.  ``value`` is layer-tokens/s (tokens x layers / device time);
+the attention kernel's TFLOP/s (unmasked causal FLOPs only) and its roofline fraction are in
+``attn_tflops`` and ``roofline``.  The reference arm (``--impl reference``) times the fp64
+CPU oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hstu_sequential_transducer_jagged_b200 import workloads as W  # noqa: E402
+
+WORKLOAD = "stack4_bf16_b8_inter"
+METRIC = "HSTU jagged causal attention TFLOP/s & layer tokens/s on 1 B200 (% of peak)"
+UNIT = "layer-tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def attention_pairs(wl) -> int:
+    pairs = 0
+    for L in wl.lengths.tolist():
+        if wl.mask == W.MASK_MFALCON:
+            n = max(L - wl.num_candidates, 0)
+            m = L - n
+            pairs += n * (n + 1) // 2 + m * (n + 1)
+        else:
+            pairs += L * (L + 1) // 2
+    return pairs
+
+
+def attention_flops(wl) -> float:
+    return 4.0 * wl.d_qk * wl.num_heads * attention_pairs(wl)
+
+
+def gemm_flops(wl) -> float:
+    n1 = 2 * wl.num_heads * (wl.d_qk + wl.d_v)
+    hv = wl.num_heads * wl.d_v
+    return 2.0 * wl.total_tokens * wl.d_model * n1 + 2.0 * wl.total_tokens * hv * wl.d_model
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def attn_traffic_bytes():
+    """DRAM bytes per attention launch from the committed ncu summary, if the kernel source is
+    unchanged since the counters were taken (else None)."""
+    summ = os.path.join(ROOT, "profiles", "attn_fwd_tc_stack4.json")
+    src = os.path.join(ROOT, "hstu_sequential_transducer_jagged_b200", "csrc", "attn_fwd_tc.cu")
+    if not os.path.exists(summ):
+        return None
+    with open(summ) as f:
+        rec = json.load(f)
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if rec.get("kernel_source_sha256") != digest:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_layer_sample(wl, seconds_min=10.0, max_reps=3):
+    """The fp64 oracle on a bounded sample of the workload: one layer over its shortest
+    sequence, repeated until seconds_min of CPU work.  Returns (tokens/s, sample, threads)."""
+    from oracle import hstu_oracle as O
+    b = int(np.argmin(wl.lengths))
+    s, e = int(wl.seq_offsets[b]), int(wl.seq_offsets[b + 1])
+    off = np.array([0, e - s])
+    lp = wl.layers[0]
+    kw = dict(num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, max_pos_dist=wl.max_pos_dist,
+              num_time_buckets=wl.num_time_buckets, alpha=wl.alpha, mask=wl.mask,
+              num_candidates=wl.num_candidates)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.layer_forward(wl.x[s:e], lp.w1, lp.w2, off, wl.timestamps[s:e], lp.rab_pos,
+                        lp.rab_time, **kw)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds_min or reps >= max_reps:
+            break
+    sample = (f"one fp64 oracle layer over sequence {b} ({e - s} tokens, the shortest) of "
+              f"{wl.name} seed 0, {reps} rep(s), {el:.1f} s")
+    return (e - s) * reps / el, sample, len(os.sched_getaffinity(0))
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    wl = W.make(WORKLOAD, seed=args.seed)
+    from oracle import hstu_oracle as O
+    b = int(np.argmin(wl.lengths))
+    s, e = int(wl.seq_offsets[b]), int(wl.seq_offsets[b + 1])
+    off = np.array([0, e - s])
+    lp = wl.layers[0]
+    kw = dict(num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, max_pos_dist=wl.max_pos_dist,
+              num_time_buckets=wl.num_time_buckets, alpha=wl.alpha, mask=wl.mask,
+              num_candidates=wl.num_candidates)
+
+    def step():
+        O.layer_forward(wl.x[s:e], lp.w1, lp.w2, off, wl.timestamps[s:e], lp.rab_pos,
+                        lp.rab_time, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = (e - s) * args.steps / el
+    cores = len(os.sched_getaffinity(0))
+    sample = f"one fp64 oracle layer over sequence {b} ({e - s} tokens, the shortest) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "seed": args.seed},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from hstu_sequential_transducer_jagged_b200 import binding as Bd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    lib = Bd.lib()
+
+    # CPU oracle baseline first (rank 0, one GPU), before any other GPU work
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl0 = W.make(WORKLOAD, seed=args.seed)
+        v, sample, cores = oracle_layer_sample(wl0)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        del wl0
+
+    wl = W.make(WORKLOAD, seed=args.seed + rank)
+    T, L = wl.total_tokens, len(wl.layers)
+    bf = torch.bfloat16
+    x = torch.from_numpy(wl.x).to(bf).to(dev)
+    off = torch.from_numpy(wl.seq_offsets).to(dev)
+    ts = torch.from_numpy(wl.timestamps).to(dev)
+    layers = []
+    for lp in wl.layers:
+        layers.append(dict(w1=torch.from_numpy(lp.w1).to(bf).to(dev),
+                           w2=torch.from_numpy(lp.w2).to(bf).to(dev),
+                           rp=torch.from_numpy(lp.rab_pos).to(dev),
+                           rt=torch.from_numpy(lp.rab_time).to(dev)))
+    bufs = [torch.empty_like(x), torch.empty_like(x)]
+    descs = [Bd.layer_desc(seq_offsets=off, total_tokens=T, max_seq_len=wl.max_seq_len,
+                           timestamps=ts, d_model=wl.d_model, num_heads=wl.num_heads,
+                           d_qk=wl.d_qk, d_v=wl.d_v, mask=wl.mask,
+                           num_candidates=wl.num_candidates, microbatch=wl.microbatch or 1,
+                           rab_pos=ly["rp"], max_pos_dist=wl.max_pos_dist, rab_time=ly["rt"],
+                           num_time_buckets=wl.num_time_buckets, alpha=wl.alpha,
+                           ln_eps=wl.ln_eps) for ly in layers]
+    ws_bytes = lib.hstu_layer_workspace_size(ctypes.byref(descs[0]))
+    ws = Bd.Workspace(ws_bytes, dev)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def run_stack(attn_events=None):
+        cur = x
+        for l in range(L):
+            out = bufs[l % 2]
+            ly = layers[l]
+            for stage in (1, 2, 3):
+                if attn_events is not None and stage == 2:
+                    attn_events[l][0].record(stream)
+                st = lib.hstu_layer_forward_stage(
+                    ctypes.byref(descs[l]), stage, ctypes.c_void_p(cur.data_ptr()),
+                    ctypes.c_void_p(ly["w1"].data_ptr()), None,
+                    ctypes.c_void_p(ly["w2"].data_ptr()), None,
+                    ctypes.c_void_p(out.data_ptr()), ws.ptr, ws.nbytes, sp)
+                if st != 0:
+                    raise Bd.HstuError(st, f"layer {l} stage {stage}")
+                if attn_events is not None and stage == 2:
+                    attn_events[l][1].record(stream)
+            cur = out
+        return cur
+
+    for _ in range(args.warmup):
+        run_stack()
+    torch.cuda.synchronize()
+    if ws.sync_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    K = args.steps
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    attn_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(L)] for _ in range(K)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(K):
+        flush.zero_()  # L2 flush between steps, outside the step events
+        step_ev[k][0].record(stream)
+        run_stack(attn_ev[k])
+        step_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop() if sampler is not None else None
+    status = ws.sync_status()
+    if status != 0:
+        raise RuntimeError(f"device status word {status} after the timed region")
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    attn_ms = [a.elapsed_time(b) for row in attn_ev for a, b in row]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        tok = torch.tensor([float(T)], device=dev, dtype=torch.float64)
+        dist.all_reduce(tok, op=dist.ReduceOp.SUM)
+        tokens_all = float(tok.item())
+    else:
+        tokens_all = float(T)
+    ms_per_step = total_ms / K
+    value = tokens_all * L * K / (total_ms / 1e3)
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if args.e2e_steps > 0:
+        xh = torch.from_numpy(wl.x).to(bf).pin_memory()
+        offh = torch.from_numpy(wl.seq_offsets).pin_memory()
+        tsh = torch.from_numpy(wl.timestamps).pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        xd, offd, tsd = torch.empty_like(x), torch.empty_like(off), torch.empty_like(ts)
+        e2e_ws = Bd.Workspace(ws_bytes, dev)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            offd.copy_(offh, non_blocking=True)
+            tsd.copy_(tsh, non_blocking=True)
+            cur = xd
+            for l in range(L):
+                ly = layers[l]
+                cur = Bd.layer_forward(cur, ly["w1"], ly["w2"], offd, wl.max_seq_len, tsd,
+                                       ly["rp"], ly["rt"], num_heads=wl.num_heads, d_qk=wl.d_qk,
+                                       d_v=wl.d_v, max_pos_dist=wl.max_pos_dist,
+                                       num_time_buckets=wl.num_time_buckets, alpha=wl.alpha,
+                                       mask=wl.mask, num_candidates=wl.num_candidates,
+                                       out=bufs[l % 2], ws=e2e_ws)
+            yh.copy_(cur, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = xh.numel() * xh.element_size() + offh.numel() * 4 + tsh.numel() * 8
+        d2h = yh.numel() * yh.element_size()
+        e2e = {"value": tokens_all * L * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "api": "binding.layer_forward (hstu_layer_forward) x layers, pinned host buffers"}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    aflops = attention_flops(wl)
+    attn_avg_ms = float(np.mean(attn_ms))
+    attn_tflops = aflops / (attn_avg_ms / 1e3) / 1e12
+    traffic = attn_traffic_bytes()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "tokens_per_rank": T,
+                   "layers": L, "global_batch": wl.num_seqs * world,
+                   "parallelism": f"independent batch per GPU x{world} (no collective)",
+                   "l2": "256 MB buffer written between timed steps (outside step events)"},
+        "attn_tflops": attn_tflops,
+        "attn_ms_per_layer": attn_avg_ms,
+        "stack_tflops": (L * (aflops + gemm_flops(wl))) / (ms_per_step / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel<64> (+ its work-list "
+                     "kernel, inside the same events)", "achieved": attn_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": attn_tflops / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} bf16 (burst)",
+                     "traffic": traffic,
+                     "algorithmic_flops_per_launch": aflops},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": 5 * L * K,
+        "wall_s_timed_region": wall,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

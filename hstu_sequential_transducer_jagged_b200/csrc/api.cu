@@ -1,0 +1,456 @@
+// api.cu — the C ABI declared in include/hstu.h: host-side argument checks, workspace layout,
+// TMA tensor-map encoding, and kernel dispatch on the caller's stream.  No device memory is
+// allocated here and nothing synchronises with the device except hstu_sync_status().
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/hstu.h"
+#include "common.cuh"
+
+namespace hstu {
+cudaError_t launch_attn_fwd_tc(int D, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const AttnGeom& g, __nv_bfloat16* out,
+                               int64_t ld_o, int grid, cudaStream_t stream);
+cudaError_t launch_gemm_bf16_tc(int epi, const CUtensorMap& ta, const CUtensorMap& tb, int M,
+                                int N, int K, const float* bias, const __nv_bfloat16* resid,
+                                int64_t ld_r, __nv_bfloat16* C, int64_t ldc, int* status,
+                                cudaStream_t stream);
+cudaError_t launch_build_worklist(const int32_t* offsets, int B, int T, int max_len, int mask,
+                                  int m, WorkItem* items, int32_t* count, int32_t* hist,
+                                  int max_cost, int32_t* status, cudaStream_t stream);
+cudaError_t launch_ln_gate(int dtype, const void* av, int64_t ld_av, const void* u, int64_t ld_u,
+                           const float* gamma, const float* beta, float eps, void* g,
+                           int64_t ld_g, int rows, int F, cudaStream_t stream);
+cudaError_t launch_jagged_padded(const int32_t* offsets, int B, int max_len, const void* jag,
+                                 int64_t jag_stride, void* pad, int64_t pad_stride,
+                                 int64_t row_bytes, int to_padded, int num_sms,
+                                 cudaStream_t stream);
+cudaError_t launch_time_buckets(const int64_t* dt, int n, int32_t* out, int nb,
+                                cudaStream_t stream);
+cudaError_t launch_attn_fwd_simt(int dtype, int D, const AttnGeom& g, const void* q, int64_t ld_q,
+                                 const void* k, int64_t ld_k, const void* v, int64_t ld_v,
+                                 void* o, int64_t ld_o, int grid, cudaStream_t stream);
+cudaError_t launch_gemm_simt(int dtype, int epi, const void* A, int64_t lda, const void* B,
+                             int64_t ldb, int M, int N, int K, const float* bias, const void* R,
+                             int64_t ldr, void* C, int64_t ldc, cudaStream_t stream);
+cudaError_t launch_attn_bwd_simt(int dtype, int D, const AttnGeom& g, const void* q, int64_t ld_q,
+                                 const void* k, int64_t ld_k, const void* v, int64_t ld_v,
+                                 const void* d_o, int64_t ld_do, void* dq, void* dk, void* dv,
+                                 float* d_pos, float* d_time, int grid, cudaStream_t stream);
+}  // namespace hstu
+
+using namespace hstu;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;  // status word at 0, work-item count at 4
+constexpr int kMaxSeqLen = 1 << 24;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ----------------------------------------------------------------- driver entry points
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int num_sms_current() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// 2D bf16 tensor map over a row-major [rows, cols] matrix with row stride ld (elements), box
+// {box_cols, box_rows}, 128-byte swizzle, zero fill out of bounds.
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                   uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+size_t elem_size(int dtype) { return dtype == HSTU_BF16 ? 2 : 4; }
+
+// Work-list sizes for a batch: an upper bound of the number of 128-row query tiles
+// (Σ ceil(L_b / 128) <= T / 128 + B) and of the cost histogram.
+int max_items(int T, int B) { return (T + kTileRows - 1) / kTileRows + B; }
+int max_cost(int max_len) { return (max_len + kTileRows - 1) / kTileRows + 1; }
+
+struct WsLayout {
+  size_t items, hist, total_attn;
+};
+
+WsLayout attn_layout(int T, int B, int max_len) {
+  WsLayout w;
+  w.items = kStatusBytes;
+  w.hist = w.items + align_up(sizeof(WorkItem) * static_cast<size_t>(max_items(T, B)));
+  w.total_attn = w.hist + align_up(sizeof(int32_t) * static_cast<size_t>(max_cost(max_len) + 1));
+  return w;
+}
+
+hstu_status_t check_common(int B, int T, int max_len, const int32_t* offsets, int H, int dqk,
+                           int dv, int mask, int m, int mb, const float* rab_pos, int P,
+                           const float* rab_time, int NB, float alpha, int dtype) {
+  if (B < 0 || T < 0 || max_len < 0 || max_len > kMaxSeqLen) return HSTU_ERR_INVALID_ARG;
+  if (B > 0 && offsets == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (H < 1 || dqk < 1 || dv < 1) return HSTU_ERR_INVALID_ARG;
+  if (mask != HSTU_MASK_CAUSAL && mask != HSTU_MASK_MFALCON) return HSTU_ERR_INVALID_ARG;
+  if (mask == HSTU_MASK_MFALCON && (m < 0 || mb < 1)) return HSTU_ERR_INVALID_ARG;
+  if (rab_pos != nullptr && P < 0) return HSTU_ERR_INVALID_ARG;
+  if (rab_time != nullptr && NB < 1) return HSTU_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return HSTU_ERR_INVALID_ARG;
+  if (dtype != HSTU_BF16 && dtype != HSTU_FP32) return HSTU_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_len) * 1 > 0 && T > 0 && static_cast<int64_t>(B) * max_len < T)
+    return HSTU_ERR_INVALID_ARG;  // max_len too small to hold T tokens in B sequences
+  if (dqk != dv) return HSTU_ERR_UNSUPPORTED;
+  if (dqk != 16 && dqk != 32 && dqk != 64 && dqk != 128) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+hstu_status_t check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < need)
+    return HSTU_ERR_WORKSPACE;
+  return HSTU_OK;
+}
+
+AttnGeom make_geom(const void* ws, const WsLayout& w, const int64_t* ts, const float* rab_pos,
+                   int P, const float* rab_time, int NB, int H, int T, int mask, int m,
+                   float alpha) {
+  uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(ws));
+  AttnGeom g;
+  g.items = reinterpret_cast<const WorkItem*>(base + w.items);
+  g.item_count = reinterpret_cast<const int32_t*>(base + 4);
+  g.ts = ts;
+  g.rab_pos = rab_pos;
+  g.rab_time = rab_time;
+  g.P = P;
+  g.NB = NB;
+  g.H = H;
+  g.T = T;
+  g.mask = mask;
+  g.num_candidates = (mask == HSTU_MASK_MFALCON) ? m : 0;
+  g.alpha = alpha;
+  g.status = reinterpret_cast<int32_t*>(base);
+  return g;
+}
+
+cudaError_t build_list(const void* ws, const WsLayout& w, const int32_t* offsets, int B, int T,
+                       int max_len, int mask, int m, cudaStream_t s) {
+  uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(ws));
+  return launch_build_worklist(offsets, B, T, max_len, mask, mask == HSTU_MASK_MFALCON ? m : 0,
+                               reinterpret_cast<WorkItem*>(base + w.items),
+                               reinterpret_cast<int32_t*>(base + 4),
+                               reinterpret_cast<int32_t*>(base + w.hist), max_cost(max_len),
+                               reinterpret_cast<int32_t*>(base), s);
+}
+
+// Attention forward on a ready work list.
+hstu_status_t attn_forward_core(const AttnGeom& g, int B, int T, int D, int dtype, const void* q,
+                                int64_t ld_q, const void* k, int64_t ld_k, const void* v,
+                                int64_t ld_v, void* o, int64_t ld_o, cudaStream_t s) {
+  const int grid = max_items(T, B) * g.H;
+  const bool tc = dtype == HSTU_BF16 && (D == 64 || D == 128) && aligned16(q) && aligned16(k) &&
+                  aligned16(v) && aligned16(o) && (ld_q % 8 == 0) && (ld_k % 8 == 0) &&
+                  (ld_v % 8 == 0) && (ld_o % 8 == 0);
+  cudaError_t e;
+  if (tc) {
+    CUtensorMap tq, tk, tv;
+    const int64_t cols = static_cast<int64_t>(g.H) * D;
+    if (!make_map_bf16(&tq, q, T, cols, ld_q, 64, kTileRows) ||
+        !make_map_bf16(&tk, k, T, cols, ld_k, 64, kTileRows) ||
+        !make_map_bf16(&tv, v, T, cols, ld_v, 64, kTileRows))
+      return HSTU_ERR_CUDA;
+    e = launch_attn_fwd_tc(D, tq, tk, tv, g, static_cast<__nv_bfloat16*>(o), ld_o, grid, s);
+  } else {
+    e = launch_attn_fwd_simt(dtype, D, g, q, ld_q, k, ld_k, v, ld_v, o, ld_o, grid, s);
+  }
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// C = epi(A[M,K] B[K,N] + bias) on tensor cores when the shapes allow, else on CUDA cores.
+hstu_status_t gemm(int dtype, int epi, const void* A, int64_t lda, const void* Bm, int64_t ldb,
+                   int M, int N, int K, const float* bias, const void* R, int64_t ldr, void* C,
+                   int64_t ldc, int32_t* status, cudaStream_t s) {
+  const bool tc = dtype == HSTU_BF16 && K % 8 == 0 && N % 8 == 0 && lda % 8 == 0 &&
+                  ldb % 8 == 0 && ldc % 8 == 0 && (R == nullptr || ldr % 8 == 0) &&
+                  aligned16(A) && aligned16(Bm) && aligned16(C) && (R == nullptr || aligned16(R));
+  cudaError_t e;
+  if (tc) {
+    CUtensorMap ta, tb;
+    if (!make_map_bf16(&ta, A, M, K, lda, 64, 128) || !make_map_bf16(&tb, Bm, K, N, ldb, 64, 64))
+      return HSTU_ERR_CUDA;
+    e = launch_gemm_bf16_tc(epi, ta, tb, M, N, K, bias, static_cast<const __nv_bfloat16*>(R), ldr,
+                            static_cast<__nv_bfloat16*>(C), ldc, status, s);
+  } else {
+    e = launch_gemm_simt(dtype, epi, A, lda, Bm, ldb, M, N, K, bias, R, ldr, C, ldc, s);
+  }
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hstu_attention_workspace_size(const hstu_attn_desc_t* d) {
+  if (d == nullptr || d->total_tokens < 0 || d->num_seqs < 0 || d->max_seq_len < 0) return 0;
+  return attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len).total_attn;
+}
+
+size_t hstu_attention_backward_workspace_size(const hstu_attn_desc_t* d) {
+  return hstu_attention_workspace_size(d);
+}
+
+hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* d, const void* q, const void* k,
+                                     const void* v, void* o, void* ws, size_t ws_bytes,
+                                     hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
+                                  d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
+                                  d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
+                                  d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
+  if (st != HSTU_OK) return st;
+  const int D = d->d_qk;
+  const int64_t cols = static_cast<int64_t>(d->num_heads) * D;
+  if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
+    return HSTU_ERR_INVALID_ARG;
+  const WsLayout w = attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len);
+  st = check_ws(ws, ws_bytes, w.total_attn);
+  if (st != HSTU_OK) return st;
+  if (d->num_seqs == 0 || d->total_tokens == 0) return HSTU_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (build_list(ws, w, d->seq_offsets, d->num_seqs, d->total_tokens, d->max_seq_len, d->mask,
+                 d->num_candidates, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                               d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
+                               d->num_candidates, d->alpha);
+  return attn_forward_core(g, d->num_seqs, d->total_tokens, D, d->dtype, q, d->ld_q, k, d->ld_k,
+                           v, d->ld_v, o, d->ld_o, s);
+}
+
+hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, const void* k,
+                                      const void* v, const void* d_o, void* dq, void* dk,
+                                      void* dv, float* d_rab_pos, float* d_rab_time, void* ws,
+                                      size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
+                                  d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
+                                  d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
+                                  d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
+  if (st != HSTU_OK) return st;
+  const int D = d->d_qk;
+  const int64_t cols = static_cast<int64_t>(d->num_heads) * D;
+  if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
+    return HSTU_ERR_INVALID_ARG;
+  if (d->rab_pos != nullptr && d_rab_pos == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (d->rab_time != nullptr && d->timestamps != nullptr && d_rab_time == nullptr)
+    return HSTU_ERR_INVALID_ARG;
+  if (d->rab_pos != nullptr && 2 * static_cast<int64_t>(d->max_pos_dist) + 1 + d->num_time_buckets > 50000)
+    return HSTU_ERR_UNSUPPORTED;  // the per-CTA bias-gradient bins live in shared memory
+  const WsLayout w = attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len);
+  st = check_ws(ws, ws_bytes, w.total_attn);
+  if (st != HSTU_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d_rab_pos != nullptr && d->rab_pos != nullptr &&
+      cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * d->max_pos_dist + 1), s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (d_rab_time != nullptr && d->rab_time != nullptr &&
+      cudaMemsetAsync(d_rab_time, 0, sizeof(float) * d->num_time_buckets, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (d->num_seqs == 0 || d->total_tokens == 0) return HSTU_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || d_o == nullptr || dq == nullptr ||
+      dk == nullptr || dv == nullptr)
+    return HSTU_ERR_INVALID_ARG;
+  if (build_list(ws, w, d->seq_offsets, d->num_seqs, d->total_tokens, d->max_seq_len, d->mask,
+                 d->num_candidates, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                               d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
+                               d->num_candidates, d->alpha);
+  const int grid = max_items(d->total_tokens, d->num_seqs) * d->num_heads;
+  cudaError_t e = launch_attn_bwd_simt(d->dtype, D, g, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o,
+                                       d->ld_o, dq, dk, dv, d_rab_pos, d_rab_time, grid, s);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+size_t hstu_layer_workspace_size(const hstu_layer_desc_t* d) {
+  if (d == nullptr || d->total_tokens < 0 || d->num_seqs < 0 || d->max_seq_len < 0 ||
+      d->num_heads < 1 || d->d_qk < 1 || d->d_v < 1)
+    return 0;
+  const WsLayout w = attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len);
+  const size_t es = elem_size(d->dtype);
+  const size_t T = static_cast<size_t>(d->total_tokens);
+  const size_t n1 = 2 * static_cast<size_t>(d->num_heads) * (d->d_qk + d->d_v);
+  const size_t hv = static_cast<size_t>(d->num_heads) * d->d_v;
+  return w.total_attn + align_up(T * n1 * es) + 2 * align_up(T * hv * es);
+}
+
+hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* d, int32_t stage,
+                                       const void* x, const void* w1, const float* b1,
+                                       const void* w2, const float* b2, void* y, void* ws,
+                                       size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (stage < HSTU_STAGE_F1 || stage > HSTU_STAGE_NORM_GATE_F2) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
+                                  d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
+                                  d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
+                                  d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
+  if (st != HSTU_OK) return st;
+  if (d->d_model < 1 || !std::isfinite(d->ln_eps) || d->ln_eps < 0.f) return HSTU_ERR_INVALID_ARG;
+  const int H = d->num_heads, D = d->d_qk, T = d->total_tokens;
+  const int hv = H * d->d_v;
+  const int n1 = 2 * H * (d->d_qk + d->d_v);
+  if (hv > 1024) return HSTU_ERR_UNSUPPORTED;  // LayerNorm row held in one warp's registers
+  const size_t need = hstu_layer_workspace_size(d);
+  st = check_ws(ws, ws_bytes, need);
+  if (st != HSTU_OK) return st;
+  if (d->num_seqs == 0 || T == 0) return HSTU_OK;
+  if (stage == HSTU_STAGE_F1 && (x == nullptr || w1 == nullptr || !aligned16(x) || !aligned16(w1)))
+    return HSTU_ERR_INVALID_ARG;
+  if (stage == HSTU_STAGE_NORM_GATE_F2 &&
+      (x == nullptr || w2 == nullptr || y == nullptr || x == y || !aligned16(x) ||
+       !aligned16(w2) || !aligned16(y)))
+    return HSTU_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout w = attn_layout(T, d->num_seqs, d->max_seq_len);
+  const size_t es = elem_size(d->dtype);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* uvqk = base + w.total_attn;
+  uint8_t* av = uvqk + align_up(static_cast<size_t>(T) * n1 * es);
+  uint8_t* gbuf = av + align_up(static_cast<size_t>(T) * hv * es);
+  int32_t* status = reinterpret_cast<int32_t*>(base);
+  const uint8_t* u_ptr = uvqk;
+  const uint8_t* v_ptr = uvqk + static_cast<size_t>(hv) * es;
+  const uint8_t* q_ptr = uvqk + static_cast<size_t>(2 * hv) * es;
+  const uint8_t* k_ptr = q_ptr + static_cast<size_t>(H) * d->d_qk * es;
+
+  if (stage == HSTU_STAGE_F1) {
+    // f1 + SiLU: [T, d_model] x [d_model, n1] -> uvqk = [U | V | Q | K]
+    return gemm(d->dtype, 0, x, d->d_model, w1, n1, T, n1, d->d_model, b1, nullptr, 0, uvqk, n1,
+                status, s);
+  }
+  if (stage == HSTU_STAGE_ATTENTION) {
+    if (build_list(ws, w, d->seq_offsets, d->num_seqs, T, d->max_seq_len, d->mask,
+                   d->num_candidates, s) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+    const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                                 d->num_time_buckets, H, T, d->mask, d->num_candidates, d->alpha);
+    return attn_forward_core(g, d->num_seqs, T, D, d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av,
+                             hv, s);
+  }
+  // Norm(AV) ⊙ U, then f2 + residual: Y = X + G W2 + b2
+  if (launch_ln_gate(d->dtype == HSTU_BF16 ? 0 : 1, av, hv, u_ptr, n1, d->ln_gamma, d->ln_beta,
+                     d->ln_eps, gbuf, hv, T, hv, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  return gemm(d->dtype, 1, gbuf, hv, w2, d->d_model, T, d->d_model, hv, b2, x, d->d_model, y,
+              d->d_model, status, s);
+}
+
+hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* d, const void* x, const void* w1,
+                                 const float* b1, const void* w2, const float* b2, void* y,
+                                 void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (x == nullptr || w1 == nullptr || w2 == nullptr || y == nullptr || x == y)
+    return d->num_seqs == 0 || d->total_tokens == 0 ? HSTU_OK : HSTU_ERR_INVALID_ARG;
+  for (int32_t stage = HSTU_STAGE_F1; stage <= HSTU_STAGE_NORM_GATE_F2; ++stage) {
+    const hstu_status_t st =
+        hstu_layer_forward_stage(d, stage, x, w1, b1, w2, b2, y, ws, ws_bytes, stream);
+    if (st != HSTU_OK) return st;
+  }
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_seqs,
+                                      int32_t max_len, const void* jagged,
+                                      int64_t jagged_row_stride_bytes, void* padded,
+                                      int64_t padded_row_stride_bytes, int64_t row_bytes,
+                                      int32_t to_padded, hstu_stream_t stream) {
+  if (num_seqs < 0 || max_len < 0 || row_bytes < 0) return HSTU_ERR_INVALID_ARG;
+  if (num_seqs == 0 || max_len == 0 || row_bytes == 0) return HSTU_OK;
+  if (seq_offsets == nullptr || jagged == nullptr || padded == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (row_bytes % 16 != 0 || jagged_row_stride_bytes % 16 != 0 ||
+      padded_row_stride_bytes % 16 != 0 || !aligned16(jagged) || !aligned16(padded) ||
+      jagged_row_stride_bytes < row_bytes || padded_row_stride_bytes < row_bytes)
+    return HSTU_ERR_INVALID_ARG;
+  cudaError_t e = launch_jagged_padded(seq_offsets, num_seqs, max_len, jagged,
+                                       jagged_row_stride_bytes, padded, padded_row_stride_bytes,
+                                       row_bytes, to_padded, num_sms_current(),
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out, int32_t nb,
+                                      hstu_stream_t stream) {
+  if (n < 0 || nb < 1) return HSTU_ERR_INVALID_ARG;
+  if (n == 0) return HSTU_OK;
+  if (dt == nullptr || out == nullptr) return HSTU_ERR_INVALID_ARG;
+  cudaError_t e = launch_time_buckets(dt, n, out, nb, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_workspace_init(void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (check_ws(ws, ws_bytes, kStatusBytes) != HSTU_OK) return HSTU_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, kStatusBytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? HSTU_OK
+             : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_sync_status(const void* ws, hstu_stream_t stream) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return HSTU_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (word != 0 && cudaMemset(const_cast<void*>(ws), 0, sizeof(word)) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (word == 0) return HSTU_OK;
+  if (word == HSTU_ERR_TIMEOUT) return HSTU_ERR_TIMEOUT;
+  return HSTU_ERR_DEVICE_CHECK;
+}
+
+const char* hstu_status_string(hstu_status_t s) {
+  switch (s) {
+    case HSTU_OK: return "ok";
+    case HSTU_ERR_INVALID_ARG: return "invalid argument";
+    case HSTU_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HSTU_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case HSTU_ERR_CUDA: return "CUDA error";
+    case HSTU_ERR_TIMEOUT: return "device wait timed out";
+    case HSTU_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* hstu_version(void) { return "hstu_b200 0.1 sm_100a"; }
+
+}  // extern "C"

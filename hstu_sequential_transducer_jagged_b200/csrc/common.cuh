@@ -1,0 +1,69 @@
+// common.cuh — types shared by the kernels and the C-ABI layer.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hstu {
+
+// Query rows of one attention tile, and key/value rows of one KV tile.
+constexpr int kTileRows = 128;
+
+// One unit of attention work: a 128-row query tile of one sequence (all heads share the list).
+// len = sequence length, row0 = first token of the sequence, qtile = tile index within it,
+// cost = number of KV tiles the tile visits (used only for the longest-first ordering).
+struct WorkItem {
+  int32_t seq;
+  int32_t qtile;
+  int32_t row0;
+  int32_t len;
+};
+
+// Geometry of the jagged problem and bias parameters, passed by value to the kernels.
+struct AttnGeom {
+  const WorkItem* items;
+  const int32_t* item_count;
+  const int64_t* ts;        // [T] or nullptr
+  const float* rab_pos;     // [2P+1] or nullptr
+  const float* rab_time;    // [NB] or nullptr
+  int32_t P;
+  int32_t NB;
+  int32_t H;
+  int32_t T;
+  int32_t mask;             // 0 causal, 1 M-FALCON
+  int32_t num_candidates;
+  float alpha;
+  int32_t* status;
+};
+
+// History length n of a sequence: every token for the causal mask, L - m under M-FALCON.
+__host__ __device__ __forceinline__ int hist_len(int L, int mask, int m) {
+  if (mask == 1) {
+    int n = L - m;
+    return n < 0 ? 0 : n;
+  }
+  return L;
+}
+
+// KV tiles a query tile visits: tiles 0 .. nh-1 cover every key j < min(qe, n) (the visible
+// history), plus the query tile's own diagonal tile when it holds candidates that only see
+// themselves beyond the history.  Causal: nh = qtile + 1 and no extra tile.
+struct KvRange {
+  int nh;
+  int diag;  // 1 if the diagonal tile is visited after the nh history tiles
+  __device__ __forceinline__ int count() const { return nh + diag; }
+  __device__ __forceinline__ int tile(int t, int qtile) const { return t < nh ? t : qtile; }
+};
+
+__device__ __forceinline__ KvRange kv_range(int qtile, int L, int n) {
+  const int qs = qtile * kTileRows;
+  const int qe = min(qs + kTileRows, L);
+  const int hv = min(qe, n);
+  KvRange r;
+  r.nh = (hv + kTileRows - 1) / kTileRows;
+  r.diag = (qe > n && qtile >= r.nh) ? 1 : 0;
+  return r;
+}
+
+}  // namespace hstu

@@ -1,0 +1,201 @@
+/*
+ * hstu.h — C ABI of the B200 (sm_100a) HSTU jagged layer library (libhstu_b200.so).
+ *
+ * What the library computes (web pages on HSTU, cited by title and section):
+ *   [Review §2.1]  "万亿参数推荐大模型：HSTU 架构如何超越传统 Self-Attention", §2.1, the three formulas
+ *                  U,V,Q,K = Split(φ1(f1(X)));  A(X)V(X) = φ2(Q Kᵀ + rab_{p,t}) V;
+ *                  Y = f2(Norm(A(X)V(X)) ⊙ U(X)), φ1 = φ2 = SiLU, f1/f2 single linear layers,
+ *                  and the block diagram's residual edge from the input X to the output Y.
+ *   [FunRec 7.1]   "HSTU：Scaling Law 的首次探索", §7.1.4 innovation 1 (pointwise SiLU aggregation,
+ *                  no softmax normalisation), innovation 2 (relative bias from position and time
+ *                  differences), §7.1.5 M-FALCON (candidates see the whole history but not each
+ *                  other; microbatches of b_m candidates; history K/V reused).
+ *   [GenRank 6.2]  "6.2 HSTU的工程突破", §6.2.2 (the same candidate mask), §6.2.3 Eq. (6.2.3)
+ *                  (relative-bias score; its backward needs the N×N bias gradient).
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   rab_{p,t}(i,j) = rab_pos[clamp(p_i - p_j, -P, P) + P] + rab_time[bucket(t_i - t_j)],
+ *   bucket(dt) = clamp(floor(log2(max(1, dt))), 0, NB-1) on int64 (bit-exact), one pair of
+ *   tables shared by all heads; score = alpha * <q_i, k_j> + rab (alpha = 1 is the literal
+ *   formula); causal mask j <= i; M-FALCON candidates (the last m tokens of each sequence)
+ *   all take the position index n = L - m; Norm = LayerNorm over the H*d_v features of a
+ *   token, biased variance; split order [U | V | Q | K], head-major within each block.
+ *
+ * Conventions shared by every entry point:
+ *   - Jagged batch: B sequences packed back to back; seq_offsets is int32 [B+1] on the device,
+ *     seq_offsets[0] = 0, non-decreasing, seq_offsets[B] = T.  total_tokens (T) and max_seq_len
+ *     are host copies, so no call synchronises with the device.  The device re-checks the
+ *     offsets; a violation sets the status word (HSTU_ERR_DEVICE_CHECK) and the kernels skip
+ *     all work.
+ *   - Ownership: the caller allocates and owns every buffer.  The library allocates no device
+ *     memory, keeps no global state apart from a per-device cache of driver entry points, and
+ *     launches everything on the caller's stream (asynchronous; reentrant per stream).
+ *   - Workspace: *_workspace_size() gives the bytes a call needs; ws must be 256-byte aligned.
+ *     Its first 256 bytes hold the device status word, which kernels set on a device-side
+ *     check failure or a bounded-wait timeout; hstu_sync_status() reports and clears it.
+ *     A new workspace is zeroed once with hstu_workspace_init() before its first use.
+ *   - Errors: argument errors are found on the host before any launch and returned; a failed
+ *     launch returns HSTU_ERR_CUDA.  No entry point aborts the process or traps the GPU.
+ *   - Device pointers must be 16-byte aligned and row strides (in elements) such that a row
+ *     starts on a 16-byte boundary; otherwise HSTU_ERR_INVALID_ARG.
+ *   - Outputs are written, never accumulated into (d_rab_* included).
+ */
+#ifndef HSTU_B200_H_
+#define HSTU_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hstu_stream_t; /* a cudaStream_t; NULL = the legacy default stream */
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,   /* a host-side argument check failed; nothing was launched */
+  HSTU_ERR_UNSUPPORTED = 2,   /* a valid combination this build does not implement */
+  HSTU_ERR_WORKSPACE = 3,     /* ws is NULL, misaligned or smaller than *_workspace_size() */
+  HSTU_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
+  HSTU_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (reported via the status word) */
+  HSTU_ERR_DEVICE_CHECK = 6   /* a device-side check failed, e.g. malformed seq_offsets */
+} hstu_status_t;
+
+typedef enum { HSTU_MASK_CAUSAL = 0, HSTU_MASK_MFALCON = 1 } hstu_mask_t;
+typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1 } hstu_dtype_t;
+
+/* Attention problem over a jagged batch ([Review §2.1] second formula; [FunRec 7.1] §7.1.4-5).
+ * Q, K: [T, num_heads * d_qk], V, O: [T, num_heads * d_v], row-major with row strides ld_*
+ * (elements), so Q/K/V may be column views of one f1 output.  Head h occupies columns
+ * [h*d, (h+1)*d) of its operand. */
+typedef struct {
+  int32_t num_seqs;           /* B >= 0 */
+  int32_t total_tokens;       /* T = seq_offsets[B] (host copy) */
+  int32_t max_seq_len;        /* upper bound of every sequence length (host copy) */
+  const int32_t* seq_offsets; /* device int32 [B+1] */
+  const int64_t* timestamps;  /* device int64 [T] (seconds); NULL disables the time bias */
+  int32_t num_heads;          /* H >= 1 */
+  int32_t d_qk;               /* per-head query/key width */
+  int32_t d_v;                /* per-head value width */
+  int64_t ld_q, ld_k, ld_v, ld_o;  /* row strides in elements */
+  int32_t mask;               /* hstu_mask_t */
+  int32_t num_candidates;     /* M-FALCON: the last m tokens of every sequence are candidates */
+  int32_t mfalcon_microbatch; /* b_m >= 1 (M-FALCON only); the output does not depend on it */
+  const float* rab_pos;       /* device fp32 [2P+1]; NULL disables the position bias */
+  int32_t max_pos_dist;       /* P >= 0 */
+  const float* rab_time;      /* device fp32 [NB]; NULL disables the time bias */
+  int32_t num_time_buckets;   /* NB >= 1 */
+  float alpha;                /* scale of <q, k>; 1.0 is the literal formula */
+  int32_t dtype;              /* hstu_dtype_t of Q/K/V/O (fp32 accumulation either way) */
+} hstu_attn_desc_t;
+
+/* Bytes of workspace hstu_attention_forward needs (status word + tile work list). */
+size_t hstu_attention_workspace_size(const hstu_attn_desc_t* desc);
+
+/* O_i = Σ_{j visible from i} SiLU(alpha <Q_i, K_j> + rab_{p,t}(i, j)) V_j per head: the
+ * pointwise aggregated attention of [Review §2.1] and [FunRec 7.1] §7.1.4 innovation 1, with
+ * the causal mask, or the M-FALCON mask of [FunRec 7.1] §7.1.5 / [GenRank 6.2] §6.2.2.
+ * q, k, v, o: device pointers of desc->dtype.  Rows of o outside every sequence are not
+ * written.  Runs entirely on the stream; no synchronisation. */
+hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* desc, const void* q,
+                                     const void* k, const void* v, void* o, void* ws,
+                                     size_t ws_bytes, hstu_stream_t stream);
+
+/* Bytes of workspace hstu_attention_backward needs (adds an fp32 dQ accumulator [T,H,d_qk]). */
+size_t hstu_attention_backward_workspace_size(const hstu_attn_desc_t* desc);
+
+/* Gradients of Σ dO ⊙ O through hstu_attention_forward ([GenRank 6.2] §6.2.3: the backward of
+ * the N×N relative bias).  With S = alpha QKᵀ + rab and A = SiLU(S) on visible pairs:
+ *   dV = Aᵀ dO, dS = (dO Vᵀ) ⊙ SiLU'(S), dQ = alpha dS K, dK = alpha dSᵀ Q,
+ *   d_rab_pos[k] = Σ dS over visible pairs with position index k (all heads and sequences),
+ *   d_rab_time[b] = Σ dS over visible pairs with time bucket b.
+ * d_o uses ld_o; dq/dk/dv use ld_q/ld_k/ld_v.  d_rab_pos / d_rab_time (fp32 [2P+1] / [NB])
+ * are overwritten; either may be NULL when the matching table is NULL. */
+hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* desc, const void* q,
+                                      const void* k, const void* v, const void* d_o, void* dq,
+                                      void* dk, void* dv, float* d_rab_pos, float* d_rab_time,
+                                      void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* One HSTU layer over a jagged batch ([Review §2.1], all three formulas + residual edge). */
+typedef struct {
+  int32_t num_seqs, total_tokens, max_seq_len;
+  const int32_t* seq_offsets;  /* device int32 [B+1] */
+  const int64_t* timestamps;   /* device int64 [T]; NULL disables the time bias */
+  int32_t d_model;
+  int32_t num_heads, d_qk, d_v;
+  int32_t mask, num_candidates, mfalcon_microbatch;
+  const float* rab_pos;  int32_t max_pos_dist;
+  const float* rab_time; int32_t num_time_buckets;
+  float alpha;
+  float ln_eps;                /* LayerNorm epsilon (1e-5 in every workload here) */
+  const float* ln_gamma;       /* fp32 [H*d_v] or NULL (= 1) */
+  const float* ln_beta;        /* fp32 [H*d_v] or NULL (= 0) */
+  int32_t dtype;               /* hstu_dtype_t of x, w1, w2, y */
+} hstu_layer_desc_t;
+
+/* Bytes of workspace hstu_layer_forward needs: status + work list + the f1 output
+ * [T, 2H(d_qk+d_v)], the attention output [T, H d_v] and the gated norm [T, H d_v]. */
+size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc);
+
+/* Y = X + f2(Norm(A(X)V(X)) ⊙ U(X)) with U,V,Q,K = Split(SiLU(X W1 + b1)) and f2(g) = g W2 + b2.
+ * x, y: [T, d_model] row-major (y may not alias x); w1: [d_model, 2H(d_qk+d_v)] row-major;
+ * w2: [H d_v, d_model] row-major; b1 / b2: device fp32 [2H(d_qk+d_v)] / [d_model] or NULL.
+ * Three kernel stages on the stream: f1 GEMM + SiLU, attention, LayerNorm⊙U, f2 GEMM +
+ * residual. */
+hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* desc, const void* x, const void* w1,
+                                 const float* b1, const void* w2, const float* b2, void* y,
+                                 void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Stages of hstu_layer_forward, callable one at a time (e.g. to time each kernel).  The
+ * intermediates live in ws at fixed offsets, so the stages must run in order on one workspace:
+ *   HSTU_STAGE_F1           uvqk = SiLU(x W1 + b1)                       (tensor-core GEMM)
+ *   HSTU_STAGE_ATTENTION    av = attention over the Q/K/V views of uvqk  (work list + kernel)
+ *   HSTU_STAGE_NORM_GATE_F2 g = Norm(av) ⊙ U;  y = x + g W2 + b2        (two kernels)
+ * Arguments a stage does not read may be NULL. */
+typedef enum {
+  HSTU_STAGE_F1 = 1,
+  HSTU_STAGE_ATTENTION = 2,
+  HSTU_STAGE_NORM_GATE_F2 = 3
+} hstu_layer_stage_t;
+
+hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* desc, int32_t stage,
+                                       const void* x, const void* w1, const float* b1,
+                                       const void* w2, const float* b2, void* y, void* ws,
+                                       size_t ws_bytes, hstu_stream_t stream);
+
+/* Copy rows between the jagged layout and a padded [B, max_len] layout (row_bytes per row,
+ * 16-byte aligned pointers, strides and row_bytes).  to_padded != 0: jagged -> padded, rows
+ * past a sequence's end are zero-filled; to_padded == 0: padded -> jagged.  Sequences longer
+ * than max_len are truncated (their status is not an error). */
+hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_seqs,
+                                      int32_t max_len, const void* jagged,
+                                      int64_t jagged_row_stride_bytes, void* padded,
+                                      int64_t padded_row_stride_bytes, int64_t row_bytes,
+                                      int32_t to_padded, hstu_stream_t stream);
+
+/* Debug export of the time-bias bucket rule: out[i] = clamp(floor(log2(max(1, dt[i]))), 0,
+ * nb-1), computed on the device by the same code the attention kernels inline, so it can be
+ * compared bit-exactly with an integer reference.  dt, out: device [n]. */
+hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out, int32_t nb,
+                                      hstu_stream_t stream);
+
+/* Zero the status word at the start of ws (asynchronously, on the stream).  Call once on a new
+ * workspace before its first use: the status word must start at zero. */
+hstu_status_t hstu_workspace_init(void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Synchronise the stream, read the status word kept in ws (a workspace previously passed to
+ * a compute call), clear it, and return it (HSTU_OK if no device-side check fired). */
+hstu_status_t hstu_sync_status(const void* ws, hstu_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* hstu_status_string(hstu_status_t status);
+
+/* Library version string, e.g. "hstu_b200 0.1 sm_100a". */
+const char* hstu_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_B200_H_ */

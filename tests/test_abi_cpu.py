@@ -1,0 +1,141 @@
+"""The C-ABI library loads, exports every symbol include/hstu.h declares, and rejects bad
+arguments on the host before touching the GPU (these tests need no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hstu_sequential_transducer_jagged_b200 import binding as B
+from hstu_sequential_transducer_jagged_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hstu.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(hstu_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_and_binding_agree():
+    assert set(_declared_functions()) == set(B.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.hstu_version().decode().startswith("hstu_b200")
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.hstu_status_string(code)
+    assert lib.hstu_status_string(99) == b"unknown status"
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: argument checks fail before any launch
+
+
+def _desc(**kw):
+    base = dict(num_seqs=2, total_tokens=100, max_seq_len=64, seq_offsets=1 << 20,
+                timestamps=None, num_heads=2, d_qk=64, d_v=64, ld_q=128, ld_k=128, ld_v=128,
+                ld_o=128, mask=0, num_candidates=0, mfalcon_microbatch=1, rab_pos=None,
+                max_pos_dist=0, rab_time=None, num_time_buckets=1, alpha=1.0, dtype=0)
+    base.update(kw)
+    return B.AttnDesc(**base)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(num_seqs=-1), dict(total_tokens=-5), dict(num_heads=0), dict(d_qk=0),
+    dict(mask=7), dict(mask=1, num_candidates=-1), dict(mask=1, mfalcon_microbatch=0),
+    dict(alpha=float("nan")), dict(dtype=5), dict(ld_q=64), dict(seq_offsets=None),
+    dict(max_seq_len=10),  # 2 sequences of <= 10 tokens cannot hold 100 tokens
+])
+def test_attention_forward_rejects_bad_arguments(lib, bad):
+    d = _desc(**bad)
+    st = lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == 1
+
+
+@pytest.mark.parametrize("bad", [dict(d_qk=48, d_v=48), dict(d_qk=64, d_v=32)])
+def test_attention_forward_unsupported_widths(lib, bad):
+    d = _desc(**bad)
+    st = lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == 2
+
+
+def test_attention_workspace_checks(lib):
+    d = _desc()
+    need = lib.hstu_attention_workspace_size(ctypes.byref(d))
+    assert need >= 256 and need % 256 == 0
+    # too small, misaligned, missing
+    assert lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, need - 1,
+                                      None) == 3
+    assert lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE,
+                                      ctypes.c_void_p((1 << 20) + 16), need, None) == 3
+    assert lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, None, need,
+                                      None) == 3
+    assert lib.hstu_attention_forward(None, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 1
+
+
+def test_workspace_size_grows_with_batch(lib):
+    small = lib.hstu_attention_workspace_size(ctypes.byref(_desc()))
+    big = lib.hstu_attention_workspace_size(ctypes.byref(_desc(num_seqs=64, total_tokens=81920,
+                                                               max_seq_len=2048)))
+    assert big > small
+
+
+def _ldesc(**kw):
+    base = dict(num_seqs=2, total_tokens=100, max_seq_len=64, seq_offsets=1 << 20,
+                timestamps=None, d_model=64, num_heads=2, d_qk=32, d_v=32, mask=0,
+                num_candidates=0, mfalcon_microbatch=1, rab_pos=None, max_pos_dist=0,
+                rab_time=None, num_time_buckets=1, alpha=1.0, ln_eps=1e-5, ln_gamma=None,
+                ln_beta=None, dtype=1)
+    base.update(kw)
+    return B.LayerDesc(**base)
+
+
+def test_layer_rejects_bad_arguments(lib):
+    d = _ldesc()
+    need = lib.hstu_layer_workspace_size(ctypes.byref(d))
+    # layer workspace holds f1 output + AV + G in fp32
+    assert need >= 100 * (2 * 2 * 64 + 2 * 64) * 4
+    ok_ws = ctypes.c_void_p(1 << 20)
+    assert lib.hstu_layer_forward(ctypes.byref(_ldesc(d_model=0)), FAKE, FAKE, None, FAKE, None,
+                                  ctypes.c_void_p(2 << 20), ok_ws, need, None) == 1
+    assert lib.hstu_layer_forward(ctypes.byref(_ldesc(ln_eps=-1.0)), FAKE, FAKE, None, FAKE,
+                                  None, ctypes.c_void_p(2 << 20), ok_ws, need, None) == 1
+    # y aliasing x
+    assert lib.hstu_layer_forward(ctypes.byref(d), FAKE, FAKE, None, FAKE, None, FAKE, ok_ws,
+                                  need, None) == 1
+    # H * d_v beyond the LayerNorm row limit
+    big = _ldesc(num_heads=16, d_qk=128, d_v=128)
+    assert lib.hstu_layer_forward(ctypes.byref(big), FAKE, FAKE, None, FAKE, None,
+                                  ctypes.c_void_p(2 << 20), ok_ws, 1 << 40, None) == 2
+
+
+def test_backward_requires_grad_buffers(lib):
+    d = _desc(rab_pos=1 << 20, max_pos_dist=4)
+    st = lib.hstu_attention_backward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     None, None, FAKE, 1 << 30, None)
+    assert st == 1
+
+
+def test_misc_entry_points_validate(lib):
+    assert lib.hstu_debug_time_buckets(FAKE, -1, FAKE, 8, None) == 1
+    assert lib.hstu_debug_time_buckets(FAKE, 4, FAKE, 0, None) == 1
+    assert lib.hstu_debug_time_buckets(None, 0, None, 8, None) == 0
+    # row_bytes not a multiple of 16
+    assert lib.hstu_jagged_padded_copy(FAKE, 2, 8, FAKE, 32, FAKE, 32, 24, 1, None) == 1
+    assert lib.hstu_jagged_padded_copy(FAKE, 0, 8, FAKE, 32, FAKE, 32, 32, 1, None) == 0
+    assert lib.hstu_sync_status(ctypes.c_void_p((1 << 20) + 8), None) == 3
+    assert lib.hstu_workspace_init(None, 256, None) == 3

@@ -1,0 +1,348 @@
+"""GPU-vs-oracle parity through the C ABI (needs a B200 and the built library).
+
+Tolerance (floating point): per element |gpu - ref| <= 2e-2 * max|ref row| + 1e-3 and relative
+Frobenius error <= 5e-3 (bf16 inputs, fp32 accumulation); time buckets and jagged copies are
+compared bit-exactly.  Sizes span several 128-row tiles with ragged tails; full-size workloads are
+checked on sampled rows (or whole sampled sequences) that the oracle computes directly.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hstu_oracle as O
+from hstu_sequential_transducer_jagged_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+ROW_TOL = 2e-2
+ABS_TOL = 1e-3
+FRO_TOL = 5e-3
+
+
+@pytest.fixture(scope="module")
+def B():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from hstu_sequential_transducer_jagged_b200 import binding
+    binding.lib()  # fails loudly if the library is missing
+    return binding
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def act(case):
+    return torch.bfloat16 if case.dtype == "bf16" else torch.float32
+
+
+def assert_close(gpu, ref, what=""):
+    g = gpu.detach().float().cpu().numpy().astype(np.float64) if torch.is_tensor(gpu) else gpu
+    ref = np.asarray(ref, dtype=np.float64)
+    g = g.reshape(ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    if ref.ndim == 1:
+        bound = ROW_TOL * np.abs(ref).max(initial=0.0) + ABS_TOL
+    else:
+        bound = ROW_TOL * np.abs(ref).max(axis=-1, keepdims=True) + ABS_TOL
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements out of tolerance, max err "
+                           f"{err.max():.3e}")
+    nref = np.linalg.norm(ref)
+    if nref > 0:
+        fro = np.linalg.norm(g - ref) / nref
+        assert fro <= FRO_TOL, f"{what}: relative Frobenius error {fro:.3e}"
+
+
+def attn_kw(case):
+    return dict(num_heads=case.num_heads, d_qk=case.d_qk, d_v=case.d_v,
+                max_pos_dist=case.max_pos_dist, num_time_buckets=case.num_time_buckets,
+                alpha=case.alpha, mask=case.mask, num_candidates=case.num_candidates)
+
+
+def gpu_attention(B, case, use_time=True, use_pos=True, microbatch=None):
+    dt = act(case)
+    q, k, v = dev(case.q, dt), dev(case.k, dt), dev(case.v, dt)
+    off = dev(case.seq_offsets)
+    ts = dev(case.timestamps) if use_time else None
+    rp = dev(case.rab_pos) if use_pos else None
+    rt = dev(case.rab_time) if use_time else None
+    out = B.attention_forward(q, k, v, off, case.max_seq_len, ts, rp, rt,
+                              num_heads=case.num_heads, max_pos_dist=case.max_pos_dist,
+                              num_time_buckets=case.num_time_buckets, alpha=case.alpha,
+                              mask=case.mask, num_candidates=case.num_candidates,
+                              microbatch=microbatch or max(case.microbatch, 1))
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_attention(case, use_time=True, use_pos=True, rows=None):
+    return O.attention_forward(case.q, case.k, case.v, case.seq_offsets,
+                               case.timestamps if use_time else None,
+                               case.rab_pos if use_pos else None,
+                               case.rab_time if use_time else None, rows=rows, **attn_kw(case))
+
+
+# ------------------------------------------------------------------------ bias indices
+def test_time_buckets_bit_exact(B):
+    vals = [0, 1, -1, -(2 ** 62), 2 ** 63 - 1]
+    for k in range(1, 63):
+        vals += [2 ** k - 1, 2 ** k, 2 ** k + 1]
+    rng = np.random.default_rng(0)
+    vals += list(rng.integers(-2 ** 40, 2 ** 62, size=5000))
+    dt = np.array(vals, dtype=np.int64)
+    for nb in (1, 16, 64, 128):
+        got = B.debug_time_buckets(dev(dt), nb).cpu().numpy()
+        assert np.array_equal(got, O.time_bucket(dt, nb)), nb
+
+
+# --------------------------------------------------------------------- attention forward
+CAUSAL_LENGTHS = [1, 127, 128, 129, 0, 300, 513, 64]
+
+
+@pytest.mark.parametrize("d", [64, 128, 32])
+def test_attention_forward_causal_small(B, d):
+    case = W.random_attention_case(100 + d, CAUSAL_LENGTHS, H=2, d=d, P=40, NB=16,
+                                   gap_mean=20.0, table_std=0.5)
+    assert_close(gpu_attention(B, case), oracle_attention(case), f"causal d={d}")
+
+
+@pytest.mark.parametrize("use_time,use_pos", [(False, True), (True, False), (False, False)])
+def test_attention_forward_bias_switches(B, use_time, use_pos):
+    case = W.random_attention_case(7, [200, 77, 256], H=3, d=64, P=8, NB=12, gap_mean=5.0)
+    assert_close(gpu_attention(B, case, use_time, use_pos),
+                 oracle_attention(case, use_time, use_pos), f"time={use_time} pos={use_pos}")
+
+
+def test_attention_forward_alpha_and_wide_scores(B):
+    case = W.random_attention_case(8, [333, 129], H=2, d=64, P=100, NB=32, qkv_std=1.0)
+    case.alpha = 0.125
+    assert_close(gpu_attention(B, case), oracle_attention(case), "alpha")
+
+
+def test_attention_forward_interleaved_timestamps(B):
+    case = W.random_attention_case(9, [700, 451], H=2, d=64, P=64, NB=32, interleaved=True)
+    assert_close(gpu_attention(B, case), oracle_attention(case), "interleaved")
+
+
+def test_attention_forward_large_position_clamp(B):
+    # P beyond the shared-memory table limit takes the global-memory table path
+    case = W.random_attention_case(10, [600, 260], H=2, d=64, P=3000, NB=64)
+    assert_close(gpu_attention(B, case), oracle_attention(case), "P=3000")
+
+
+@pytest.mark.parametrize("m,lengths", [(40, [240, 190, 128, 300]), (64, [64 + 64, 5 + 64, 30]),
+                                       (200, [456, 200, 1])])
+def test_attention_forward_mfalcon(B, m, lengths):
+    case = W.random_attention_case(11 + m, lengths, H=2, d=64, P=50, NB=16, mask=W.MASK_MFALCON,
+                                   num_candidates=m, gap_mean=30.0)
+    assert_close(gpu_attention(B, case), oracle_attention(case), f"mfalcon m={m}")
+
+
+def test_attention_forward_mfalcon_microbatch_invariance(B):
+    case = W.random_attention_case(12, [300, 420], H=2, d=64, P=32, NB=16, mask=W.MASK_MFALCON,
+                                   num_candidates=150)
+    outs = [gpu_attention(B, case, microbatch=mb) for mb in (1, 64, 128, 150)]
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    ref = O.attention_forward_mfalcon_microbatched(
+        case.q, case.k, case.v, case.seq_offsets, case.timestamps, case.rab_pos, case.rab_time,
+        num_heads=2, d_qk=64, d_v=64, max_pos_dist=32, num_time_buckets=16,
+        num_candidates=150, microbatch=64)
+    assert_close(outs[0], ref, "mfalcon microbatched oracle")
+
+
+def test_attention_forward_fp32(B):
+    case = W.random_attention_case(13, [100, 17, 130], H=2, d=32, P=20, NB=16, bf16=False)
+    assert_close(gpu_attention(B, case), oracle_attention(case), "fp32")
+
+
+def test_attention_forward_full_size_sampled_rows(B):
+    """The 4-layer stack's attention shape (B=8, L~U{2048..8192}, H=8, d=64) at full size."""
+    case = W.make_attn_fwdbwd_bf16_b64(seed=3, B=8, lo=2048, hi=8192)
+    case.q = W.round_to_bf16(case.q * 0.25)
+    case.k = W.round_to_bf16(case.k * 0.25)
+    out = gpu_attention(B, case).float().cpu().numpy()
+    off = case.seq_offsets
+    rng = np.random.default_rng(5)
+    rows = []
+    for b in range(case.num_seqs):
+        s, e = int(off[b]), int(off[b + 1])
+        rows += [s, s + 127, s + 128, e - 1] + list(rng.integers(s, e, size=4))
+    rows = np.unique(np.array(rows))
+    ref = oracle_attention(case, rows=rows)
+    assert_close(out[rows], ref[rows], "full-size sampled rows")
+
+
+# -------------------------------------------------------------------------- layer forward
+def gpu_layer(B, case, layer_idx=0, x=None, out=None):
+    dt = act(case)
+    lp = case.layers[layer_idx]
+    xx = dev(case.x, dt) if x is None else x
+    y = B.layer_forward(xx, dev(lp.w1, dt), dev(lp.w2, dt), dev(case.seq_offsets),
+                        case.max_seq_len, dev(case.timestamps), dev(lp.rab_pos),
+                        dev(lp.rab_time), num_heads=case.num_heads, d_qk=case.d_qk,
+                        d_v=case.d_v, max_pos_dist=case.max_pos_dist,
+                        num_time_buckets=case.num_time_buckets, alpha=case.alpha,
+                        mask=case.mask, num_candidates=case.num_candidates,
+                        microbatch=max(case.microbatch, 1), out=out)
+    return y
+
+
+def oracle_layer(case, layer_idx=0, x=None):
+    lp = case.layers[layer_idx]
+    return O.layer_forward(case.x if x is None else x, lp.w1, lp.w2, case.seq_offsets,
+                           case.timestamps, lp.rab_pos, lp.rab_time, **attn_kw(case))
+
+
+@pytest.mark.parametrize("bf16", [True, False])
+def test_layer_forward_small(B, bf16):
+    case = W.random_layer_case(20, [150, 1, 129, 64, 0, 260], d_model=128, H=2, d=64, P=30,
+                               NB=16, bf16=bf16, w_std=0.05)
+    y = gpu_layer(B, case)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_layer(case), f"layer bf16={bf16}")
+
+
+def test_layer_forward_mfalcon_small(B):
+    case = W.random_layer_case(21, [300, 250], d_model=128, H=2, d=64, P=30, NB=16,
+                               mask=W.MASK_MFALCON, num_candidates=100)
+    y = gpu_layer(B, case)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_layer(case), "layer mfalcon")
+
+
+def test_layer_fp32_b4_workload(B):
+    case = W.make("layer_fp32_b4")
+    y = gpu_layer(B, case)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_layer(case), "layer_fp32_b4")
+
+
+def test_layer_bf16_b32_geo_workload(B):
+    case = W.make("layer_bf16_b32_geo")
+    y = gpu_layer(B, case)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_layer(case), "layer_bf16_b32_geo")
+
+
+def _sequence_subcase(case, b):
+    """The single sequence b of a workload as its own jagged batch (sequences are independent)."""
+    s, e = int(case.seq_offsets[b]), int(case.seq_offsets[b + 1])
+    return s, e, np.array([0, e - s], dtype=np.int64)
+
+
+def test_stack4_workload_sampled_sequence(B):
+    """Full 4-layer stack on the GPU; the shortest and longest sequences checked in fp64."""
+    case = W.make("stack4_bf16_b8_inter")
+    dt = act(case)
+    x = dev(case.x, dt)
+    for l in range(len(case.layers)):
+        x = gpu_layer(B, case, l, x=x)
+    torch.cuda.synchronize()
+    y = x.float().cpu().numpy()
+    for b in (int(np.argmin(case.lengths)), int(np.argmax(case.lengths))):
+        s, e, off = _sequence_subcase(case, b)
+        ref = O.stack_forward(case.x[s:e], case.layers, off, case.timestamps[s:e],
+                              round_between=W.round_to_bf16, **attn_kw(case))
+        assert_close(y[s:e], ref, f"stack4 sequence {b}")
+
+
+def test_mfalcon_workload_sampled_sequence(B):
+    case = W.make("mfalcon_bf16_b16")
+    dt = act(case)
+    x = dev(case.x, dt)
+    for l in range(len(case.layers)):
+        x = gpu_layer(B, case, l, x=x)
+    torch.cuda.synchronize()
+    y = x.float().cpu().numpy()
+    s, e, off = _sequence_subcase(case, 5)
+    ref = O.stack_forward(case.x[s:e], case.layers, off, case.timestamps[s:e],
+                          round_between=W.round_to_bf16, **attn_kw(case))
+    assert_close(y[s:e], ref, "mfalcon sequence 5")
+
+
+# ----------------------------------------------------------------------- attention backward
+def gpu_backward(B, case):
+    dt = act(case)
+    q, k, v, d_o = (dev(case.q, dt), dev(case.k, dt), dev(case.v, dt), dev(case.d_o, dt))
+    res = B.attention_backward(q, k, v, d_o, dev(case.seq_offsets), case.max_seq_len,
+                               dev(case.timestamps), dev(case.rab_pos), dev(case.rab_time),
+                               num_heads=case.num_heads, max_pos_dist=case.max_pos_dist,
+                               num_time_buckets=case.num_time_buckets, alpha=case.alpha,
+                               mask=case.mask, num_candidates=case.num_candidates,
+                               microbatch=max(case.microbatch, 1))
+    torch.cuda.synchronize()
+    return res
+
+
+def oracle_backward(case):
+    return O.attention_backward(case.q, case.k, case.v, case.d_o, case.seq_offsets,
+                                case.timestamps, case.rab_pos, case.rab_time, **attn_kw(case))
+
+
+@pytest.mark.parametrize("mask,m", [(W.MASK_CAUSAL, 0), (W.MASK_MFALCON, 50)])
+def test_attention_backward_small(B, mask, m):
+    case = W.random_attention_case(30 + m, [200, 1, 129, 77], H=2, d=64, P=20, NB=16,
+                                   mask=mask, num_candidates=m, gap_mean=20.0, qkv_std=0.5)
+    got = gpu_backward(B, case)
+    ref = oracle_backward(case)
+    for name, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got, ref):
+        assert_close(g, r, f"backward {name}")
+
+
+def test_attention_backward_mid_size(B):
+    case = W.make_attn_fwdbwd_bf16_b64(seed=1, B=4, lo=512, hi=2048)
+    got = gpu_backward(B, case)
+    ref = oracle_backward(case)
+    for name, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got, ref):
+        assert_close(g, r, f"backward mid {name}")
+
+
+def test_attention_backward_full_size_sampled(B):
+    """Full attention-only backward workload; per-sequence gradients of sampled sequences, and
+    the invariant that both bias-table gradients total Σ dS over every visible pair."""
+    case = W.make("attn_fwdbwd_bf16_b64")
+    dq, dk, dv, dp, dtm = gpu_backward(B, case)
+    for b in (0, int(np.argmax(case.lengths))):
+        s, e, off = _sequence_subcase(case, b)
+        ref = O.attention_backward(case.q[s:e], case.k[s:e], case.v[s:e], case.d_o[s:e], off,
+                                   case.timestamps[s:e], case.rab_pos, case.rab_time,
+                                   **attn_kw(case))
+        for name, g, r in zip(("dq", "dk", "dv"), (dq[s:e], dk[s:e], dv[s:e]), ref[:3]):
+            assert_close(g, r, f"full backward seq {b} {name}")
+    tp, tt = float(dp.double().sum()), float(dtm.double().sum())
+    assert abs(tp - tt) <= 1e-3 * max(abs(tp), abs(tt), 1.0)
+
+
+# ---------------------------------------------------------------------------- misc kernels
+def test_jagged_padded_roundtrip(B):
+    lengths = np.array([5, 0, 130, 1, 64])
+    off = W.offsets_from_lengths(lengths)
+    T = int(off[-1])
+    vals = torch.randn(T, 24, device="cuda").to(torch.bfloat16)  # 48-byte rows
+    padded = B.jagged_to_padded(vals, dev(off), 130)
+    ref = torch.zeros(5, 130, 24, dtype=torch.bfloat16, device="cuda")
+    for b in range(5):
+        ref[b, :lengths[b]] = vals[off[b]:off[b + 1]]
+    assert torch.equal(padded, ref)
+    back = B.padded_to_jagged(padded, dev(off), T)
+    assert torch.equal(back, vals)
+    trunc = B.jagged_to_padded(vals, dev(off), 64)
+    assert torch.equal(trunc, ref[:, :64])
+
+
+def test_malformed_offsets_set_device_check(B):
+    case = W.random_attention_case(40, [100, 50], H=1, d=64)
+    dt = act(case)
+    q = dev(case.q, dt)
+    bad = dev(np.array([0, 120, 150], dtype=np.int32))  # first length 120 > max_seq_len 100
+    ws = B.Workspace(1 << 20, q.device)
+    out = torch.full_like(q, 7.0)
+    B.attention_forward(q, q, q, bad, 100, None, None, None, num_heads=1, out=out, ws=ws)
+    assert ws.sync_status() == 6
+    assert torch.all(out == 7.0)
+    assert ws.sync_status() == 0  # reading the status clears it
