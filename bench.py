@@ -201,6 +201,49 @@ def run_reference(args, rank):
 
 
 # ------------------------------------------------------------------------------- our arm
+def truncate_batch(wl, b):
+    """The first b sequences of a workload (a smaller case of the same shapes)."""
+    T = int(wl.seq_offsets[b])
+    wl.lengths = wl.lengths[:b]
+    wl.seq_offsets = wl.seq_offsets[:b + 1]
+    wl.timestamps = wl.timestamps[:T]
+    wl.x = wl.x[:T]
+    return wl
+
+
+def run_attention_only(args, lib, Bd, desc, ly, x, y, ws, stream, wl):
+    """Time the attention stage of layer 0 alone (f1 runs once first to fill Q/K/V)."""
+    import torch
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def stage(k):
+        st = lib.hstu_layer_forward_stage(
+            ctypes.byref(desc), k, ctypes.c_void_p(x.data_ptr()),
+            ctypes.c_void_p(ly["w1"].data_ptr()), None, ctypes.c_void_p(ly["w2"].data_ptr()),
+            None, ctypes.c_void_p(y.data_ptr()), ws.ptr, ws.nbytes, sp)
+        if st != 0:
+            raise Bd.HstuError(st, f"stage {k}")
+
+    stage(1)
+    for _ in range(args.warmup):
+        stage(2)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        stage(2)
+        b.record(stream)
+    torch.cuda.synchronize()
+    if ws.sync_status() != 0:
+        raise RuntimeError("device status word set")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    fl = attention_flops(wl)
+    print(json.dumps({"mode": "attn", "workload": wl.name, "seqs": wl.num_seqs,
+                      "tokens": wl.total_tokens, "attn_ms": ms,
+                      "attn_tflops": fl / (ms / 1e3) / 1e12}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -210,6 +253,10 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--mode", default="stack", choices=["stack", "attn"],
+                    help="attn: time only the attention stage of layer 0 (profiling aid)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="use only the first B sequences of the workload (profiling aid)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -241,6 +288,8 @@ def main():
         del wl0
 
     wl = W.make(WORKLOAD, seed=args.seed + rank)
+    if args.batch > 0:
+        wl = truncate_batch(wl, args.batch)
     T, L = wl.total_tokens, len(wl.layers)
     bf = torch.bfloat16
     x = torch.from_numpy(wl.x).to(bf).to(dev)
@@ -285,6 +334,10 @@ def main():
                     attn_events[l][1].record(stream)
             cur = out
         return cur
+
+    if args.mode == "attn":
+        run_attention_only(args, lib, Bd, descs[0], layers[0], x, bufs[0], ws, stream, wl)
+        return
 
     for _ in range(args.warmup):
         run_stack()

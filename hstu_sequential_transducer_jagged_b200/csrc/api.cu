@@ -20,8 +20,14 @@ cudaError_t launch_gemm_bf16_tc(int epi, const CUtensorMap& ta, const CUtensorMa
                                 int64_t ld_r, __nv_bfloat16* C, int64_t ldc, int* status,
                                 cudaStream_t stream);
 cudaError_t launch_build_worklist(const int32_t* offsets, int B, int T, int max_len, int mask,
-                                  int m, WorkItem* items, int32_t* count, int32_t* hist,
-                                  int max_cost, int32_t* status, cudaStream_t stream);
+                                  int m, int group, WorkItem* items, int32_t* count,
+                                  int32_t* hist, int max_cost, int32_t* status,
+                                  cudaStream_t stream);
+cudaError_t launch_attn_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const CUtensorMap& tts,
+                                 const AttnGeom& g, __nv_bfloat16* out, int64_t ld_o, int grid,
+                                 cudaStream_t stream);
+size_t attn_fwd_pair_smem(int P, bool has_pos);
 cudaError_t launch_ln_gate(int dtype, const void* av, int64_t ld_av, const void* u, int64_t ld_u,
                            const float* gamma, const float* beta, float eps, void* g,
                            int64_t ld_g, int rows, int F, cudaStream_t stream);
@@ -97,12 +103,28 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t col
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// 1D int64 tensor map over n elements, box of `box` elements, no swizzle, zero fill.
+bool make_map_i64_1d(CUtensorMap* map, const void* base, int64_t n, uint32_t box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[1] = {static_cast<cuuint64_t>(n)};
+  cuuint64_t strides[1] = {8};
+  cuuint32_t boxd[1] = {box};
+  cuuint32_t estr[1] = {1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_INT64, 1, const_cast<void*>(base), dims, strides,
+                  boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 size_t elem_size(int dtype) { return dtype == HSTU_BF16 ? 2 : 4; }
 
 // Work-list sizes for a batch: an upper bound of the number of 128-row query tiles
 // (Σ ceil(L_b / 128) <= T / 128 + B) and of the cost histogram.
-int max_items(int T, int B) { return (T + kTileRows - 1) / kTileRows + B; }
-int max_cost(int max_len) { return (max_len + kTileRows - 1) / kTileRows + 1; }
+int max_items(int T, int B, int group = 1) {
+  return (T + kTileRows * group - 1) / (kTileRows * group) + B;
+}
+int max_cost(int max_len) { return 2 * ((max_len + kTileRows - 1) / kTileRows + 1); }
 
 struct WsLayout {
   size_t items, hist, total_attn;
@@ -163,23 +185,43 @@ AttnGeom make_geom(const void* ws, const WsLayout& w, const int64_t* ts, const f
 }
 
 cudaError_t build_list(const void* ws, const WsLayout& w, const int32_t* offsets, int B, int T,
-                       int max_len, int mask, int m, cudaStream_t s) {
+                       int max_len, int mask, int m, int group, cudaStream_t s) {
   uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(ws));
   return launch_build_worklist(offsets, B, T, max_len, mask, mask == HSTU_MASK_MFALCON ? m : 0,
+                               group,
                                reinterpret_cast<WorkItem*>(base + w.items),
                                reinterpret_cast<int32_t*>(base + 4),
                                reinterpret_cast<int32_t*>(base + w.hist), max_cost(max_len),
                                reinterpret_cast<int32_t*>(base), s);
 }
 
-// Attention forward on a ready work list.
-hstu_status_t attn_forward_core(const AttnGeom& g, int B, int T, int D, int dtype, const void* q,
-                                int64_t ld_q, const void* k, int64_t ld_k, const void* v,
-                                int64_t ld_v, void* o, int64_t ld_o, cudaStream_t s) {
-  const int grid = max_items(T, B) * g.H;
-  const bool tc = dtype == HSTU_BF16 && (D == 64 || D == 128) && aligned16(q) && aligned16(k) &&
-                  aligned16(v) && aligned16(o) && (ld_q % 8 == 0) && (ld_k % 8 == 0) &&
-                  (ld_v % 8 == 0) && (ld_o % 8 == 0);
+// True when the tensor-core kernels take this attention problem.
+bool attn_uses_tc(int D, int dtype, const void* q, int64_t ld_q, const void* k, int64_t ld_k,
+                  const void* v, int64_t ld_v, const void* o, int64_t ld_o) {
+  return dtype == HSTU_BF16 && (D == 64 || D == 128) && aligned16(q) && aligned16(k) &&
+         aligned16(v) && aligned16(o) && (ld_q % 8 == 0) && (ld_k % 8 == 0) && (ld_v % 8 == 0) &&
+         (ld_o % 8 == 0);
+}
+
+// Builds the work list (pairs of query tiles for the head-width-64 tensor-core kernel, single
+// tiles otherwise) and launches the attention forward.
+hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t* offsets,
+                                int max_len, const AttnGeom& g, int B, int T, int D, int dtype,
+                                const void* q, int64_t ld_q, const void* k, int64_t ld_k,
+                                const void* v, int64_t ld_v, void* o, int64_t ld_o,
+                                cudaStream_t s) {
+  const bool tc = attn_uses_tc(D, dtype, q, ld_q, k, ld_k, v, ld_v, o, ld_o);
+  // the paired kernel keeps the position tables in shared memory (P <= 2048) and loads the
+  // timestamps with TMA (16-byte aligned base)
+  const bool use_time = g.ts != nullptr && g.rab_time != nullptr;
+  const bool pair = tc && D == 64 && (g.rab_pos == nullptr || g.P <= 2048) &&
+                    (!use_time || aligned16(g.ts)) &&
+                    attn_fwd_pair_smem(g.P, g.rab_pos != nullptr) <= 227 * 1024;
+  const int group = pair ? 2 : 1;
+  if (build_list(ws, w, offsets, B, T, max_len, g.mask, g.num_candidates, group, s) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int grid = max_items(T, B, group) * g.H;
   cudaError_t e;
   if (tc) {
     CUtensorMap tq, tk, tv;
@@ -188,7 +230,17 @@ hstu_status_t attn_forward_core(const AttnGeom& g, int B, int T, int D, int dtyp
         !make_map_bf16(&tk, k, T, cols, ld_k, 64, kTileRows) ||
         !make_map_bf16(&tv, v, T, cols, ld_v, 64, kTileRows))
       return HSTU_ERR_CUDA;
-    e = launch_attn_fwd_tc(D, tq, tk, tv, g, static_cast<__nv_bfloat16*>(o), ld_o, grid, s);
+    if (pair) {
+      CUtensorMap tts;
+      std::memset(&tts, 0, sizeof(tts));
+      if (use_time && !make_map_i64_1d(&tts, g.ts, T, 136)) return HSTU_ERR_CUDA;
+      // persistent: one CTA per SM, each walking the work list with a stride
+      const int pgrid = grid < num_sms_current() ? grid : num_sms_current();
+      e = launch_attn_fwd_pair(tq, tk, tv, tts, g, static_cast<__nv_bfloat16*>(o), ld_o, pgrid,
+                               s);
+    }
+    else
+      e = launch_attn_fwd_tc(D, tq, tk, tv, g, static_cast<__nv_bfloat16*>(o), ld_o, grid, s);
   } else {
     e = launch_attn_fwd_simt(dtype, D, g, q, ld_q, k, ld_k, v, ld_v, o, ld_o, grid, s);
   }
@@ -247,14 +299,12 @@ hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* d, const void* q, c
   if (d->num_seqs == 0 || d->total_tokens == 0) return HSTU_OK;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return HSTU_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (build_list(ws, w, d->seq_offsets, d->num_seqs, d->total_tokens, d->max_seq_len, d->mask,
-                 d->num_candidates, s) != cudaSuccess)
-    return HSTU_ERR_CUDA;
   const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
                                d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
                                d->num_candidates, d->alpha);
-  return attn_forward_core(g, d->num_seqs, d->total_tokens, D, d->dtype, q, d->ld_q, k, d->ld_k,
-                           v, d->ld_v, o, d->ld_o, s);
+  return attn_forward_core(ws, w, d->seq_offsets, d->max_seq_len, g, d->num_seqs,
+                           d->total_tokens, D, d->dtype, q, d->ld_q, k, d->ld_k, v, d->ld_v, o,
+                           d->ld_o, s);
 }
 
 hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, const void* k,
@@ -291,7 +341,7 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
       dk == nullptr || dv == nullptr)
     return HSTU_ERR_INVALID_ARG;
   if (build_list(ws, w, d->seq_offsets, d->num_seqs, d->total_tokens, d->max_seq_len, d->mask,
-                 d->num_candidates, s) != cudaSuccess)
+                 d->num_candidates, 1, s) != cudaSuccess)
     return HSTU_ERR_CUDA;
   const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
                                d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
@@ -359,13 +409,10 @@ hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* d, int32_t stage
                 status, s);
   }
   if (stage == HSTU_STAGE_ATTENTION) {
-    if (build_list(ws, w, d->seq_offsets, d->num_seqs, T, d->max_seq_len, d->mask,
-                   d->num_candidates, s) != cudaSuccess)
-      return HSTU_ERR_CUDA;
     const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
                                  d->num_time_buckets, H, T, d->mask, d->num_candidates, d->alpha);
-    return attn_forward_core(g, d->num_seqs, T, D, d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av,
-                             hv, s);
+    return attn_forward_core(ws, w, d->seq_offsets, d->max_seq_len, g, d->num_seqs, T, D,
+                             d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av, hv, s);
   }
   // Norm(AV) ⊙ U, then f2 + residual: Y = X + G W2 + b2
   if (launch_ln_gate(d->dtype == HSTU_BF16 ? 0 : 1, av, hv, u_ptr, n1, d->ln_gamma, d->ln_beta,

@@ -292,11 +292,9 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
     for (int t = 0; t < nkv; ++t) {
       const int st = t % kStages;
       const int c0l = kr.tile(t, it.qtile) * kTileRows;
-      if (use_time && !mbar_wait(&sm.kv_full[st], (t / kStages) & 1, abort_flag, g.status)) {
-        ok = false;
-        break;
-      }
-      if (!mbar_wait(&sm.s_full, t & 1, abort_flag, g.status)) {
+      bool w = !use_time || mbar_wait(&sm.kv_full[st], (t / kStages) & 1, abort_flag, g.status);
+      w = w && mbar_wait(&sm.s_full, t & 1, abort_flag, g.status);
+      if (!warp_all(w)) {
         ok = false;
         break;
       }
@@ -346,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
       tc_fence_before();
       mbar_arrive(&sm.p_full);
     }
-    if (ok && mbar_wait(&sm.o_full, 0, abort_flag, g.status)) {
+    if (ok && warp_all(mbar_wait(&sm.o_full, 0, abort_flag, g.status))) {
       tc_fence_after();
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {

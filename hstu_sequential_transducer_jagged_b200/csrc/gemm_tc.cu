@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const int quad = warp & 3;
     const int row = m0 + quad * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    if (mbar_wait(&sm.acc_full, 0, abort_flag, status)) {
+    if (warp_all(mbar_wait(&sm.acc_full, 0, abort_flag, status))) {
       tc_fence_after();
 #pragma unroll 1
       for (int ch = 0; ch < kBN / 32; ++ch) {

@@ -12,14 +12,24 @@
 namespace hstu {
 
 // ------------------------------------------------------------------------------ work list
-// One CTA.  Validates offsets (offsets[0] == 0, non-decreasing, offsets[B] == T, every length
-// <= max_len); on failure writes the device-check status and an empty list.  Items are placed
-// in decreasing order of cost (the number of KV tiles visited) by a counting sort, so that the
-// longest tiles start first.  hist holds max_cost + 1 counters (global workspace).
+// One CTA.  Validates offsets (offsets[0] == 0, offsets[B] == T, every length in [0, max_len]);
+// on failure writes the device-check status and an empty list.  An item is a group of
+// `group` consecutive 128-row query tiles of one sequence (1 or 2); items are placed in
+// decreasing order of cost (KV tiles visited, summed over the group) by a counting sort, so the
+// longest items start first.  hist holds max_cost + 1 counters (global workspace).
+__device__ __forceinline__ int item_cost(int qt0, int group, int L, int n) {
+  int cost = 0;
+  for (int a = 0; a < group; ++a) {
+    const int qt = qt0 + a;
+    if (qt * kTileRows < L) cost += kv_range(qt, L, n).count();
+  }
+  return cost;
+}
+
 __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B, int T,
-                                      int max_len, int mask, int m, WorkItem* __restrict__ items,
-                                      int32_t* __restrict__ count, int32_t* __restrict__ hist,
-                                      int max_cost, int32_t* status) {
+                                      int max_len, int mask, int m, int group,
+                                      WorkItem* __restrict__ items, int32_t* __restrict__ count,
+                                      int32_t* __restrict__ hist, int max_cost, int32_t* status) {
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   for (int c = threadIdx.x; c <= max_cost; c += blockDim.x) hist[c] = 0;
@@ -27,10 +37,7 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
   if (threadIdx.x == 0 && (offsets[0] != 0 || offsets[B] != T)) bad = 1;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int L = offsets[b + 1] - offsets[b];
-    if (L < 0 || L > max_len) {
-      bad = 1;
-      continue;
-    }
+    if (L < 0 || L > max_len) bad = 1;
   }
   __syncthreads();
   if (bad) {
@@ -40,19 +47,14 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
     }
     return;
   }
-  // histogram of costs
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int L = offsets[b + 1] - offsets[b];
     const int n = hist_len(L, mask, m);
     const int nt = (L + kTileRows - 1) / kTileRows;
-    for (int qt = 0; qt < nt; ++qt) {
-      const KvRange r = kv_range(qt, L, n);
-      atomicAdd(&hist[r.count()], 1);
-    }
+    for (int qt = 0; qt < nt; qt += group) atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
   }
   __syncthreads();
-  // exclusive scan in decreasing cost (single thread: max_cost is small)
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0) {  // exclusive scan in decreasing cost
     int run = 0;
     for (int c = max_cost; c >= 0; --c) {
       const int h = hist[c];
@@ -66,9 +68,8 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
     const int L = offsets[b + 1] - offsets[b];
     const int n = hist_len(L, mask, m);
     const int nt = (L + kTileRows - 1) / kTileRows;
-    for (int qt = 0; qt < nt; ++qt) {
-      const KvRange r = kv_range(qt, L, n);
-      const int pos = atomicAdd(&hist[r.count()], 1);
+    for (int qt = 0; qt < nt; qt += group) {
+      const int pos = atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
       WorkItem it;
       it.seq = b;
       it.qtile = qt;
@@ -80,10 +81,11 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
 }
 
 cudaError_t launch_build_worklist(const int32_t* offsets, int B, int T, int max_len, int mask,
-                                  int m, WorkItem* items, int32_t* count, int32_t* hist,
-                                  int max_cost, int32_t* status, cudaStream_t stream) {
-  build_worklist_kernel<<<1, 1024, 0, stream>>>(offsets, B, T, max_len, mask, m, items, count,
-                                                hist, max_cost, status);
+                                  int m, int group, WorkItem* items, int32_t* count,
+                                  int32_t* hist, int max_cost, int32_t* status,
+                                  cudaStream_t stream) {
+  build_worklist_kernel<<<1, 1024, 0, stream>>>(offsets, B, T, max_len, mask, m, group, items,
+                                                count, hist, max_cost, status);
   return cudaGetLastError();
 }
 
