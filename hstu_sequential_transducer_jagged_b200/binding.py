@@ -28,13 +28,17 @@ EXPORTED = [
     "hstu_layer_workspace_size", "hstu_layer_forward", "hstu_layer_forward_stage",
     "hstu_jagged_padded_copy",
     "hstu_debug_time_buckets", "hstu_workspace_init", "hstu_sync_status",
-    "hstu_status_string", "hstu_version",
+    "hstu_status_string", "hstu_version", "hstu_last_error_string",
 ]
 
 
 class HstuError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, 'unknown')} (status {status})")
+        detail = ""
+        if status == 4 and _LIB is not None:
+            detail = ": " + _LIB.hstu_last_error_string().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, 'unknown')} (status {status})"
+                         f"{detail}")
         self.status = status
 
 
@@ -89,6 +93,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_sync_status": (i32, [vp, vp]),
         "hstu_status_string": (ctypes.c_char_p, [i32]),
         "hstu_version": (ctypes.c_char_p, []),
+        "hstu_last_error_string": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -52,6 +53,15 @@ cudaError_t launch_attn_bwd_simt(int dtype, int D, const AttnGeom& g, const void
 using namespace hstu;
 
 namespace {
+
+thread_local char g_last_error[256] = "";
+
+// Records a CUDA error's text for hstu_last_error_string() and maps it to HSTU_ERR_CUDA.
+hstu_status_t cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return HSTU_ERR_CUDA;
+}
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;  // status word at 0, work-item count at 4
@@ -244,7 +254,7 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
   } else {
     e = launch_attn_fwd_simt(dtype, D, g, q, ld_q, k, ld_k, v, ld_v, o, ld_o, grid, s);
   }
-  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
 // C = epi(A[M,K] B[K,N] + bias) on tensor cores when the shapes allow, else on CUDA cores.
@@ -264,7 +274,7 @@ hstu_status_t gemm(int dtype, int epi, const void* A, int64_t lda, const void* B
   } else {
     e = launch_gemm_simt(dtype, epi, A, lda, Bm, ldb, M, N, K, bias, R, ldr, C, ldc, s);
   }
-  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
 }  // namespace
@@ -349,7 +359,7 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
   const int grid = max_items(d->total_tokens, d->num_seqs) * d->num_heads;
   cudaError_t e = launch_attn_bwd_simt(d->dtype, D, g, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o,
                                        d->ld_o, dq, dk, dv, d_rab_pos, d_rab_time, grid, s);
-  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* d) {
@@ -452,7 +462,7 @@ hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_se
                                        jagged_row_stride_bytes, padded, padded_row_stride_bytes,
                                        row_bytes, to_padded, num_sms_current(),
                                        reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
 hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out, int32_t nb,
@@ -461,7 +471,7 @@ hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out
   if (n == 0) return HSTU_OK;
   if (dt == nullptr || out == nullptr) return HSTU_ERR_INVALID_ARG;
   cudaError_t e = launch_time_buckets(dt, n, out, nb, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
 hstu_status_t hstu_workspace_init(void* ws, size_t ws_bytes, hstu_stream_t stream) {
@@ -499,5 +509,7 @@ const char* hstu_status_string(hstu_status_t s) {
 }
 
 const char* hstu_version(void) { return "hstu_b200 0.1 sm_100a"; }
+
+const char* hstu_last_error_string(void) { return g_last_error; }
 
 }  // extern "C"

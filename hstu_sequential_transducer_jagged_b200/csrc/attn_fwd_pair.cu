@@ -14,11 +14,13 @@
 //
 // One CTA per SM walks the longest-first work list with a fixed stride (CTA b takes items
 // b, b + grid, ...); barrier phases run on across items, so the producer streams the next
-// item's tiles while the current one drains.  Warps: 0 TMA producer; 1 TMEM allocation;
-// 2-5 warpgroup 0 and 6-9 warpgroup 1 (warp w owns TMEM lanes 32*(w%4) .. +31: one query row
-// per thread).  Each warpgroup issues its own MMAs: after its 128 threads have written P (a
-// named barrier), one elected thread issues O += P V and the next S = Q Kᵀ, so the hand-off
-// costs a named barrier instead of two mbarrier round trips through a separate MMA warp.
+// item's tiles while the current one drains.  Warpgroup 0: warp 0 TMA producer; warp 1 TMEM
+// allocation and single-thread tcgen05.mma issue (a thread that issues MMAs stalls for about
+// their execution time, so issuing stays off the epilogue warps); warp 2 timestamps (per KV
+// tile: min / max timestamp and int32 copies for the bias classification and gathers); warp 3
+// spare.  Warpgroups 1 and 2: the two epilogue warpgroups (warp w owns TMEM lanes
+// 32*(w%4) .. +31: one query row per thread).  After set-up warpgroup 0 gives registers to the
+// epilogue warpgroups (setmaxnreg 88 / 208).
 // TMEM (512 columns): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O0 [384,448)
 // O1 [448,512); P is bf16, two per 32-bit column, and feeds the PV MMA as its A operand.
 //
@@ -40,7 +42,7 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kTileBytes = kTileRows * kD * 2;  // 16 KB bf16 tile, 128-byte swizzle
 constexpr int kTsBox = 136;      // timestamps loaded per KV tile (x rounded down to even)
 constexpr int kTsStride = 144;   // per-stage buffer: 1152 bytes keeps every TMA destination 128-byte aligned
@@ -56,16 +58,19 @@ struct PairSmem {
   alignas(1024) uint8_t k[kStages][kTileBytes];
   alignas(1024) uint8_t v[kStages][kTileBytes];
   alignas(128) long long ts[kStages][kTsStride];
+  alignas(16) int ts32[kStages][kTileRows];  // low 32 bits of the tile's 128 timestamps
   float rab_time_h[kTimeSmem];  // 0.5 x rab_time, clamped index
-  long long tmin[kStages];       // min / max timestamp of each stage's in-range columns
+  long long tmin[kStages];       // min / max timestamp of each stage's in-sequence columns
   long long tmax[kStages];
   uint64_t q_full, q_empty;
   uint64_t kv_full[kStages];
-  uint64_t ts_ready[kStages];    // tmin / tmax of the stage published (warp 1)
+  uint64_t ts_ready[kStages];    // ts32 / tmin / tmax of the stage published (warp 10)
   uint64_t kv_empty[kStages];
   uint64_t s_full[2];
+  uint64_t p_full[2];
   uint64_t o_full[2];
-  uint64_t drain[2];
+  uint64_t o_empty[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
   // followed by: float4 pos4[P+1] (16-byte aligned), float pos_h[2P+1]
@@ -145,108 +150,101 @@ __device__ __forceinline__ int bucket_small(int d, int nbm1) {
 }
 
 // Per-row constants of one KV tile's epilogue.  The bias modes are warp-uniform (a warp takes
-// the per-element path for all of its rows when any row needs it: the per-element formulas are
+// a per-element path for all of its rows when any row needs it; the per-element formulas are
 // exact for every row), so no branch inside the epilogue diverges.
 struct RowCtx {
   float half_alpha;
   float half_bias;    // 0.5 x (the parts of the bias that are constant along the row segment)
-  bool pos_elem;      // position term per element (shifted table; exact for visible rows)
+  bool pos_elem;      // position term per element from the shifted table
   int t4_base;        // pos4 index of column c is clamp(t4_base - c, 0, P)
-  int pi_plus_p;      // p_i + P
-  int P, P2;
-  int time_mode;      // 0 in half_bias, 1 per element on 32-bit differences, 2 on 64-bit ones
+  int P;
+  int time_mode;      // 0 constant, 1 threshold (row spans <= 2 buckets), 2 per element 32-bit,
+                      // 3 per element 64-bit
+  int thr;            // time_mode 1: dt >= thr takes t_hi
+  float t_lo, t_hi;
   int ti_lo;
   long long ti;
-  int nbm1;
+  int pi_plus_p, P2, nbm1;
   int i, n, c0l;      // mask data (query index, history length, first column)
   bool row_valid;
   int mode;           // warp-uniform: 0 constant bias, 1 per-element bias, 2 masked
 };
 
-// hb[e] = 0.5 x bias of column ch*32+e of this row's segment (segments without a mask).
-__device__ __forceinline__ void bias_visible(float (&hb)[32], int ch, const RowCtx& rc,
-                                             const float4* pos4, const float* time_h,
-                                             const long long* ts) {
-#pragma unroll
-  for (int e = 0; e < 32; ++e) hb[e] = rc.half_bias;
-  if (rc.pos_elem) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      const float4 pv = pos4[clampi(rc.t4_base - (ch * 32 + e), 0, rc.P)];
-      hb[e] += pv.x;
-      hb[e + 1] += pv.y;
-      hb[e + 2] += pv.z;
-      hb[e + 3] += pv.w;
-    }
-  }
-  const int* ts_lo = reinterpret_cast<const int*>(ts);  // low word of each int64 (little endian)
-  if (rc.time_mode == 1) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      hb[e] += time_h[bucket_small(rc.ti_lo - ts_lo[2 * (ch * 32 + e)], rc.nbm1)];
-  } else if (rc.time_mode == 2) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) hb[e] += time_h[time_bucket64(rc.ti - ts[ch * 32 + e], rc.nbm1 + 1)];
-  }
+// 0.5 x rab_time of bucket(d) for |d| < 2^23 (table indexed by the biased fp32 exponent).
+__device__ __forceinline__ float time_term32(const float* time_h, int d) {
+  d = d < 1 ? 1 : (d > 0x7FFFFF ? 0x7FFFFF : d);
+  const float f = __int_as_float(0x4B000000 | d) - 8388608.0f;
+  return time_h[(__float_as_int(f) >> 23) - 127];
 }
 
-// hb[e] for segments on the causal diagonal or with candidate keys: general per-element bias.
-__device__ __forceinline__ void bias_masked(float (&hb)[32], int ch, const RowCtx& rc,
-                                            const float* pos_h, const float* time_h,
-                                            const long long* ts, bool use_pos, bool use_time) {
-#pragma unroll
-  for (int e = 0; e < 32; ++e) hb[e] = 0.f;
-  if (use_pos) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int j = rc.c0l + ch * 32 + e;  // candidate keys (j >= n) sit at position n
-      hb[e] += pos_h[clampi(rc.pi_plus_p - (j < rc.n ? j : rc.n), 0, rc.P2)];
-    }
-  }
-  if (use_time) {
-    const int* ts_lo = reinterpret_cast<const int*>(ts);
-    if (rc.time_mode == 2) {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) hb[e] += time_h[time_bucket64(rc.ti - ts[ch * 32 + e], rc.nbm1 + 1)];
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        hb[e] += time_h[bucket_small(rc.ti_lo - ts_lo[2 * (ch * 32 + e)], rc.nbm1)];
-    }
-  }
-}
+__device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_fast(h), h); }
 
-// One 32-column chunk: P = SiLU(alpha S + bias) as packed bf16.  MODE 0: constant bias;
-// MODE 1: per-element bias without mask; MODE 2: masked segment.
+// One 32-column chunk: P = SiLU(alpha S + bias) as packed bf16.
 template <int MODE>
 __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&pk)[16], int ch,
                                            const RowCtx& rc, const float4* pos4,
                                            const float* pos_h, const float* time_h,
-                                           const long long* ts, bool use_pos, bool use_time) {
-  float hb[32];
+                                           const int* ts32, const long long* ts, bool use_pos,
+                                           bool use_time) {
   if (MODE == 0) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) hb[e] = rc.half_bias;
-  } else if (MODE == 1) {
-    bias_visible(hb, ch, rc, pos4, time_h, ts);
-  } else {
-    bias_masked(hb, ch, rc, pos_h, time_h, ts, use_pos, use_time);
+    for (int e = 0; e < 32; e += 2)
+      pk[e >> 1] = pack_bf16x2(silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e]), rc.half_bias)),
+                               silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e + 1]), rc.half_bias)));
+    return;
   }
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
-    float pv[2];
+  for (int e = 0; e < 32; e += 4) {
+    const int c = ch * 32 + e;
+    float b[4];
+    if (MODE == 1) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const float h = fmaf(rc.half_alpha, __uint_as_float(s[e + u]), hb[e + u]);
-      float p = fmaf(h, tanh_fast(h), h);
-      if (MODE == 2) {
-        const int j = rc.c0l + ch * 32 + e + u;
-        const bool vis = rc.row_valid && (j <= rc.i) && (j < rc.n || j == rc.i);
-        p = vis ? p : 0.f;
+      for (int q = 0; q < 4; ++q) b[q] = rc.half_bias;
+      if (rc.pos_elem) {
+        const float4 pv = pos4[clampi(rc.t4_base - c, 0, rc.P)];
+        b[0] += pv.x;
+        b[1] += pv.y;
+        b[2] += pv.z;
+        b[3] += pv.w;
       }
-      pv[u] = p;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        b[q] = 0.f;
+        if (use_pos) {
+          const int j = rc.c0l + c + q;  // candidate keys (j >= n) sit at position n
+          b[q] = pos_h[clampi(rc.pi_plus_p - (j < rc.n ? j : rc.n), 0, rc.P2)];
+        }
+      }
     }
-    pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+    if (rc.time_mode == 1) {
+      const int4 tv = *reinterpret_cast<const int4*>(ts32 + c);
+      b[0] += (rc.ti_lo - tv.x >= rc.thr) ? rc.t_hi : rc.t_lo;
+      b[1] += (rc.ti_lo - tv.y >= rc.thr) ? rc.t_hi : rc.t_lo;
+      b[2] += (rc.ti_lo - tv.z >= rc.thr) ? rc.t_hi : rc.t_lo;
+      b[3] += (rc.ti_lo - tv.w >= rc.thr) ? rc.t_hi : rc.t_lo;
+    } else if (rc.time_mode == 2) {
+      const int4 tv = *reinterpret_cast<const int4*>(ts32 + c);
+      b[0] += time_term32(time_h, rc.ti_lo - tv.x);
+      b[1] += time_term32(time_h, rc.ti_lo - tv.y);
+      b[2] += time_term32(time_h, rc.ti_lo - tv.z);
+      b[3] += time_term32(time_h, rc.ti_lo - tv.w);
+    } else if (rc.time_mode == 3) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) b[q] += time_h[time_bucket64(rc.ti - ts[c + q], rc.nbm1 + 1)];
+    }
+    float p[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      p[q] = silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e + q]), b[q]));
+      if (MODE == 2) {
+        const int j = rc.c0l + c + q;
+        const bool vis = rc.row_valid && (j <= rc.i) && (j < rc.n || j == rc.i);
+        p[q] = vis ? p[q] : 0.f;
+      }
+    }
+    pk[e >> 1] = pack_bf16x2(p[0], p[1]);
+    pk[(e >> 1) + 1] = pack_bf16x2(p[2], p[3]);
   }
 }
 
@@ -254,25 +252,25 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p
 template <int MODE>
 __device__ __forceinline__ void tile_epilogue(uint32_t s_addr, uint32_t p_addr, const RowCtx& rc,
                                               const float4* pos4, const float* pos_h,
-                                              const float* time_h, const long long* ts,
-                                              bool use_pos, bool use_time) {
+                                              const float* time_h, const int* ts32,
+                                              const long long* ts, bool use_pos, bool use_time) {
   uint32_t b0[32], b1[32];
   uint32_t pk[16];
   tmem_ld32(s_addr, b0);
   tmem_wait_ld_regs(b0);
   tmem_ld32(s_addr + 32, b1);
-  silu_chunk<MODE>(b0, pk, 0, rc, pos4, pos_h, time_h, ts, use_pos, use_time);
+  silu_chunk<MODE>(b0, pk, 0, rc, pos4, pos_h, time_h, ts32, ts, use_pos, use_time);
   tmem_st16(p_addr, pk);
   tmem_wait_ld_regs(b1);
   tmem_ld32(s_addr + 64, b0);
-  silu_chunk<MODE>(b1, pk, 1, rc, pos4, pos_h, time_h, ts, use_pos, use_time);
+  silu_chunk<MODE>(b1, pk, 1, rc, pos4, pos_h, time_h, ts32, ts, use_pos, use_time);
   tmem_st16(p_addr + 16, pk);
   tmem_wait_ld_regs(b0);
   tmem_ld32(s_addr + 96, b1);
-  silu_chunk<MODE>(b0, pk, 2, rc, pos4, pos_h, time_h, ts, use_pos, use_time);
+  silu_chunk<MODE>(b0, pk, 2, rc, pos4, pos_h, time_h, ts32, ts, use_pos, use_time);
   tmem_st16(p_addr + 32, pk);
   tmem_wait_ld_regs(b1);
-  silu_chunk<MODE>(b1, pk, 3, rc, pos4, pos_h, time_h, ts, use_pos, use_time);
+  silu_chunk<MODE>(b1, pk, 3, rc, pos4, pos_h, time_h, ts32, ts, use_pos, use_time);
   tmem_st16(p_addr + 48, pk);
 }
 
@@ -306,6 +304,81 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Bias classification of one row segment [c0l, c0l + 128) (this thread's query row; the
+// stage's timestamps and their min / max must be published).  Returns the row context with the
+// warp-uniform epilogue mode.  Everything is passed and returned by value so the context stays
+// in registers.
+__device__ __forceinline__ RowCtx classify_segment(RowCtx rc, int c0l, int i, int n, int pi,
+                                                   long long ti, bool row_valid, bool use_pos,
+                                                   bool use_time, int P, int NB,
+                                                   long long tmin, long long tmax,
+                                                   const float* pos_h, const float* time_h) {
+  const int last = c0l + kTileRows - 1;
+  const bool full_vis = last <= i && last < n;
+  const bool need_mask = row_valid && !full_vis;
+  const bool pos_elem = use_pos && row_valid && !(full_vis && pi - last >= P);
+  bool fits32 = true, multi = false;
+  int b_lo = 0, b_hi = 0;
+  if (use_time) {
+    const long long dt_lo = ti - tmax;
+    const long long dt_hi = ti - tmin;
+    fits32 = !row_valid || (dt_hi < (1ll << 23) && dt_lo > -(1ll << 23));
+    b_lo = fits32 ? bucket_small(static_cast<int>(dt_lo), NB - 1) : time_bucket64(dt_lo, NB);
+    b_hi = fits32 ? bucket_small(static_cast<int>(dt_hi), NB - 1) : time_bucket64(dt_hi, NB);
+    multi = row_valid && b_hi > b_lo + 1;
+  }
+  const bool w_mask = __any_sync(0xffffffffu, need_mask);
+  const bool w_pos = __any_sync(0xffffffffu, pos_elem);
+  const bool w_tvar = __any_sync(0xffffffffu, row_valid && b_hi != b_lo);
+  const bool w_multi = __any_sync(0xffffffffu, multi);
+  const bool w_fits = __all_sync(0xffffffffu, fits32);
+  float hbias = 0.f;
+  if (use_pos && !w_pos) hbias = pos_h[2 * P];  // every valid row is beyond the clamp
+  int tm = 0;
+  if (use_time) {
+    if (!w_tvar && !w_mask) {
+      hbias += time_h[b_lo];                      // one bucket for every valid row
+    } else if (!w_mask && !w_multi && w_fits) {
+      tm = 1;                                     // at most two buckets per row
+      rc.thr = 1 << (b_lo + 1);
+      rc.t_lo = time_h[b_lo];
+      rc.t_hi = time_h[b_hi];
+    } else {
+      tm = w_fits ? 2 : 3;
+    }
+  }
+  rc.c0l = c0l;
+  rc.pos_elem = w_pos;
+  rc.t4_base = pi - c0l - 3;  // pos_base - (P + 3) with pos_base = pi - c0l + P
+  rc.time_mode = tm;
+  rc.half_bias = hbias;
+  rc.mode = w_mask ? 2 : ((w_pos || tm != 0) ? 1 : 0);
+  return rc;
+}
+
+// One query tile's MMAs for the current KV tile: wait for its P, (on the item's first tile) wait
+// until the previous item's O was read, issue O (+)= P V, then the next S or the O commit.
+__device__ __forceinline__ bool mma_step(PairSmem& sm, uint32_t tmem, const PairPlan& plan,
+                                         int gu, int a, int st, int& pc, int& cnt, int oc,
+                                         volatile int* abort_flag, int* status) {
+  bool ok = mbar_wait(&sm.p_full[a], pc & 1, abort_flag, status);
+  ++pc;
+  if (ok && cnt == 0 && oc > 0) ok = mbar_wait(&sm.o_empty[a], (oc - 1) & 1, abort_flag, status);
+  if (!ok) return false;
+  tc_fence_after();
+  issue_pv_mma(tmem + col_o(a), tmem + col_p(a), smem_u32(sm.v[st]), cnt > 0);
+  ++cnt;
+  if (cnt < plan.count(a)) {
+    const int u2 = gu + plan.uidx(a, cnt);
+    if (!mbar_wait(&sm.kv_full[u2 % kStages], (u2 / kStages) & 1, abort_flag, status)) return false;
+    tc_fence_after();
+    issue_s_mma(tmem + col_s(a), smem_u32(sm.q[a]), smem_u32(sm.k[u2 % kStages]), &sm.s_full[a]);
+  } else {
+    mma_commit(&sm.o_full[a]);
+  }
+  return true;
+}
+
 __device__ __forceinline__ void tma_load_1d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x) {
   asm volatile(
@@ -315,6 +388,9 @@ __device__ __forceinline__ void tma_load_1d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// 12 warps launch with 168 registers each (3 warps per SM sub-partition, 16K registers each);
+// after set-up warpgroup 0 drops to 88 and the epilogue warpgroups rise to 208 (88 + 2 x 208 =
+// 504 registers per sub-partition slot, the same 64512 the block launched with).
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -352,17 +428,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm.rab_time_h[e] = 0.5f * g.rab_time[e < g.NB ? e : g.NB - 1];
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 2);      // one commit per warpgroup and item
+    mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 2);  // one commit per warpgroup (two from a sole user)
+      mbar_init(&sm.kv_empty[s], 1);
       mbar_init(&sm.ts_ready[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.s_full[a], 1);
+      mbar_init(&sm.p_full[a], 4);   // one elected lane per epilogue warp
       mbar_init(&sm.o_full[a], 1);
-      mbar_init(&sm.drain[a], 1);
+      mbar_init(&sm.o_empty[a], 4);
     }
+    mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -376,7 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
   const int stride = static_cast<int>(gridDim.x);
-
+  if (warp < 4) {
+  setmaxnreg_dec<88>();
   if (warp == 0) {
     // ============================================================ producer
     if (lane == 0) {
@@ -422,11 +501,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ============================================================ timestamp statistics
-    // For every KV tile the CTA loads: min / max timestamp of its columns inside the sequence,
-    // published on ts_ready[stage] for the warpgroups' bias classification.  A stage is
-    // refilled only after both warpgroups issued (and finished) their PV for it, which comes
-    // after they read these values.
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      int gu = 0, qi = 0;
+      int pc0 = 0, pc1 = 0;  // p_full phases consumed per query tile
+      int oc0 = 0, oc1 = 0;  // items whose O was produced per query tile
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < total; w += stride, ++qi) {
+        const WorkItem it = g.items[w / g.H];
+        const PairPlan plan =
+            make_plan(it.qtile, it.len, hist_len(it.len, g.mask, g.num_candidates));
+        ok = mbar_wait(&sm.q_full, qi & 1, abort_flag, g.status);
+        // first S of each query tile (the S buffers are free: the previous item's epilogue
+        // finished reading them before its last p_full)
+        for (int a = 0; ok && a < 2; ++a) {
+          if (plan.count(a) == 0) continue;
+          const int u = gu + plan.uidx(a, 0);
+          ok = mbar_wait(&sm.kv_full[u % kStages], (u / kStages) & 1, abort_flag, g.status);
+          if (ok) {
+            tc_fence_after();
+            issue_s_mma(tmem + col_s(a), smem_u32(sm.q[a]), smem_u32(sm.k[u % kStages]),
+                        &sm.s_full[a]);
+          }
+        }
+        int cnt0 = 0, cnt1 = 0;
+        for (int u = 0; ok && u < plan.nU; ++u) {
+          const int st = (gu + u) % kStages;
+          if (plan.member(0, u)) ok = ok && mma_step(sm, tmem, plan, gu, 0, st, pc0, cnt0, oc0, abort_flag, g.status);
+          if (plan.member(1, u)) ok = ok && mma_step(sm, tmem, plan, gu, 1, st, pc1, cnt1, oc1, abort_flag, g.status);
+          if (!ok) break;
+          mma_commit(&sm.kv_empty[st]);
+        }
+        if (plan.count(0) > 0) ++oc0;
+        if (plan.count(1) > 0) ++oc1;
+        gu += plan.nU;
+        mma_commit(&sm.q_empty);
+      }
+      if (!ok) {
+        mma_commit(&sm.drain);
+        mbar_wait(&sm.drain, 0, nullptr, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ============================================================ timestamp warp
+    // For every KV tile the CTA loads: int32 copies of its 128 timestamps and the min / max
+    // over its columns inside the sequence, published on ts_ready[stage].  A stage is refilled
+    // only after both warpgroups' PV for it (after they used these values).
     if (use_time) {
       int gu = 0;
       bool ok = true;
@@ -439,14 +560,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = warp_wait(&sm.kv_full[st], (gu / kStages) & 1, abort_flag, g.status);
           if (!ok) break;
           const int c0l = plan.tile_of(u) * kTileRows;
-          const int c0 = it.row0 + c0l;
-          const long long* ts_tile = sm.ts[st] + (c0 & 1);
+          const long long* ts_tile = sm.ts[st] + ((it.row0 + c0l) & 1);
           long long mn = LLONG_MAX, mx = LLONG_MIN;
 #pragma unroll
           for (int w4 = 0; w4 < kTileRows / 32; ++w4) {
             const int c = lane + 32 * w4;
+            const long long tv = ts_tile[c];
+            sm.ts32[st][c] = static_cast<int>(tv);
             if (c0l + c < it.len) {  // the sequence's own columns
-              const long long tv = ts_tile[c];
               mn = tv < mn ? tv : mn;
               mx = tv > mx ? tv : mx;
             }
@@ -467,67 +588,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  }
   } else {
-    // ============================================================ warpgroups 0 and 1
-    const int a = (warp - 2) >> 2;
+    setmaxnreg_inc<208>();
+    // ============================================================ epilogue warpgroups
+    const int a = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const bool leader = (warp == 2 + 4 * a) && lane == 0;  // issues this warpgroup's MMAs
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t qb = smem_u32(sm.q[a]);
-    const uint32_t s_tmem = tmem + col_s(a);
-    const uint32_t p_tmem = tmem + col_p(a);
-    const uint32_t o_tmem = tmem + col_o(a);
     RowCtx rc;
     rc.half_alpha = 0.5f * g.alpha;
     rc.P = g.P;
     rc.P2 = 2 * g.P;
     rc.nbm1 = g.NB - 1;
-    int gu = 0, qi = 0, sk = 0, oc = 0;
+
+    int gu = 0, sk = 0, oc = 0;
     bool ok = true;
-
-    // Bias classification of the row segment [c0l, c0l + 128) (KV tile uu of the item; the
-    // timestamps of its stage must be ready).  Sets rc.{c0l, half_bias, pos_elem, t4_base,
-    // time_mode, mode}.
-    auto classify = [&](const PairPlan& plan, int uu, int st, int row0, int i, int n, int pi,
-                        long long ti, bool row_valid) {
-      const int c0l = plan.tile_of(uu) * kTileRows;
-      const int last = c0l + kTileRows - 1;
-      const bool full_vis = last <= i && last < n;
-      const bool need_mask = row_valid && !full_vis;
-      float hbias = 0.f;
-      bool pos_elem = false, time_elem = false, fits32 = true;
-      if (use_pos) pos_elem = row_valid && !(full_vis && pi - last >= g.P);
-      int b_lo = 0;
-      if (use_time) {
-        const long long dt_lo = ti - sm.tmax[st];
-        const long long dt_hi = ti - sm.tmin[st];
-        fits32 = !row_valid || (dt_hi < (1ll << 23) && dt_lo > -(1ll << 23));
-        b_lo = fits32 ? bucket_small(static_cast<int>(dt_lo), g.NB - 1) : time_bucket64(dt_lo, g.NB);
-        const int b_hi = fits32 ? bucket_small(static_cast<int>(dt_hi), g.NB - 1)
-                                : time_bucket64(dt_hi, g.NB);
-        time_elem = row_valid && b_lo != b_hi;
-      }
-      const bool w_mask = __any_sync(0xffffffffu, need_mask);
-      const bool w_pos = __any_sync(0xffffffffu, pos_elem);
-      const bool w_time = __any_sync(0xffffffffu, time_elem);
-      const bool w_fits = __all_sync(0xffffffffu, fits32);
-      rc.c0l = c0l;
-      rc.pos_elem = w_pos;
-      rc.t4_base = pi - c0l - 3;  // pos_base - (P + 3) with pos_base = pi - c0l + P
-      // constant parts: every valid row of a warp without per-element position terms is beyond
-      // the clamp, and every valid row of a warp without per-element time terms has one bucket
-      if (use_pos && !w_pos) hbias = pos_h[2 * g.P];
-      rc.time_mode = w_time ? (w_fits ? 1 : 2) : 0;
-      if (use_time && !w_time) hbias += sm.rab_time_h[b_lo];
-      rc.half_bias = hbias;
-      rc.mode = w_mask ? 2 : ((w_pos || w_time) ? 1 : 0);
-      if (w_mask) rc.time_mode = w_fits ? 1 : 2;
-    };
-
-    // After a failed (timed-out) wait a warp keeps walking the loops "dry": it skips waits, TMEM
-    // accesses and MMAs but still reaches every named barrier, so its siblings never block.
-    for (int w = blockIdx.x; w < total; w += stride, ++qi) {
+    for (int w = blockIdx.x; ok && w < total; w += stride) {
       const WorkItem it = g.items[w / g.H];
       const int head = w % g.H;
       const int L = it.len;
@@ -544,78 +621,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       rc.n = n;
       rc.row_valid = row_valid;
       const int cnt = plan.count(a);
-      // the item's first S (its Q tiles are loaded once the previous item released them)
-      if (leader && ok) {
-        ok = mbar_wait(&sm.q_full, qi & 1, abort_flag, g.status);
-        if (ok && cnt > 0) {
-          const int u = gu + plan.uidx(a, 0);
-          ok = mbar_wait(&sm.kv_full[u % kStages], (u / kStages) & 1, abort_flag, g.status);
-          if (ok) {
-            tc_fence_after();
-            issue_s_mma(s_tmem, qb, smem_u32(sm.k[u % kStages]), &sm.s_full[a]);
-          }
-        } else if (ok) {
-          mbar_arrive(&sm.q_empty);  // this warpgroup has no rows in the item
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (cnt > 0) {  // classify the first tile
         const int u = gu + plan.uidx(a, 0);
-        if (ok && use_time) ok = warp_wait(&sm.ts_ready[u % kStages], (u / kStages) & 1, abort_flag, g.status);
-        classify(plan, plan.uidx(a, 0), u % kStages, it.row0, i, n, pi, ti, row_valid);
+        if (use_time) ok = warp_wait(&sm.ts_ready[u % kStages], (u / kStages) & 1, abort_flag, g.status);
+        if (!ok) break;
+        const int st0 = u % kStages;
+        rc = classify_segment(rc, plan.tile_of(plan.uidx(a, 0)) * kTileRows, i, n, pi, ti,
+                              row_valid, use_pos, use_time, g.P, g.NB, sm.tmin[st0],
+                              sm.tmax[st0], pos_h, sm.rab_time_h);
       }
       for (int k = 0; k < cnt; ++k, ++sk) {
-        const int uu = plan.uidx(a, k);
-        const int u = gu + uu;
+        const int u = gu + plan.uidx(a, k);
         const int st = u % kStages;
         const long long* ts_tile = sm.ts[st] + ((it.row0 + rc.c0l) & 1);
-        if (ok) ok = warp_wait(&sm.s_full[a], sk & 1, abort_flag, g.status);
+        ok = warp_wait(&sm.s_full[a], sk & 1, abort_flag, g.status);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t s_addr = lane_addr + col_s(a);
         const uint32_t p_addr = lane_addr + col_p(a);
         // warp-uniform choice (tile_epilogue holds .sync.aligned TMEM loads/stores)
-        if (!ok) {
-          // dry: nothing to compute
-        } else if (rc.mode == 0)
-          tile_epilogue<0>(s_addr, p_addr, rc, pos4, pos_h, sm.rab_time_h, ts_tile, use_pos,
-                           use_time);
+        if (rc.mode == 0)
+          tile_epilogue<0>(s_addr, p_addr, rc, pos4, pos_h, sm.rab_time_h, sm.ts32[st], ts_tile,
+                           use_pos, use_time);
         else if (rc.mode == 1)
-          tile_epilogue<1>(s_addr, p_addr, rc, pos4, pos_h, sm.rab_time_h, ts_tile, use_pos,
-                           use_time);
+          tile_epilogue<1>(s_addr, p_addr, rc, pos4, pos_h, sm.rab_time_h, sm.ts32[st], ts_tile,
+                           use_pos, use_time);
         else
-          tile_epilogue<2>(s_addr, p_addr, rc, pos4, pos_h, sm.rab_time_h, ts_tile, use_pos,
-                           use_time);
+          tile_epilogue<2>(s_addr, p_addr, rc, pos4, pos_h, sm.rab_time_h, sm.ts32[st], ts_tile,
+                           use_pos, use_time);
         tmem_wait_st();
         tc_fence_before();
-        named_barrier_sync(1 + a, 128);  // all of P (and every read of S) is done
-        if (leader && ok) {
-          tc_fence_after();
-          issue_pv_mma(o_tmem, p_tmem, smem_u32(sm.v[st]), k > 0);
-          mma_commit(&sm.kv_empty[st]);
-          if (!plan.member(1 - a, uu)) mma_commit(&sm.kv_empty[st]);  // sole user of the tile
-          if (k + 1 < cnt) {
-            const int u2 = gu + plan.uidx(a, k + 1);
-            ok = mbar_wait(&sm.kv_full[u2 % kStages], (u2 / kStages) & 1, abort_flag, g.status);
-            if (ok) issue_s_mma(s_tmem, qb, smem_u32(sm.k[u2 % kStages]), &sm.s_full[a]);
-          } else {
-            mma_commit(&sm.o_full[a]);
-            mma_commit(&sm.q_empty);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[a]);
         if (k + 1 < cnt) {  // classify the next tile while this tile's MMAs run
           const int u2 = gu + plan.uidx(a, k + 1);
-          if (ok && use_time)
+          if (use_time)
             ok = warp_wait(&sm.ts_ready[u2 % kStages], (u2 / kStages) & 1, abort_flag, g.status);
-          classify(plan, plan.uidx(a, k + 1), u2 % kStages, it.row0, i, n, pi, ti, row_valid);
+          if (!ok) break;
+          const int st2 = u2 % kStages;
+          rc = classify_segment(rc, plan.tile_of(plan.uidx(a, k + 1)) * kTileRows, i, n, pi, ti,
+                                row_valid, use_pos, use_time, g.P, g.NB, sm.tmin[st2],
+                                sm.tmax[st2], pos_h, sm.rab_time_h);
         }
       }
+      if (!ok) break;
       gu += plan.nU;
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (cnt > 0 && ok) ok = warp_wait(&sm.o_full[a], oc & 1, abort_flag, g.status);
-      if (cnt > 0) ++oc;
-      if (cnt > 0 && ok) {
-        // the item's output: its last PV is done; read O from TMEM, store bf16 rows
+      if (cnt > 0) {
+        // the item's output: wait for its last PV, read O from TMEM, store bf16 rows
+        ok = warp_wait(&sm.o_full[a], oc & 1, abort_flag, g.status);
+        if (!ok) break;
+        ++oc;
         tc_fence_after();
         uint32_t o[32];
 #pragma unroll 1
@@ -637,13 +692,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.o_empty[a]);
       }
     }
-    if (!ok && leader) {  // no MMA of this warpgroup may still be writing TMEM at the exit
-      mma_commit(&sm.drain[a]);
-      mbar_wait(&sm.drain[a], 0, nullptr, nullptr);
-    }
-    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -188,6 +188,10 @@ hstu_status_t hstu_workspace_init(void* ws, size_t ws_bytes, hstu_stream_t strea
  * a compute call), clear it, and return it (HSTU_OK if no device-side check fired). */
 hstu_status_t hstu_sync_status(const void* ws, hstu_stream_t stream);
 
+/* Text of the last CUDA error this library saw on the calling thread ("" if none); useful
+ * after HSTU_ERR_CUDA.  The string stays valid until the thread's next library call. */
+const char* hstu_last_error_string(void);
+
 /* Human-readable name of a status code (static string). */
 const char* hstu_status_string(hstu_status_t status);
 
