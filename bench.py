@@ -103,7 +103,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(gpu_index)], stdout=subprocess.PIPE,
+                 "-lms", "50", "-i", str(gpu_index)], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -137,7 +137,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_layer_sample(wl, seconds_min=10.0, max_reps=3):
+def oracle_layer_sample(wl, seconds_min=12.0, max_reps=12):
     """The fp64 oracle on a bounded sample of the workload: one layer over its shortest
     sequence, repeated until seconds_min of CPU work.  Returns (tokens/s, sample, threads)."""
     from oracle import hstu_oracle as O
@@ -247,7 +247,7 @@ def run_attention_only(args, lib, Bd, desc, ly, x, y, ws, stream, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
@@ -452,7 +452,7 @@ def main():
         "attn_tflops": attn_tflops,
         "attn_ms_per_layer": attn_avg_ms,
         "stack_tflops": (L * (aflops + gemm_flops(wl))) / (ms_per_step / 1e3) / 1e12,
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel<64> (+ its work-list "
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_pair_kernel (+ its work-list "
                      "kernel, inside the same events)", "achieved": attn_tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": attn_tflops / peaks["bf16_tflops"],
