@@ -29,6 +29,8 @@ cudaError_t launch_attn_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                  const AttnGeom& g, __nv_bfloat16* out, int64_t ld_o, int grid,
                                  cudaStream_t stream);
 size_t attn_fwd_pair_smem(int P, bool has_pos);
+int attn_fwd_pair_kv_rows();
+int attn_fwd_pair_ts_box();
 cudaError_t launch_ln_gate(int dtype, const void* av, int64_t ld_av, const void* u, int64_t ld_u,
                            const float* gamma, const float* beta, float eps, void* g,
                            int64_t ld_g, int rows, int F, cudaStream_t stream);
@@ -236,14 +238,17 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
   if (tc) {
     CUtensorMap tq, tk, tv;
     const int64_t cols = static_cast<int64_t>(g.H) * D;
+    // the paired kernel streams K / V in shorter tiles than its query tiles
+    const uint32_t kv_rows = pair ? static_cast<uint32_t>(attn_fwd_pair_kv_rows()) : kTileRows;
     if (!make_map_bf16(&tq, q, T, cols, ld_q, 64, kTileRows) ||
-        !make_map_bf16(&tk, k, T, cols, ld_k, 64, kTileRows) ||
-        !make_map_bf16(&tv, v, T, cols, ld_v, 64, kTileRows))
+        !make_map_bf16(&tk, k, T, cols, ld_k, 64, kv_rows) ||
+        !make_map_bf16(&tv, v, T, cols, ld_v, 64, kv_rows))
       return HSTU_ERR_CUDA;
     if (pair) {
       CUtensorMap tts;
       std::memset(&tts, 0, sizeof(tts));
-      if (use_time && !make_map_i64_1d(&tts, g.ts, T, 136)) return HSTU_ERR_CUDA;
+      if (use_time && !make_map_i64_1d(&tts, g.ts, T, attn_fwd_pair_ts_box()))
+        return HSTU_ERR_CUDA;
       // persistent: one CTA per SM, each walking the work list with a stride
       const int pgrid = grid < num_sms_current() ? grid : num_sms_current();
       e = launch_attn_fwd_pair(tq, tk, tv, tts, g, static_cast<__nv_bfloat16*>(o), ld_o, pgrid,
