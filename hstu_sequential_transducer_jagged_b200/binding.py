@@ -29,6 +29,7 @@ EXPORTED = [
     "hstu_jagged_padded_copy",
     "hstu_debug_time_buckets", "hstu_workspace_init", "hstu_sync_status",
     "hstu_status_string", "hstu_version", "hstu_last_error_string",
+    "hstu_attention_forward_static_ws",
 ]
 
 
@@ -94,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_status_string": (ctypes.c_char_p, [i32]),
         "hstu_version": (ctypes.c_char_p, []),
         "hstu_last_error_string": (ctypes.c_char_p, []),
+        "hstu_attention_forward_static_ws": (i32, [adp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -209,6 +211,33 @@ def attention_forward(q, k, v, seq_offsets, max_seq_len, timestamps=None, rab_po
     _check(lib().hstu_attention_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                         ws.ptr, ws.nbytes, _stream_ptr(stream)),
            "hstu_attention_forward")
+    return out
+
+
+def attention_forward_static_ws(q, k, v, seq_offsets, max_seq_len, timestamps=None,
+                                rab_pos=None, rab_time=None, *, num_heads, max_pos_dist=0,
+                                num_time_buckets=1, alpha=1.0, mask=MASK_CAUSAL,
+                                num_candidates=0, microbatch=128, out=None, status_out=None,
+                                stream=None):
+    """O = hstu_attention_forward_static_ws(...): the attention forward on the library's
+    built-in scratch array instead of a workspace.  For callers that may not allocate device
+    memory while running; `out` (and `status_out`, a device int32 tensor) must then be passed in
+    preallocated.  Calls that overlap in time on one device race on the shared array."""
+    T = q.shape[0]
+    d = q.shape[1] // num_heads
+    if out is None:
+        out = torch.empty((T, v.shape[1]), dtype=q.dtype, device=q.device)
+    desc = attn_desc(seq_offsets=seq_offsets, total_tokens=T, max_seq_len=max_seq_len,
+                     timestamps=timestamps, num_heads=num_heads, d_qk=d, d_v=v.shape[1] // num_heads,
+                     ld_q=q.stride(0), ld_k=k.stride(0), ld_v=v.stride(0), ld_o=out.stride(0),
+                     mask=mask, num_candidates=num_candidates, microbatch=microbatch,
+                     rab_pos=rab_pos, max_pos_dist=max_pos_dist, rab_time=rab_time,
+                     num_time_buckets=num_time_buckets, alpha=alpha, dtype=_dtype_code(q))
+    st = lib().hstu_attention_forward_static_ws(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                                _ptr(out), _ptr(status_out), _stream_ptr(stream))
+    if st != HSTU_OK:
+        detail = lib().hstu_last_error_string().decode(errors="replace")
+        raise HstuError(st, f"hstu_attention_forward_static_ws ({detail})")
     return out
 
 

@@ -518,3 +518,81 @@ const char* hstu_version(void) { return "hstu_b200 0.1 sm_100a"; }
 const char* hstu_last_error_string(void) { return g_last_error; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- built-in scratch variant
+// The scratch of hstu_attention_forward_static_ws: a fixed array in every device context that
+// loads the library, so that call needs no workspace from its caller.
+static __device__ __align__(256) unsigned char g_static_scratch[HSTU_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of the current device's scratch array, looked up once per device.
+hstu_status_t static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxScratchDevices) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "device %d is beyond the %d devices the built-in scratch supports", dev,
+                  kMaxScratchDevices);
+    return HSTU_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (p == nullptr || (reinterpret_cast<uintptr_t>(p) % kAlign) != 0) {
+      std::snprintf(g_last_error, sizeof(g_last_error),
+                    "built-in scratch address is null or not %zu-byte aligned", kAlign);
+      return HSTU_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return HSTU_OK;
+}
+
+}  // namespace
+
+extern "C" hstu_status_t hstu_attention_forward_static_ws(const hstu_attn_desc_t* d,
+                                                          const void* q, const void* k,
+                                                          const void* v, void* o,
+                                                          int32_t* status_out,
+                                                          hstu_stream_t stream) {
+  // host-side argument checks first, so a bad call touches no device state
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
+                                  d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
+                                  d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
+                                  d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
+  if (st != HSTU_OK) return st;
+  if (status_out != nullptr && (reinterpret_cast<uintptr_t>(status_out) % 4) != 0)
+    return HSTU_ERR_INVALID_ARG;
+  const size_t need = hstu_attention_workspace_size(d);
+  if (need > HSTU_STATIC_SCRATCH_BYTES) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "attention forward needs %zu bytes of scratch, the built-in area holds %zu: "
+                  "use hstu_attention_forward with a caller workspace",
+                  need, static_cast<size_t>(HSTU_STATIC_SCRATCH_BYTES));
+    return HSTU_ERR_WORKSPACE;
+  }
+  void* ws = nullptr;
+  st = static_scratch(&ws);
+  if (st != HSTU_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents; only the status word must start at zero
+  cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = hstu_attention_forward(d, q, k, v, o, ws, HSTU_STATIC_SCRATCH_BYTES, stream);
+  if (st != HSTU_OK) return st;
+  if (status_out != nullptr) {
+    e = cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return HSTU_OK;
+}

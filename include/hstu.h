@@ -102,6 +102,33 @@ hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* desc, const void* q
                                      const void* k, const void* v, void* o, void* ws,
                                      size_t ws_bytes, hstu_stream_t stream);
 
+/* ---- Built-in scratch variant.  The pages define no such call: it is a library convenience.
+ * Size of the scratch area built into the library (one area per device). */
+#define HSTU_STATIC_SCRATCH_BYTES ((size_t)1 << 20)
+
+/* hstu_attention_forward without a caller workspace.  For callers that must not allocate device
+ * memory once they are running (a serving process whose memory is fully budgeted at start-up,
+ * an embedding application with no device allocator of its own, a host thread that may not
+ * take an allocator lock): the status word and the tile work list live in a fixed
+ * HSTU_STATIC_SCRATCH_BYTES array compiled into the library, so neither the caller nor the
+ * library allocates anything.
+ *   - Limit: the call needs hstu_attention_workspace_size(desc) bytes; above
+ *     HSTU_STATIC_SCRATCH_BYTES (about 65,000 work items: several million tokens) it returns
+ *     HSTU_ERR_WORKSPACE before any launch, and hstu_last_error_string() gives both sizes.
+ *   - Set-up: the first call on each device looks the array's device address up (with that
+ *     device current) and caches it; make that first call before any stream capture begins.
+ *   - Sharing: every call on a device uses the same array, which keeps the last call's contents;
+ *     each call zeroes the status word on its stream first (the work list is rebuilt in full).
+ *     Calls that overlap in time on one device (different streams or host threads without
+ *     ordering between them) race on the array and give undefined results: order them.
+ *   - status_out: optional device int32; when the stream reaches the end of the call it holds
+ *     the call's status word (0 when no device-side check fired, HSTU_ERR_TIMEOUT or
+ *     HSTU_ERR_DEVICE_CHECK otherwise).  NULL skips the copy.
+ * Every other argument and the result are those of hstu_attention_forward. */
+hstu_status_t hstu_attention_forward_static_ws(const hstu_attn_desc_t* desc, const void* q,
+                                               const void* k, const void* v, void* o,
+                                               int32_t* status_out, hstu_stream_t stream);
+
 /* Bytes of workspace hstu_attention_backward needs (adds an fp32 dQ accumulator [T,H,d_qk]). */
 size_t hstu_attention_backward_workspace_size(const hstu_attn_desc_t* desc);
 

@@ -139,3 +139,21 @@ def test_misc_entry_points_validate(lib):
     assert lib.hstu_jagged_padded_copy(FAKE, 0, 8, FAKE, 32, FAKE, 32, 32, 1, None) == 0
     assert lib.hstu_sync_status(ctypes.c_void_p((1 << 20) + 8), None) == 3
     assert lib.hstu_workspace_init(None, 256, None) == 3
+
+
+def test_static_scratch_call_rejects_on_the_host(lib):
+    # the built-in scratch call checks its arguments and its size limit before touching CUDA
+    assert lib.hstu_attention_forward_static_ws(None, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.hstu_attention_forward_static_ws(ctypes.byref(_desc(mask=7)), FAKE, FAKE, FAKE,
+                                                FAKE, None, None) == 1
+    assert lib.hstu_attention_forward_static_ws(ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE,
+                                                ctypes.c_void_p((1 << 20) + 2), None) == 1
+    limit = 1 << 20  # HSTU_STATIC_SCRATCH_BYTES
+    assert f"HSTU_STATIC_SCRATCH_BYTES ((size_t)1 << 20)" in open(HEADER).read()
+    big = _desc(num_seqs=100000, total_tokens=100000, max_seq_len=1)
+    need = lib.hstu_attention_workspace_size(ctypes.byref(big))
+    assert need > limit
+    assert lib.hstu_attention_forward_static_ws(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, None,
+                                                None) == 3
+    msg = lib.hstu_last_error_string().decode()
+    assert str(need) in msg and str(limit) in msg
