@@ -7,16 +7,17 @@
 // softmax and no normalisation, "HSTU：Scaling Law 的首次探索" §7.1.4 innovation 1; causal mask,
 // or the M-FALCON candidate mask of §7.1.5.)
 //
-// A work item is two 128-row query tiles of one sequence and head; keys and values stream
-// through in 64-row tiles (TMA, 6-stage ring, the tile's timestamps with them) that both query
-// tiles use.  Each query tile owns two S buffers and two P buffers in tensor memory: while its
+// A work item is two 128-row query tiles of one sequence and head (Q double-buffered, so the
+// next item's Q arrives while this one runs); keys and values stream through in 64-row tiles
+// (TMA, 6-stage ring, the tile's timestamps with them) that both query tiles use.  Each query tile owns two S buffers and two P buffers in tensor memory: while its
 // epilogue warpgroup turns S(k) into P(k), the tensor core already holds S(k+1), and S(k+2) is
 // issued into the buffer S(k) leaves as soon as P(k) is written, so an epilogue warpgroup does
 // not wait for the MMA chain and the two warpgroups keep the SFU (the SiLU's tanh) busy.
 //
-// Warpgroup 0: warp 0 TMA producer; warp 1 TMEM allocation and single-thread tcgen05.mma issue
-// (a thread that issues MMAs stalls about as long as they execute, so issue stays off the
-// epilogue warps); warp 2 timestamps (per KV tile: min / max and int32 copies); warp 3 spare.
+// Warpgroup 0: warp 0 TMA producer; warps 1 and 3 issue the tcgen05.mma of query tile 0 and 1
+// (one thread each: a thread waits about 50 cycles per MMA it issues and over 100 per commit or
+// barrier check, so two issuers overlap those waits, and issue stays off the epilogue warps);
+// warp 1 also owns the TMEM allocation; warp 2 timestamps (per KV tile: min / max, int32 copies).
 // Warpgroups 1 and 2: one epilogue warpgroup per query tile (warp w owns TMEM lanes
 // 32*(w%4) .. +31, one query row per thread).  setmaxnreg moves registers from warpgroup 0
 // (88) to the epilogue warpgroups (208).
@@ -48,7 +49,7 @@ constexpr int kD = 64;
 constexpr int kQ = kTileRows;           // query tile rows (128)
 constexpr int kKV = 64;                 // key/value tile rows
 constexpr int kStages = 6;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;          // 5 warpgroups
 constexpr int kQBytes = kQ * kD * 2;    // 16 KB, 128-byte swizzle
 constexpr int kKVBytes = kKV * kD * 2;  // 8 KB
 constexpr int kTsBox = 72;              // timestamps loaded per KV tile (x rounded down to even)
@@ -60,23 +61,25 @@ __device__ __forceinline__ uint32_t col_p(int a, int b) { return 256u + 32u * (2
 __device__ __forceinline__ uint32_t col_o(int a) { return 384u + 64u * a; }
 
 struct PairSmem {
-  alignas(1024) uint8_t q[2][kQBytes];
+  alignas(1024) uint8_t q[2][2][kQBytes];  // [item slot][query tile]
   alignas(1024) uint8_t k[kStages][kKVBytes];
   alignas(1024) uint8_t v[kStages][kKVBytes];
   alignas(128) long long ts[kStages][kTsStride];
   alignas(16) int ts32[kStages][kKV];   // low 32 bits of the tile's timestamps
   float rab_time_h[kTimeSmem];           // 0.5 x rab_time, index clamped to NB - 1
-  long long tmin[kStages];               // min / max timestamp of the tile's in-sequence columns
-  long long tmax[kStages];
-  uint64_t q_full, q_empty;
+  long long tmin[kStages][2];            // min / max timestamp of each 32-column half's
+  long long tmax[kStages][2];            // in-sequence columns
+  int2 cls[kStages][16];                 // per (query tile, row quarter, half): mode, bias
+  long long rows_t[8][2];                // per (query tile, row quarter): min / max t_i
+  uint64_t q_full[2], q_empty[2];        // per item slot
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t ts_ready[kStages];
+  uint64_t cls_ready[kStages];           // the tile's classification and timestamps
   uint64_t s_full[2][2];
   uint64_t p_full[2][2];
   uint64_t o_full[2];
   uint64_t o_empty[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort_flag;
   // followed by float4 pos4[2P + 4]: 0.5 x (tab[x], tab[x-1], tab[x-2], tab[x-3]), clamped
@@ -125,12 +128,6 @@ struct PairPlan {
   }
   // (selects instead of indexing by a runtime a keep the plan in registers)
   __device__ __forceinline__ KvRange64 range(int a) const { return a == 0 ? r[0] : r[1]; }
-  __device__ __forceinline__ bool member(int a, int u) const {
-    const KvRange64 ra = range(a);
-    const int ba = a == 0 ? base[0] : base[1];
-    if (!(a == 0 ? valid[0] : valid[1])) return false;
-    return u < nhm ? (u < ra.nh) : (u >= ba && u < ba + ra.nd);
-  }
   __device__ __forceinline__ int count(int a) const {
     const KvRange64 ra = range(a);
     return (a == 0 ? valid[0] : valid[1]) ? ra.nh + ra.nd : 0;
@@ -197,208 +194,180 @@ __device__ __forceinline__ float time_term32(const float* time_h, int d) {
 
 __device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_fast(h), h); }
 
-// Per-row constants of one KV tile's epilogue.  The mode and the per-element switches are
-// warp-uniform (a warp takes a per-element path for all of its rows when any row needs it; the
-// per-element formulas are exact for every row), so no branch in the epilogue diverges.
+// Per-row constants of one 32-column segment's epilogue.  The mode and the time-term kind are
+// warp-uniform: a warp takes the per-element path for all of its rows when any row needs it
+// (the per-element formulas are exact for every row), so no branch in the epilogue diverges.
 struct RowCtx {
   float half_alpha;
-  float half_bias;   // 0.5 x (the parts of the bias that are constant along the row segment)
-  bool pos_elem;     // position term per element from pos4
-  bool mask;         // causal mask inside the segment (diagonal tiles)
-  int pbase;         // pos4 index of column c is clamp(pbase - c, 0, 2P+3)
+  float half_bias;   // 0.5 x (the parts of the bias that are constant along the segment)
+  int pbase;         // pos4 index of tile column c is clamp(pbase - c, 0, 2P+3)
   int time_mode;     // 0 constant, 1 threshold (<= 2 buckets), 2 per element 32-bit, 3 64-bit
   int thr;
   float t_lo, t_hi;
   int ti_lo;
   long long ti;
   int pi_plus_p, P2, nbm1;
-  int i, n, c0l;
+  int i, n, c0t;     // query row, history length, first column of the KV tile
   bool row_valid;
-  int mode;          // 0 constant bias, 1 per-element bias (+ causal mask), 2 general
+  int mode;          // kModeConst, kModeElem, kModeGeneral or kModeZero
 };
 
-// 0.5 x bias of columns ch*32 .. ch*32+31 (modes 1 and 2).
-template <int MODE>
-__device__ __forceinline__ void chunk_bias(float (&b)[32], int ch, const RowCtx& rc,
-                                           const float4* pos4, const float* time_h,
-                                           const int* ts32, const long long* ts, bool use_pos) {
-  if (MODE == 1) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) b[e] = rc.half_bias;
-    if (rc.pos_elem) {
-#pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 pv = pos4[clampi(rc.pbase - (ch * 32 + e), 0, rc.P2 + 3)];
-        b[e] += pv.x;
-        b[e + 1] += pv.y;
-        b[e + 2] += pv.z;
-        b[e + 3] += pv.w;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      b[e] = 0.f;
-      if (use_pos) {
-        const int j = rc.c0l + ch * 32 + e;  // candidate keys (j >= n) sit at position n
-        b[e] = pos4[clampi(rc.pi_plus_p - (j < rc.n ? j : rc.n), 0, rc.P2)].x;
-      }
-    }
-  }
-  if (rc.time_mode == 1) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      const int4 tv = *reinterpret_cast<const int4*>(ts32 + ch * 32 + e);
-      b[e] += (rc.ti_lo - tv.x >= rc.thr) ? rc.t_hi : rc.t_lo;
-      b[e + 1] += (rc.ti_lo - tv.y >= rc.thr) ? rc.t_hi : rc.t_lo;
-      b[e + 2] += (rc.ti_lo - tv.z >= rc.thr) ? rc.t_hi : rc.t_lo;
-      b[e + 3] += (rc.ti_lo - tv.w >= rc.thr) ? rc.t_hi : rc.t_lo;
-    }
-  } else if (rc.time_mode == 2) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      const int4 tv = *reinterpret_cast<const int4*>(ts32 + ch * 32 + e);
-      b[e] += time_term32(time_h, rc.ti_lo - tv.x);
-      b[e + 1] += time_term32(time_h, rc.ti_lo - tv.y);
-      b[e + 2] += time_term32(time_h, rc.ti_lo - tv.z);
-      b[e + 3] += time_term32(time_h, rc.ti_lo - tv.w);
-    }
-  } else if (rc.time_mode == 3) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      b[e] += time_h[time_bucket64(rc.ti - ts[ch * 32 + e], rc.nbm1 + 1)];
-  }
-}
+constexpr int kModeConst = 0;    // one bias value per row
+constexpr int kModeElem = 1;     // position term per element (+ time term), nothing masked
+constexpr int kModeCausal = 2;   // as kModeElem, with the causal diagonal masked
+constexpr int kModeGeneral = 3;  // M-FALCON candidates: everything per element, 64-bit time
+constexpr int kModeZero = 4;     // every entry masked
 
-// One 32-column chunk: P = SiLU(alpha S + bias) as packed bf16, masked entries zero.
-template <int MODE>
-__device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&pk)[16], int ch,
-                                           const RowCtx& rc, const float4* pos4,
-                                           const float* time_h, const int* ts32,
-                                           const long long* ts, bool use_pos) {
-  if (MODE == 0) {
+// P = SiLU(alpha S + bias) for the 32 columns h*32 .. h*32+31 of the tile, as packed bf16.
+// TM is the time term's kind: 0 constant (in half_bias), 1 threshold, 2 per element from the
+// 32-bit differences, 3 per element from the 64-bit differences.
+template <int MODE, int TM>
+__device__ __forceinline__ void silu_seg(const uint32_t (&s)[32], uint32_t (&pk)[16], int h,
+                                         const RowCtx& rc, const float4* pos4,
+                                         const float* time_h, const int* ts32,
+                                         const long long* ts) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2)
-      pk[e >> 1] =
-          pack_bf16x2(silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e]), rc.half_bias)),
-                      silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e + 1]), rc.half_bias)));
-  } else {
-    float b[32];
-    chunk_bias<MODE>(b, ch, rc, pos4, time_h, ts32, ts, use_pos);
-    if (MODE == 1 && !rc.mask) {
+  for (int q = 0; q < 32; q += 4) {
+    const int c = h * 32 + q;  // column of the first of these 4 within the KV tile
+    float bb[4];
+    if (MODE == kModeConst) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 2)
-        pk[e >> 1] =
-            pack_bf16x2(silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e]), b[e])),
-                        silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e + 1]), b[e + 1])));
+      for (int u = 0; u < 4; ++u) bb[u] = rc.half_bias;
+    } else if (MODE == kModeElem || MODE == kModeCausal) {
+      // exact for every row: beyond the band the clamped table repeats its last entry
+      const float4 pv = pos4[clampi(rc.pbase - c, 0, rc.P2 + 3)];
+      bb[0] = rc.half_bias + pv.x;
+      bb[1] = rc.half_bias + pv.y;
+      bb[2] = rc.half_bias + pv.z;
+      bb[3] = rc.half_bias + pv.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float pv[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int j = rc.c0l + ch * 32 + e + u;
-          const float p = silu_half(fmaf(rc.half_alpha, __uint_as_float(s[e + u]), b[e + u]));
-          bool vis = j <= rc.i;
-          if (MODE == 2) vis = rc.row_valid && vis && (j < rc.n || j == rc.i);
-          pv[u] = vis ? p : 0.f;
-        }
-        pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+      for (int u = 0; u < 4; ++u) {
+        const int j = rc.c0t + c + u;  // candidate keys (j >= n) sit at position n
+        bb[u] = pos4[clampi(rc.pi_plus_p - (j < rc.n ? j : rc.n), 0, rc.P2)].x;
       }
     }
+    if (TM == 1 || TM == 2) {
+      const int4 tv = *reinterpret_cast<const int4*>(ts32 + c);
+      const int d[4] = {rc.ti_lo - tv.x, rc.ti_lo - tv.y, rc.ti_lo - tv.z, rc.ti_lo - tv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        bb[u] += TM == 1 ? (d[u] >= rc.thr ? rc.t_hi : rc.t_lo) : time_term32(time_h, d[u]);
+    } else if (TM == 3) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) bb[u] += time_h[time_bucket64(rc.ti - ts[c + u], rc.nbm1 + 1)];
+    }
+    float p[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      p[u] = silu_half(fmaf(rc.half_alpha, __uint_as_float(s[q + u]), bb[u]));
+      const int j = rc.c0t + c + u;
+      if (MODE == kModeCausal) p[u] = j <= rc.i ? p[u] : 0.f;
+      if (MODE == kModeGeneral) {
+        const bool vis = rc.row_valid && j <= rc.i && (j < rc.n || j == rc.i);
+        p[u] = vis ? p[u] : 0.f;
+      }
+    }
+    pk[q >> 1] = pack_bf16x2(p[0], p[1]);
+    pk[(q >> 1) + 1] = pack_bf16x2(p[2], p[3]);
   }
 }
 
-// S (TMEM, the 64 columns of this thread's row) -> P (TMEM, bf16); the second load overlaps the
-// first chunk's math.
-template <int MODE>
-__device__ __forceinline__ void tile_epilogue(uint32_t s_addr, uint32_t p_addr, const RowCtx& rc,
-                                              const float4* pos4, const float* time_h,
-                                              const int* ts32, const long long* ts, bool use_pos) {
-  uint32_t b0[32], b1[32];
+// S (TMEM, this warp's 32 columns of its rows) -> P (TMEM, bf16).
+template <int MODE, int TM>
+__device__ __forceinline__ void seg_epilogue(uint32_t s_addr, uint32_t p_addr, int h,
+                                             const RowCtx& rc, const float4* pos4,
+                                             const float* time_h, const int* ts32,
+                                             const long long* ts) {
+  uint32_t s[32];
   uint32_t pk[16];
-  tmem_ld32(s_addr, b0);
-  tmem_wait_ld_regs(b0);
-  tmem_ld32(s_addr + 32, b1);
-  silu_chunk<MODE>(b0, pk, 0, rc, pos4, time_h, ts32, ts, use_pos);
+  tmem_ld32(s_addr, s);
+  tmem_wait_ld_regs(s);
+  silu_seg<MODE, TM>(s, pk, h, rc, pos4, time_h, ts32, ts);
   tmem_st16(p_addr, pk);
-  tmem_wait_ld_regs(b1);
-  silu_chunk<MODE>(b1, pk, 1, rc, pos4, time_h, ts32, ts, use_pos);
-  tmem_st16(p_addr + 16, pk);
 }
 
-// Bias classification of this thread's row segment [c0l, c0l + 64).  Passed and returned by
-// value so the context stays in registers.
-__device__ __forceinline__ RowCtx classify_segment(RowCtx rc, int c0l, int i, int n, int pi,
-                                                   long long ti, bool row_valid, bool use_pos,
-                                                   bool use_time, int P, int NB,
-                                                   long long tmin, long long tmax,
-                                                   const float4* pos4, const float* time_h) {
-  const int last = c0l + kKV - 1;
-  const bool cand = row_valid && i >= n && last >= n;  // a candidate row meets candidate keys
-  const bool need_mask = row_valid && last > i;
-  const bool pos_elem = use_pos && row_valid && !(pi - last >= P);
-  bool fits32 = true, multi = false;
-  int b_lo = 0, b_hi = 0;
-  if (use_time) {
-    const long long dt_lo = ti - tmax;
-    const long long dt_hi = ti - tmin;
-    fits32 = !row_valid || (dt_hi < (1ll << 23) && dt_lo > -(1ll << 23));
-    b_lo = fits32 ? bucket_small(static_cast<int>(dt_lo), NB - 1) : time_bucket64(dt_lo, NB);
-    b_hi = fits32 ? bucket_small(static_cast<int>(dt_hi), NB - 1) : time_bucket64(dt_hi, NB);
-    multi = row_valid && b_hi > b_lo + 1;
+// Mode and bias of one (query tile, 32-row quarter, 32-column half) segment of a KV tile,
+// decided by the classifier warp from the quarter's row ranges, so exact for every row:
+// all entries masked; some entry masked or a candidate row meeting candidate keys (general);
+// every key beyond the position clamp and every (row, key) pair in one time bucket (constant);
+// else per element.  cls.x = mode | time-constant flag << 2, cls.y = 0.5 x the constant terms.
+struct QuarterRows {
+  int i0, i1;            // first and last valid row (i1 < i0: none)
+  int pmin;              // smallest position among them
+  long long tlo, thi;    // their timestamp range
+};
+
+__device__ __forceinline__ int2 classify_quarter(const QuarterRows& q, int c0, int n, int P,
+                                                 bool use_pos, bool use_time, int NB,
+                                                 long long tmin, long long tmax,
+                                                 const float4* pos4, int P2,
+                                                 const float* time_h) {
+  const int last = c0 + 31;
+  int mode;
+  if (q.i1 < q.i0 || c0 > q.i1) {
+    mode = kModeZero;
+  } else if (q.i1 >= n && last >= n) {
+    mode = kModeGeneral;   // a candidate row meets candidate keys
+  } else if (last > q.i0) {
+    mode = kModeCausal;    // the causal diagonal (keys past the sequence are past it too)
+  } else {
+    mode = (use_pos && q.pmin - last < P) ? kModeElem : kModeConst;
   }
-  const bool w_cand = __any_sync(0xffffffffu, cand);
-  const bool w_mask = __any_sync(0xffffffffu, need_mask);
-  const bool w_pos = __any_sync(0xffffffffu, pos_elem);
-  const bool w_tvar = __any_sync(0xffffffffu, row_valid && b_hi != b_lo);
-  const bool w_multi = __any_sync(0xffffffffu, multi);
-  const bool w_fits = __all_sync(0xffffffffu, fits32);
-  float hbias = 0.f;
-  if (use_pos && !w_pos) hbias = pos4[2 * P].x;  // every valid row is beyond the clamp
+  bool tconst = true;
+  float hb = 0.f;
+  if (use_time && mode != kModeZero && mode != kModeGeneral) {
+    // tmin / tmax cover the half's in-sequence keys, every key a row can see
+    const int b_lo = time_bucket64(q.tlo - tmax, NB);
+    const int b_hi = time_bucket64(q.thi - tmin, NB);
+    tconst = b_lo == b_hi;
+    if (tconst) hb = time_h[b_lo];
+    else if (mode == kModeConst) mode = kModeElem;
+  }
+  if (mode == kModeConst) hb += pos4[P2 + 3].x;  // beyond the clamp: the table's last entry
+  return make_int2(mode | (tconst ? 8 : 0), __float_as_int(hb));
+}
+
+// The per-row part of a segment's set-up: the time term's kind when the quarter's rows do not
+// share one bucket (threshold when every row spans at most two buckets, else per element), and
+// the row constants.  Passed and returned by value so the context stays in registers.
+__device__ __forceinline__ RowCtx segment_ctx(RowCtx rc, int2 cls, int c0t, int h, long long ti,
+                                              bool row_valid, bool use_time, int NB,
+                                              const long long* tmin, const long long* tmax,
+                                              const float* time_h) {
+  int mode = cls.x & 7;
+  const bool tconst = (cls.x & 8) != 0;
   int tm = 0;
-  if (use_time) {
-    if (!w_tvar) {
-      hbias += time_h[b_lo];                       // one bucket for each valid row
-    } else if (!w_multi && w_fits) {
-      tm = 1;                                      // at most two buckets per row
-      rc.thr = 1 << (b_lo + 1);
-      rc.t_lo = time_h[b_lo];
-      rc.t_hi = time_h[b_hi];
+  if (use_time && !tconst) {
+    const long long dt_lo = ti - *tmax;
+    const long long dt_hi = ti - *tmin;
+    const bool fits32 = !row_valid || (dt_hi < (1ll << 23) && dt_lo > -(1ll << 23));
+    const bool w_fits = __all_sync(0xffffffffu, fits32);
+    if (w_fits) {
+      const int b_lo = bucket_small(static_cast<int>(dt_lo), NB - 1);
+      const int b_hi = bucket_small(static_cast<int>(dt_hi), NB - 1);
+      const bool w_multi = __any_sync(0xffffffffu, row_valid && b_hi > b_lo + 1);
+      if (!w_multi) {
+        tm = 1;
+        rc.thr = 1 << (b_lo + 1);
+        rc.t_lo = time_h[b_lo];
+        rc.t_hi = time_h[b_hi];
+      } else {
+        tm = 2;
+      }
     } else {
-      tm = w_fits ? 2 : 3;
+      tm = 3;
     }
   }
-  rc.c0l = c0l;
-  rc.pos_elem = w_pos;
-  rc.mask = w_mask;
-  rc.pbase = pi - c0l + P;
+  if (mode == kModeGeneral) tm = use_time ? 3 : 0;
+  // 64-bit differences: the general path (its visibility rule is exact for the causal mask too)
+  if (tm == 3) mode = kModeGeneral;
+  rc.c0t = c0t;
+  rc.pbase = rc.pi_plus_p - c0t;
   rc.time_mode = tm;
-  rc.half_bias = hbias;
-  rc.mode = w_cand ? 2 : ((w_pos || w_mask || tm != 0) ? 1 : 0);
-  if (rc.mode == 2) rc.time_mode = use_time ? (w_fits ? 2 : 3) : 0;
+  rc.half_bias = __int_as_float(cls.y);
+  rc.mode = mode;
   return rc;
-}
-
-// S = Q Kᵀ for a 128 x 64 tile (4 MMAs of K = 16), completion signalled on bar.
-__device__ __forceinline__ void issue_s_mma(uint32_t d_tmem, uint32_t qb, uint32_t kb,
-                                            uint64_t* bar) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, kKV, 0, 0);
-#pragma unroll
-  for (int kk = 0; kk < kD / 16; ++kk)
-    mma_bf16_ss(d_tmem, smem_desc_sw128(qb + kk * 32, 16, 1024),
-                smem_desc_sw128(kb + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-  mma_commit(bar);
-}
-
-// O (+)= P V with P (bf16, 128 x 64) read from TMEM and V (MN-major) from shared memory.
-__device__ __forceinline__ void issue_pv_mma(uint32_t o_tmem, uint32_t p_tmem, uint32_t vb,
-                                             bool acc) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, kD, 0, 1);
-#pragma unroll
-  for (int kk = 0; kk < kKV / 16; ++kk)
-    mma_bf16_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, kKVBytes, 1024), idesc,
-                (acc || kk > 0) ? 1u : 0u);
 }
 
 // Wait by one lane of the warp, then release the warp (the barrier's data is then visible to
@@ -407,6 +376,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
                                           int* status) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// warp_wait on two barriers; both probes are issued before either result is needed.
+__device__ __forceinline__ bool warp_wait2(uint64_t* bar1, uint32_t parity1, uint64_t* bar2,
+                                           uint32_t parity2, volatile int* abort, int* status) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    const bool p1 = mbar_try_wait(bar1, parity1);
+    const bool p2 = mbar_try_wait(bar2, parity2);
+    if (!p1) ok = mbar_wait(bar1, parity1, abort, status);
+    if (ok && !p2) ok = mbar_wait(bar2, parity2, abort, status);
+  }
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -419,42 +401,44 @@ __device__ __forceinline__ void tma_load_1d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// MMA-warp state of one query tile: S issued (gs) and P consumed (gp) in total (the buffers
-// alternate across items), S issued and PV done in the current item, items with output (oc).
-struct MmaTileState {
-  int gs, gp, issued, done, oc;
+// Issuer-side constants of one query tile: shared-memory descriptors of the first K and V
+// stages and of the Q tile (a stage's descriptor adds stage x 512, the stage size >> 4), the
+// tensor-memory columns, and the barriers.  Computed once so that the single issuing thread
+// does no address arithmetic between MMAs.
+struct IssuerCtx {
+  uint64_t dq[2], dk0, dv0;        // dq per item slot
+  uint32_t s_col0, p_col0, o_col;  // buffer 1 lies 64 (S) or 32 (P) columns further
+  uint64_t* s_full0;               // buffer 1's barriers follow buffer 0's
+  uint64_t* p_full0;
+  uint64_t* o_full;
+  uint64_t* o_empty;
+  uint64_t* kv_full;
 };
 
-// The PV of query tile a's current tile, then its S two tiles ahead (into the buffer just
-// freed), and the output commit after its last tile.
-__device__ __forceinline__ bool mma_step(PairSmem& sm, uint32_t tmem, const PairPlan& plan,
-                                         int gu, int a, int st, MmaTileState& t,
-                                         volatile int* abort_flag, int* status) {
-  const int b = t.gp & 1;
-  bool ok = mbar_wait(&sm.p_full[a][b], (t.gp >> 1) & 1, abort_flag, status);
-  ++t.gp;
-  if (ok && t.done == 0 && t.oc > 0)
-    ok = mbar_wait(&sm.o_empty[a], (t.oc - 1) & 1, abort_flag, status);
-  if (!ok) return false;
-  tc_fence_after();
-  issue_pv_mma(tmem + col_o(a), tmem + col_p(a, b), smem_u32(sm.v[st]), t.done > 0);
-  ++t.done;
-  if (t.issued < plan.count(a)) {
-    const int u2 = gu + plan.uidx(a, t.issued);
-    if (!mbar_wait(&sm.kv_full[u2 % kStages], (u2 / kStages) & 1, abort_flag, status)) return false;
-    tc_fence_after();
-    const int bs = t.gs & 1;
-    issue_s_mma(tmem + col_s(a, bs), smem_u32(sm.q[a]), smem_u32(sm.k[u2 % kStages]),
-                &sm.s_full[a][bs]);
-    ++t.gs;
-    ++t.issued;
-  }
-  if (t.done == plan.count(a)) mma_commit(&sm.o_full[a]);
-  return true;
+constexpr uint32_t kStageDesc = kKVBytes >> 4;  // descriptor step between K (or V) stages
+static_assert(sizeof(PairSmem::k[0]) == kKVBytes && sizeof(PairSmem::v[0]) == kKVBytes,
+              "K and V stages are contiguous");
+
+__device__ __forceinline__ void issue_s(const IssuerCtx& c, uint64_t dq, int bs, int st) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, kKV, 0, 0);
+  const uint64_t dk = c.dk0 + static_cast<uint64_t>(st) * kStageDesc;
+#pragma unroll
+  for (int kk = 0; kk < kD / 16; ++kk)
+    mma_bf16_ss(c.s_col0 + 64u * bs, dq + 2 * kk, dk + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+  mma_commit(c.s_full0 + bs);
 }
 
-// 12 warps launch with 168 registers each (3 warps per SM sub-partition); after set-up
-// warpgroup 0 drops to 88 and the epilogue warpgroups rise to 208 (88 + 2 x 208 = 3 x 168).
+__device__ __forceinline__ void issue_pv(const IssuerCtx& c, int b, int st, bool acc) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, kD, 0, 1);
+  const uint64_t dv = c.dv0 + static_cast<uint64_t>(st) * kStageDesc;
+#pragma unroll
+  for (int kk = 0; kk < kKV / 16; ++kk)
+    mma_bf16_ts(c.o_col, c.p_col0 + 32u * b + kk * 8, dv + 128 * kk, idesc,
+                (acc || kk > 0) ? 1u : 0u);
+}
+
+// 20 warps launch with 96 registers each (5 warps per SM sub-partition); after set-up
+// warpgroup 0 drops to 64 and the four epilogue warpgroups rise to 104 (64 + 4 x 104 = 5 x 96).
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -476,32 +460,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- one-time setup: tables, barriers, TMEM
-  if (use_pos) {
-    const int P2 = 2 * g.P;
-    for (int x = threadIdx.x; x <= P2 + 3; x += kThreads)
-      pos4[x] = make_float4(0.5f * g.rab_pos[clampi(x, 0, P2)], 0.5f * g.rab_pos[clampi(x - 1, 0, P2)],
-                            0.5f * g.rab_pos[clampi(x - 2, 0, P2)], 0.5f * g.rab_pos[clampi(x - 3, 0, P2)]);
-  }
+  // (without a position table pos4 holds 4 zero entries, so the per-element path adds 0)
+  const int P2 = use_pos ? 2 * g.P : 0;
+  for (int x = threadIdx.x; x <= P2 + 3; x += kThreads)
+    pos4[x] = use_pos ? make_float4(0.5f * g.rab_pos[clampi(x, 0, P2)],
+                                    0.5f * g.rab_pos[clampi(x - 1, 0, P2)],
+                                    0.5f * g.rab_pos[clampi(x - 2, 0, P2)],
+                                    0.5f * g.rab_pos[clampi(x - 3, 0, P2)])
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
   if (use_time)
     for (int e = threadIdx.x; e < kTimeSmem; e += kThreads)
       sm.rab_time_h[e] = 0.5f * g.rab_time[e < g.NB ? e : g.NB - 1];
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
+    for (int sl = 0; sl < 2; ++sl) {
+      mbar_init(&sm.q_full[sl], 1);
+      mbar_init(&sm.q_empty[sl], 2);  // both issuers
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
-      mbar_init(&sm.ts_ready[s], 1);
+      mbar_init(&sm.kv_empty[s], 2);  // one release per query tile
+      mbar_init(&sm.cls_ready[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sm.s_full[a][b], 1);
-        mbar_init(&sm.p_full[a][b], 4);  // one elected lane per epilogue warp
+        mbar_init(&sm.p_full[a][b], 8);  // one elected lane per epilogue warp of tile a
       }
       mbar_init(&sm.o_full[a], 1);
-      mbar_init(&sm.o_empty[a], 4);
+      mbar_init(&sm.o_empty[a], 8);
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain[0], 1);
+    mbar_init(&sm.drain[1], 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -517,30 +506,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int stride = static_cast<int>(gridDim.x);
 
   if (warp < 4) {
-    setmaxnreg_dec<88>();
+    setmaxnreg_dec<64>();
     if (warp == 0) {
       // ============================================================ producer
       if (lane == 0) {
         int gu = 0;  // KV tiles issued by this CTA so far
         int qi = 0;  // work items so far
+        int qn = 0;  // Q loads issued
         bool ok = true;
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         if (use_time) tma_prefetch_desc(&tm_ts);
+        WorkItem nxt = g.items[blockIdx.x / g.H];  // the next item is loaded one item ahead
         for (int w = blockIdx.x; ok && w < total; w += stride, ++qi) {
-          const WorkItem it = g.items[w / g.H];
+          const WorkItem it = nxt;
+          if (w + stride < total) nxt = g.items[(w + stride) / g.H];
           const int head = w % g.H;
           const PairPlan plan =
               make_plan(it.qtile, it.len, hist_len(it.len, g.mask, g.num_candidates));
-          if (qi > 0 && !mbar_wait(&sm.q_empty, (qi - 1) & 1, abort_flag, g.status)) {
+          const int sl = qi & 1;
+          if (qi > 1 && !mbar_wait(&sm.q_empty[sl], ((qi >> 1) - 1) & 1, abort_flag, g.status)) {
             ok = false;
             break;
           }
           const int nq = plan.valid[1] ? 2 : 1;
-          mbar_arrive_expect_tx(&sm.q_full, nq * kQBytes);
+          mbar_arrive_expect_tx(&sm.q_full[sl], nq * kQBytes);
           for (int a = 0; a < nq; ++a)
-            tma_load_2d(sm.q[a], &tm_q, &sm.q_full, head * kD, it.row0 + plan.q[a] * kQ);
+            tma_load_2d(sm.q[sl][a], &tm_q, &sm.q_full[sl], head * kD, it.row0 + plan.q[a] * kQ);
+          ++qn;
           for (int u = 0; u < plan.nU; ++u, ++gu) {
             const int st = gu % kStages;
             if (gu >= kStages &&
@@ -558,88 +552,146 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) {  // leave no TMA write in flight into shared memory about to be released
           for (int u = (gu > kStages ? gu - kStages : 0); u < gu; ++u)
             mbar_wait(&sm.kv_full[u % kStages], (u / kStages) & 1, nullptr, nullptr);
-          if (qi > 0) mbar_wait(&sm.q_full, (qi - 1) & 1, nullptr, nullptr);
+          for (int q2 = (qn > 2 ? qn - 2 : 0); q2 < qn; ++q2)
+            mbar_wait(&sm.q_full[q2 & 1], (q2 >> 1) & 1, nullptr, nullptr);
         }
       }
       __syncwarp();
-    } else if (warp == 1) {
-      // ============================================================ MMA issuer
+    } else if (warp == 1 || warp == 3) {
+      // ============================================================ MMA issuers
+      // Query tile a's issuer walks every KV tile of each item in load order: for its own tiles
+      // it issues PV and the S two tiles ahead; for the other tile's (candidate) tiles it waits
+      // until the stage is loaded and releases it at once, so that neither side can release a
+      // stage's next fill before its current one.  The epilogue of query tile a releases the
+      // stages of its own tiles once their PV has completed.
       if (lane == 0) {
-        int gu = 0, qi = 0;
-        MmaTileState t0{0, 0, 0, 0, 0}, t1{0, 0, 0, 0, 0};
+        const int a = warp == 1 ? 0 : 1;
+        IssuerCtx c;
+        c.dq[0] = smem_desc_sw128(smem_u32(sm.q[0][a]), 16, 1024);
+        c.dq[1] = smem_desc_sw128(smem_u32(sm.q[1][a]), 16, 1024);
+        c.dk0 = smem_desc_sw128(smem_u32(sm.k[0]), 16, 1024);
+        c.dv0 = smem_desc_sw128(smem_u32(sm.v[0]), kKVBytes, 1024);
+        c.s_col0 = tmem + col_s(a, 0);
+        c.p_col0 = tmem + col_p(a, 0);
+        c.s_full0 = &sm.s_full[a][0];
+        c.p_full0 = &sm.p_full[a][0];
+        c.o_col = tmem + col_o(a);
+        c.o_full = &sm.o_full[a];
+        c.o_empty = &sm.o_empty[a];
+        c.kv_full = sm.kv_full;
+        int gu = 0, qi = 0, gs = 0, gp = 0, oc = 0;
         bool ok = true;
+        WorkItem nxt = g.items[blockIdx.x / g.H];  // the next item is loaded one item ahead
         for (int w = blockIdx.x; ok && w < total; w += stride, ++qi) {
-          const WorkItem it = g.items[w / g.H];
+          const WorkItem it = nxt;
+          if (w + stride < total) nxt = g.items[(w + stride) / g.H];
           const PairPlan plan =
               make_plan(it.qtile, it.len, hist_len(it.len, g.mask, g.num_candidates));
-          ok = mbar_wait(&sm.q_full, qi & 1, abort_flag, g.status);
-          t0.issued = t0.done = t1.issued = t1.done = 0;
-          // prologue: the first two S of each query tile (the epilogue read their buffers'
-          // previous contents before the P that this warp has already consumed)
-#pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            MmaTileState& t = a == 0 ? t0 : t1;
-            const int first = ok ? min(2, plan.count(a)) : 0;
-            for (int kk = 0; ok && kk < first; ++kk) {
-              const int u = gu + plan.uidx(a, kk);
-              ok = mbar_wait(&sm.kv_full[u % kStages], (u / kStages) & 1, abort_flag, g.status);
+          // this query tile's KV tiles in load order: [0, nh) and [cb, ce)
+          const KvRange64 rg = plan.range(a);
+          const int cnt = plan.count(a);
+          const int nh = cnt > 0 ? rg.nh : 0;
+          const int cb = a == 0 ? plan.base[0] : plan.base[1];
+          const int ce = cnt > 0 ? cb + rg.nd : cb;
+          const int sl = qi & 1;
+          const uint64_t dq = sl ? c.dq[1] : c.dq[0];
+          ok = mbar_wait(&sm.q_full[sl], (qi >> 1) & 1, abort_flag, g.status);
+          // prologue: the first two S (the epilogue read their buffers' previous contents
+          // before the P that this thread has already consumed)
+          const int first = ok ? min(2, cnt) : 0;
+          for (int kk = 0; kk < first; ++kk) {
+            const int u = gu + (kk < nh ? kk : cb + (kk - nh));
+            // cls_ready follows kv_full: the classifier waited for the tile's load
+            ok = mbar_wait(&sm.cls_ready[u % kStages], (u / kStages) & 1, abort_flag, g.status);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(c, dq, gs & 1, u % kStages);
+            ++gs;
+          }
+          int issued = first, done = 0;
+          int st = gu % kStages, ph = (gu / kStages) & 1;  // stage and phase of tile u
+          for (int u = 0; ok && u < plan.nU; ++u) {
+            if (u < nh || (u >= cb && u < ce)) {
+              const int b = gp & 1;
+              ok = mbar_wait(c.p_full0 + b, (gp >> 1) & 1, abort_flag, g.status);
+              ++gp;
+              if (ok && done == 0 && oc > 0) ok = mbar_wait(c.o_empty, (oc - 1) & 1, abort_flag, g.status);
               if (!ok) break;
               tc_fence_after();
-              const int bs = t.gs & 1;
-              issue_s_mma(tmem + col_s(a, bs), smem_u32(sm.q[a]), smem_u32(sm.k[u % kStages]),
-                          &sm.s_full[a][bs]);
-              ++t.gs;
-              ++t.issued;
+              issue_pv(c, b, st, done > 0);
+              ++done;
+              if (issued < cnt) {
+                const int u2 = issued < nh ? issued : cb + (issued - nh);
+                int st2 = st + (u2 - u), ph2 = ph;
+                while (st2 >= kStages) {
+                  st2 -= kStages;
+                  ph2 ^= 1;
+                }
+                ok = mbar_wait(&sm.cls_ready[st2], ph2, abort_flag, g.status);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(c, dq, gs & 1, st2);
+                ++gs;
+                ++issued;
+              }
+              if (done == cnt) mma_commit(c.o_full);
+            } else {
+              ok = mbar_wait(&c.kv_full[st], ph, abort_flag, g.status);
+              if (!ok) break;
+              mbar_arrive(&sm.kv_empty[st]);
+            }
+            if (++st == kStages) {
+              st = 0;
+              ph ^= 1;
             }
           }
-          for (int u = 0; ok && u < plan.nU; ++u) {
-            const int st = (gu + u) % kStages;
-            if (plan.member(0, u)) ok = mma_step(sm, tmem, plan, gu, 0, st, t0, abort_flag, g.status);
-            if (ok && plan.member(1, u))
-              ok = mma_step(sm, tmem, plan, gu, 1, st, t1, abort_flag, g.status);
-            if (!ok) break;
-            mma_commit(&sm.kv_empty[st]);
-          }
-          if (plan.count(0) > 0) ++t0.oc;
-          if (plan.count(1) > 0) ++t1.oc;
+          if (cnt > 0) ++oc;
           gu += plan.nU;
-          mma_commit(&sm.q_empty);
+          mma_commit(&sm.q_empty[sl]);
         }
-        if (!ok) {  // every MMA issued so far completes before TMEM is released
-          mma_commit(&sm.drain);
-          mbar_wait(&sm.drain, 0, nullptr, nullptr);
+        if (!ok) {  // every MMA this thread issued completes before TMEM is released
+          mma_commit(&sm.drain[a]);
+          mbar_wait(&sm.drain[a], 0, nullptr, nullptr);
         }
       }
       __syncwarp();
     } else if (warp == 2) {
-      // ============================================================ timestamp warp
-      // For every KV tile the CTA loads: int32 copies of its 64 timestamps and the min / max
-      // over its columns inside the sequence, published on ts_ready[stage].  A stage is refilled
-      // only after both query tiles' PV for it, which follows their use of these values.
-      if (use_time) {
-        int gu = 0;
-        bool ok = true;
-        for (int w = blockIdx.x; ok && w < total; w += stride) {
-          const WorkItem it = g.items[w / g.H];
-          const PairPlan plan =
-              make_plan(it.qtile, it.len, hist_len(it.len, g.mask, g.num_candidates));
-          for (int u = 0; u < plan.nU; ++u, ++gu) {
-            const int st = gu % kStages;
-            ok = warp_wait(&sm.kv_full[st], (gu / kStages) & 1, abort_flag, g.status);
-            if (!ok) break;
-            const int c0l = plan.tile_of(u) * kKV;
-            const long long* ts_tile = sm.ts[st] + ((it.row0 + c0l) & 1);
-            long long mn = LLONG_MAX, mx = LLONG_MIN;
+      // ============================================================ classifier warp
+      // For every KV tile the CTA loads: int32 copies of its timestamps, each 32-column half's
+      // timestamp range over its in-sequence columns, and the mode and constant bias of the 16
+      // (query tile, row quarter, half) segments, published on cls_ready[stage].  The issuers
+      // wait for it before the tile's S, so an epilogue that has S has these too.  A stage is
+      // refilled only after both query tiles released it, which follows their use of them.
+      int gu = 0;
+      bool ok = true;
+      WorkItem nxt = g.items[blockIdx.x / g.H];  // the next item is loaded one item ahead
+      for (int w = blockIdx.x; ok && w < total; w += stride) {
+        const WorkItem it = nxt;
+        if (w + stride < total) nxt = g.items[(w + stride) / g.H];
+        const int L = it.len;
+        const int n = hist_len(L, g.mask, g.num_candidates);
+        const PairPlan plan = make_plan(it.qtile, L, n);
+        // row ranges of the 8 (query tile, quarter) groups: lane c < 8 keeps group c's
+        QuarterRows qr;
+        {
+          const int c = lane & 7;
+          qr.i0 = (plan.q[0] + (c >> 2)) * kQ + 32 * (c & 3);
+          qr.i1 = min(qr.i0 + 31, L - 1);
+          qr.pmin = min(qr.i0, n);
+          qr.tlo = qr.thi = 0;
+        }
+        if (use_time) {
+          long long tg[8];  // all 8 loads in flight together
 #pragma unroll
-            for (int w2 = 0; w2 < kKV / 32; ++w2) {
-              const int c = lane + 32 * w2;
-              const long long tv = ts_tile[c];
-              sm.ts32[st][c] = static_cast<int>(tv);
-              if (c0l + c < it.len) {  // the sequence's own columns
-                mn = tv < mn ? tv : mn;
-                mx = tv > mx ? tv : mx;
-              }
-            }
+          for (int c = 0; c < 8; ++c) {
+            const int i = (plan.q[0] + (c >> 2)) * kQ + 32 * (c & 3) + lane;
+            tg[c] = i < L ? g.ts[it.row0 + i] : 0;
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int i = (plan.q[0] + (c >> 2)) * kQ + 32 * (c & 3) + lane;
+            const bool v = i < L;
+            long long mn = v ? tg[c] : LLONG_MAX, mx = v ? tg[c] : LLONG_MIN;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
               const long long omn = __shfl_xor_sync(0xffffffffu, mn, off);
@@ -647,31 +699,93 @@ __global__ void __launch_bounds__(kThreads, 1)
               mn = omn < mn ? omn : mn;
               mx = omx > mx ? omx : mx;
             }
-            if (lane == 0) {
-              sm.tmin[st] = mn;
-              sm.tmax[st] = mx;
+            if ((lane & 7) == c) {
+              qr.tlo = mn;
+              qr.thi = mx;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.ts_ready[st]);
           }
+        }
+        for (int u = 0; u < plan.nU; ++u, ++gu) {
+          const int st = gu % kStages;
+          ok = warp_wait(&sm.kv_full[st], (gu / kStages) & 1, abort_flag, g.status);
+          if (!ok) break;
+          const int c0t = plan.tile_of(u) * kKV;
+          long long hmin[2] = {0, 0}, hmax[2] = {0, 0};
+          if (use_time) {
+            const long long* ts_tile = sm.ts[st] + ((it.row0 + c0t) & 1);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int c = lane + 32 * hf;
+              const long long tv = ts_tile[c];
+              sm.ts32[st][c] = static_cast<int>(tv);
+              const bool in_seq = c0t + c < L;  // the sequence's own columns
+              long long mn = in_seq ? tv : LLONG_MAX, mx = in_seq ? tv : LLONG_MIN;
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) {
+                const long long omn = __shfl_xor_sync(0xffffffffu, mn, off);
+                const long long omx = __shfl_xor_sync(0xffffffffu, mx, off);
+                mn = omn < mn ? omn : mn;
+                mx = omx > mx ? omx : mx;
+              }
+              hmin[hf] = mn;
+              hmax[hf] = mx;
+            }
+            if (lane < 2) {
+              sm.tmin[st][lane] = lane == 0 ? hmin[0] : hmin[1];
+              sm.tmax[st][lane] = lane == 0 ? hmax[0] : hmax[1];
+            }
+          }
+          // lane s < 16 classifies segment s = (query tile, quarter, half) = (s >> 3, s >> 1 & 3,
+          // s & 1); group (tile, quarter) = s >> 1 is held by lane s >> 1
+          const int grp = (lane >> 1) & 7;
+          QuarterRows mine;
+          mine.i0 = __shfl_sync(0xffffffffu, qr.i0, grp);
+          mine.i1 = __shfl_sync(0xffffffffu, qr.i1, grp);
+          mine.pmin = __shfl_sync(0xffffffffu, qr.pmin, grp);
+          mine.tlo = __shfl_sync(0xffffffffu, qr.tlo, grp);
+          mine.thi = __shfl_sync(0xffffffffu, qr.thi, grp);
+          if (lane < 16) {
+            const int hf = lane & 1;
+            sm.cls[st][lane] = classify_quarter(mine, c0t + 32 * hf, n, use_pos ? g.P : 0,
+                                                use_pos, use_time, g.NB, hf ? hmin[1] : hmin[0],
+                                                hf ? hmax[1] : hmax[0], pos4, P2, sm.rab_time_h);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.cls_ready[st]);
         }
       }
     }
   } else {
-    setmaxnreg_inc<208>();
+    setmaxnreg_inc<104>();
     // ============================================================ epilogue warpgroups
-    const int a = (warp - 4) >> 2;
+    // Warpgroup 1 + 2 a + h handles query tile a, columns 32 h .. 32 h + 31 of every S tile
+    // (and of O); warp w reads TMEM lanes 32 (w % 4) .. + 31: one query row per thread.
+    const int e = warp - 4;
+    const int a = e >> 3;
+    const int h = (e >> 2) & 1;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
+    const bool lead = h == 0 && quad == 0 && lane == 0;  // releases KV stages for tile a
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     RowCtx rc;
     rc.half_alpha = 0.5f * g.alpha;
-    rc.P2 = 2 * g.P;
+    rc.P2 = P2;
     rc.nbm1 = g.NB - 1;
+    rc.thr = 0;
+    rc.t_lo = rc.t_hi = 0.f;
     int gu = 0, gk = 0, oc = 0;  // gk: this query tile's KV tiles so far (selects S/P buffers)
     bool ok = true;
+    WorkItem nxt = g.items[blockIdx.x / g.H];  // the next item is loaded one item ahead
+    long long ti_next = 0;                     // and this row's timestamp in it
+    {
+      const int n0 = hist_len(nxt.len, g.mask, g.num_candidates);
+      const PairPlan p0 = make_plan(nxt.qtile, nxt.len, n0);
+      const int i0 = (a == 0 ? p0.q[0] : p0.q[1]) * kQ + r;
+      if (use_time && i0 < nxt.len) ti_next = g.ts[nxt.row0 + i0];
+    }
     for (int w = blockIdx.x; ok && w < total; w += stride) {
-      const WorkItem it = g.items[w / g.H];
+      const WorkItem it = nxt;
+      if (w + stride < total) nxt = g.items[(w + stride) / g.H];
       const int head = w % g.H;
       const int L = it.len;
       const int n = hist_len(L, g.mask, g.num_candidates);
@@ -679,8 +793,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = (a == 0 ? plan.q[0] : plan.q[1]) * kQ + r;
       const bool row_valid = i < L;
       const int pi = i < n ? i : n;
-      const long long ti = (use_time && row_valid) ? g.ts[it.row0 + i] : 0;
-      rc.pi_plus_p = pi + g.P;
+      const long long ti = ti_next;
+      rc.pi_plus_p = pi + (use_pos ? g.P : 0);
       rc.ti = ti;
       rc.ti_lo = static_cast<int>(ti);
       rc.i = i;
@@ -691,61 +805,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int uk = plan.uidx(a, k);
         const int u = gu + uk;
         const int st = u % kStages;
-        if (use_time) ok = warp_wait(&sm.ts_ready[st], (u / kStages) & 1, abort_flag, g.status);
-        if (!ok) break;
-        const int c0l = plan.tile_of(uk) * kKV;
-        rc = classify_segment(rc, c0l, i, n, pi, ti, row_valid, use_pos, use_time, g.P, g.NB,
-                              sm.tmin[st], sm.tmax[st], pos4, sm.rab_time_h);
-        const long long* ts_tile = sm.ts[st] + ((it.row0 + c0l) & 1);
+        const int c0t = plan.tile_of(uk) * kKV;
+        const long long* ts_tile = sm.ts[st] + ((it.row0 + c0t) & 1);
         const int b = gk & 1;
-        ok = warp_wait(&sm.s_full[a][b], (gk >> 1) & 1, abort_flag, g.status);
+        // S(k) follows the tile's classification (its issuer waited for it); the probe of
+        // cls_ready makes that ordering explicit at almost no cost
+        ok = warp_wait2(&sm.s_full[a][b], (gk >> 1) & 1, &sm.cls_ready[st], (u / kStages) & 1,
+                        abort_flag, g.status);
         if (!ok) break;
+        rc = segment_ctx(rc, sm.cls[st][8 * a + 2 * quad + h], c0t, h, ti, row_valid, use_time,
+                         g.NB, &sm.tmin[st][h], &sm.tmax[st][h], sm.rab_time_h);
+        // S(k) was issued after PV(k-2) by the same thread, so PV(k-2) has completed, and all
+        // eight warps of tile a finished tile k-2 (its P preceded S(k)): its stage is free
+        if (k >= 2 && lead) mbar_arrive(&sm.kv_empty[(gu + plan.uidx(a, k - 2)) % kStages]);
         tc_fence_after();
-        const uint32_t s_addr = lane_addr + col_s(a, b);
-        const uint32_t p_addr = lane_addr + col_p(a, b);
-        // warp-uniform choice (tile_epilogue holds .sync.aligned TMEM loads / stores)
-        if (rc.mode == 0)
-          tile_epilogue<0>(s_addr, p_addr, rc, pos4, sm.rab_time_h, sm.ts32[st], ts_tile, use_pos);
-        else if (rc.mode == 1)
-          tile_epilogue<1>(s_addr, p_addr, rc, pos4, sm.rab_time_h, sm.ts32[st], ts_tile, use_pos);
-        else
-          tile_epilogue<2>(s_addr, p_addr, rc, pos4, sm.rab_time_h, sm.ts32[st], ts_tile, use_pos);
+        const uint32_t s_addr = lane_addr + col_s(a, b) + 32 * h;
+        const uint32_t p_addr = lane_addr + col_p(a, b) + 16 * h;
+        const int* ts32 = sm.ts32[st];
+        // warp-uniform choice (the epilogues hold .sync.aligned TMEM loads / stores)
+        if (rc.mode == kModeConst) {
+          seg_epilogue<kModeConst, 0>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        } else if (rc.mode == kModeElem) {
+          if (rc.time_mode == 0)
+            seg_epilogue<kModeElem, 0>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+          else if (rc.time_mode == 1)
+            seg_epilogue<kModeElem, 1>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+          else
+            seg_epilogue<kModeElem, 2>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        } else if (rc.mode == kModeCausal) {
+          if (rc.time_mode == 0)
+            seg_epilogue<kModeCausal, 0>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+          else if (rc.time_mode == 1)
+            seg_epilogue<kModeCausal, 1>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+          else
+            seg_epilogue<kModeCausal, 2>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        } else if (rc.mode == kModeZero) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int z = 0; z < 16; ++z) pk[z] = 0u;
+          tmem_st16(p_addr, pk);
+        } else {  // M-FALCON candidates, or 64-bit time differences
+          seg_epilogue<kModeGeneral, 3>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.p_full[a][b]);
       }
       if (!ok) break;
-      gu += plan.nU;
+      if (use_time && w + stride < total) {  // the next item's row timestamp
+        const int n2 = hist_len(nxt.len, g.mask, g.num_candidates);
+        const PairPlan p2 = make_plan(nxt.qtile, nxt.len, n2);
+        const int i2 = (a == 0 ? p2.q[0] : p2.q[1]) * kQ + r;
+        ti_next = i2 < nxt.len ? g.ts[nxt.row0 + i2] : 0;
+      }
       if (cnt > 0) {
-        // the item's output: wait for its last PV, read O from TMEM, store bf16 rows
+        // the item's output: wait for its last PV, read this warpgroup's 32 columns of O from
+        // TMEM, store them as bf16
         ok = warp_wait(&sm.o_full[a], oc & 1, abort_flag, g.status);
         if (!ok) break;
         ++oc;
+        if (lead)  // every PV of the item has completed: release the last two tiles' stages
+          for (int k = max(0, cnt - 2); k < cnt; ++k)
+            mbar_arrive(&sm.kv_empty[(gu + plan.uidx(a, k)) % kStages]);
         tc_fence_after();
         uint32_t o[32];
-#pragma unroll 1
-        for (int ch = 0; ch < kD / 32; ++ch) {
-          tmem_ld32(lane_addr + col_o(a) + ch * 32, o);
-          tmem_wait_ld_regs(o);
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(it.row0 + i) * ld_o +
-                                                  head * kD + ch * 32);
+        tmem_ld32(lane_addr + col_o(a) + 32 * h, o);
+        tmem_wait_ld_regs(o);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(it.row0 + i) * ld_o +
+                                                head * kD + 32 * h);
 #pragma unroll
-            for (int w4 = 0; w4 < 4; ++w4) {
-              uint4 vv;
-              vv.x = pack_bf16x2(__uint_as_float(o[8 * w4 + 0]), __uint_as_float(o[8 * w4 + 1]));
-              vv.y = pack_bf16x2(__uint_as_float(o[8 * w4 + 2]), __uint_as_float(o[8 * w4 + 3]));
-              vv.z = pack_bf16x2(__uint_as_float(o[8 * w4 + 4]), __uint_as_float(o[8 * w4 + 5]));
-              vv.w = pack_bf16x2(__uint_as_float(o[8 * w4 + 6]), __uint_as_float(o[8 * w4 + 7]));
-              dst[w4] = vv;
-            }
+          for (int w4 = 0; w4 < 4; ++w4) {
+            uint4 vv;
+            vv.x = pack_bf16x2(__uint_as_float(o[8 * w4 + 0]), __uint_as_float(o[8 * w4 + 1]));
+            vv.y = pack_bf16x2(__uint_as_float(o[8 * w4 + 2]), __uint_as_float(o[8 * w4 + 3]));
+            vv.z = pack_bf16x2(__uint_as_float(o[8 * w4 + 4]), __uint_as_float(o[8 * w4 + 5]));
+            vv.w = pack_bf16x2(__uint_as_float(o[8 * w4 + 6]), __uint_as_float(o[8 * w4 + 7]));
+            dst[w4] = vv;
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.o_empty[a]);
       }
+      gu += plan.nU;
     }
   }
   tc_fence_before();
@@ -761,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Shared memory the paired kernel needs for position-table span P.
 size_t attn_fwd_pair_smem(int P, bool has_pos) {
   size_t s = sizeof(PairSmem) + 1024;
-  if (has_pos) s += sizeof(float4) * (2 * P + 4);
+  s += sizeof(float4) * (has_pos ? 2 * P + 4 : 4);
   return s;
 }
 
