@@ -78,8 +78,8 @@ def load_peaks():
 def attn_traffic_bytes():
     """DRAM bytes per attention launch from the committed ncu summary, if the kernel source is
     unchanged since the counters were taken (else None)."""
-    summ = os.path.join(ROOT, "profiles", "attn_fwd_tc_stack4.json")
-    src = os.path.join(ROOT, "hstu_sequential_transducer_jagged_b200", "csrc", "attn_fwd_tc.cu")
+    summ = os.path.join(ROOT, "profiles", "attn_fwd_pair_stack4.json")
+    src = os.path.join(ROOT, "hstu_sequential_transducer_jagged_b200", "csrc", "attn_fwd_pair.cu")
     if not os.path.exists(summ):
         return None
     with open(summ) as f:

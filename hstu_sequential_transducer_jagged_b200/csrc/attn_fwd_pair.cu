@@ -8,27 +8,27 @@
 // or the M-FALCON candidate mask of §7.1.5.)
 //
 // A work item is two 128-row query tiles of one sequence and head (Q double-buffered, so the
-// next item's Q arrives while this one runs); keys and values stream through in 64-row tiles
-// (TMA, 6-stage ring, the tile's timestamps with them) that both query tiles use.  Each query tile owns two S buffers and two P buffers in tensor memory: while its
-// epilogue warpgroup turns S(k) into P(k), the tensor core already holds S(k+1), and S(k+2) is
-// issued into the buffer S(k) leaves as soon as P(k) is written, so an epilogue warpgroup does
-// not wait for the MMA chain and the two warpgroups keep the SFU (the SiLU's tanh) busy.
+// next item's Q arrives while this one runs); keys and values stream through in 96-row tiles
+// (TMA, 5-stage ring, the tile's timestamps with them) that both query tiles use.  Each query
+// tile owns two 96-column score buffers in tensor memory and its epilogue writes P (bf16) over
+// the S it has just read, so 2 x 2 x 96 + 2 x 64 (O) columns fit the 512 of an SM: while the
+// epilogue turns S(k) into P(k), the tensor core already holds S(k+1), and S(k+2) goes into the
+// buffer of S(k) once the PV that read P(k) from it has completed.
 //
 // Warpgroup 0: warp 0 TMA producer; warps 1 and 3 issue the tcgen05.mma of query tile 0 and 1
-// (one thread each: a thread waits about 50 cycles per MMA it issues and over 100 per commit or
-// barrier check, so two issuers overlap those waits, and issue stays off the epilogue warps);
-// warp 1 also owns the TMEM allocation; warp 2 timestamps (per KV tile: min / max, int32 copies).
-// Warpgroups 1 and 2: one epilogue warpgroup per query tile (warp w owns TMEM lanes
-// 32*(w%4) .. +31, one query row per thread).  setmaxnreg moves registers from warpgroup 0
-// (88) to the epilogue warpgroups (208).
-// TMEM (512 columns): S[a][b] at 64*(2a+b), P[a][b] (bf16 pairs) at 256 + 32*(2a+b),
-// O[a] at 384 + 64*a, for query tile a and buffer b.
+// (one thread each; warp 1 also owns the TMEM allocation); warp 2 classifies each KV tile (bias
+// mode per segment, int32 timestamps, timestamp ranges) before its S is issued.  Warpgroups 1-4
+// are the epilogue: warpgroup 1 + 2a + h handles query tile a, columns 48h .. 48h+47 of each
+// score tile; warp w reads TMEM lanes 32 (w % 4) .. + 31, one query row per thread.  setmaxnreg
+// moves registers from warpgroup 0 (64) to the epilogue warpgroups (104).
+// TMEM (512 columns): score buffer b of query tile a at 96 (2a + b) (P of columns 48h.. at
+// +48h, 24 columns of bf16 pairs), O of query tile a at 384 + 64 a.
 //
 // One CTA per SM walks the longest-first work list with a fixed stride; barrier phases run on
 // across items (the S/P buffers alternate by a per-query-tile tile counter that never resets).
 //
 // The relative bias rab_pos[clamp(p_i - p_j)] + rab_time[bucket(t_i - t_j)] is formed per row
-// segment (one row, one KV tile): constant when every key is beyond the position clamp and in
+// segment (one row, one half of a KV tile): constant when every key is beyond the position clamp and in
 // one log2 time bucket (from the tile's min / max timestamp; exact for any timestamp order since
 // the bucket rule is monotone); else the position term comes from a 4-wide shifted table (one
 // 16-byte shared load per 4 scores, exact with clamping at both ends) and the time term from a
@@ -47,17 +47,17 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kQ = kTileRows;           // query tile rows (128)
-constexpr int kKV = 64;                 // key/value tile rows
-constexpr int kStages = 6;
+constexpr int kKV = 96;                 // key/value tile rows
+constexpr int kSeg = 48;                // columns of a score tile per epilogue warp
+constexpr int kStages = 5;
 constexpr int kThreads = 640;          // 5 warpgroups
 constexpr int kQBytes = kQ * kD * 2;    // 16 KB, 128-byte swizzle
-constexpr int kKVBytes = kKV * kD * 2;  // 8 KB
-constexpr int kTsBox = 72;              // timestamps loaded per KV tile (x rounded down to even)
-constexpr int kTsStride = 80;           // 640-byte stages keep every TMA destination 128-aligned
+constexpr int kKVBytes = kKV * kD * 2;  // 12 KB
+constexpr int kTsBox = 98;              // timestamps loaded per KV tile (x rounded down to even)
+constexpr int kTsStride = 112;          // 896-byte stages keep every TMA destination 128-aligned
 constexpr int kTimeSmem = 64;
 
-__device__ __forceinline__ uint32_t col_s(int a, int b) { return 64u * (2 * a + b); }
-__device__ __forceinline__ uint32_t col_p(int a, int b) { return 256u + 32u * (2 * a + b); }
+__device__ __forceinline__ uint32_t col_buf(int a, int b) { return 96u * (2 * a + b); }
 __device__ __forceinline__ uint32_t col_o(int a) { return 384u + 64u * a; }
 
 struct PairSmem {
@@ -67,16 +67,16 @@ struct PairSmem {
   alignas(128) long long ts[kStages][kTsStride];
   alignas(16) int ts32[kStages][kKV];   // low 32 bits of the tile's timestamps
   float rab_time_h[kTimeSmem];           // 0.5 x rab_time, index clamped to NB - 1
-  long long tmin[kStages][2];            // min / max timestamp of each 32-column half's
+  long long tmin[kStages][2];            // min / max timestamp of each 48-column half's
   long long tmax[kStages][2];            // in-sequence columns
   int2 cls[kStages][16];                 // per (query tile, row quarter, half): mode, bias
-  long long rows_t[8][2];                // per (query tile, row quarter): min / max t_i
   uint64_t q_full[2], q_empty[2];        // per item slot
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t cls_ready[kStages];           // the tile's classification and timestamps
   uint64_t s_full[2][2];
   uint64_t p_full[2][2];
+  uint64_t pv_done[2][2];                // the PV that read P from score buffer [a][b]
   uint64_t o_full[2];
   uint64_t o_empty[2];
   uint64_t drain[2];
@@ -89,9 +89,11 @@ static_assert((kTsStride * 8) % 128 == 0, "timestamp stages must keep 128-byte a
 static_assert(kTsStride >= kTsBox, "timestamp stage holds one box");
 static_assert(offsetof(PairSmem, ts) % 128 == 0, "timestamp buffer alignment");
 static_assert(sizeof(PairSmem) % 16 == 0, "the position table follows the struct");
+static_assert(kKVBytes % 1024 == 0, "K / V stages keep the 1024-byte swizzle alignment");
+static_assert(kKV == 2 * kSeg && kSeg == 48, "two 48-column halves: a 32- and a 16-column chunk");
 
-// KV tiles (64 rows) a 128-row query tile visits: history tiles 0..nh-1 (keys j < min(qe, n)),
-// then nd (0..2) tiles from d0 on that hold the candidate rows' own keys beyond the history.
+// KV tiles (96 rows) a 128-row query tile visits: history tiles 0..nh-1 (keys j < min(qe, n)),
+// then nd (0..3) tiles from d0 on that hold the candidate rows' own keys beyond the history.
 struct KvRange64 {
   int nh, d0, nd;
 };
@@ -111,8 +113,8 @@ __device__ __forceinline__ KvRange64 kv_range64(int qt, int L, int n) {
 }
 
 // The KV tiles of a pair of query tiles, in load order U: history tiles 0..nhm-1, then the
-// candidate tiles of query tile 0, then those of query tile 1.  A query tile's next tile is at
-// most 4 positions ahead of its current one in U, inside the 6-stage ring.
+// candidate tiles of query tile 0, then those of query tile 1.  A query tile's tiles are at
+// most 5 positions apart in U.
 struct PairPlan {
   int q[2];
   bool valid[2];
@@ -194,7 +196,7 @@ __device__ __forceinline__ float time_term32(const float* time_h, int d) {
 
 __device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_fast(h), h); }
 
-// Per-row constants of one 32-column segment's epilogue.  The mode and the time-term kind are
+// Per-row constants of one 48-column segment's epilogue.  The mode and the time-term kind are
 // warp-uniform: a warp takes the per-element path for all of its rows when any row needs it
 // (the per-element formulas are exact for every row), so no branch in the epilogue diverges.
 struct RowCtx {
@@ -218,17 +220,17 @@ constexpr int kModeCausal = 2;   // as kModeElem, with the causal diagonal maske
 constexpr int kModeGeneral = 3;  // M-FALCON candidates: everything per element, 64-bit time
 constexpr int kModeZero = 4;     // every entry masked
 
-// P = SiLU(alpha S + bias) for the 32 columns h*32 .. h*32+31 of the tile, as packed bf16.
+// P = SiLU(alpha S + bias) for the W columns cb .. cb+W-1 of the tile, as packed bf16.
 // TM is the time term's kind: 0 constant (in half_bias), 1 threshold, 2 per element from the
 // 32-bit differences, 3 per element from the 64-bit differences.
-template <int MODE, int TM>
-__device__ __forceinline__ void silu_seg(const uint32_t (&s)[32], uint32_t (&pk)[16], int h,
-                                         const RowCtx& rc, const float4* pos4,
-                                         const float* time_h, const int* ts32,
-                                         const long long* ts) {
+template <int MODE, int TM, int W>
+__device__ __forceinline__ void silu_chunk(const uint32_t (&s)[W], uint32_t (&pk)[W / 2], int cb,
+                                           const RowCtx& rc, const float4* pos4,
+                                           const float* time_h, const int* ts32,
+                                           const long long* ts) {
 #pragma unroll
-  for (int q = 0; q < 32; q += 4) {
-    const int c = h * 32 + q;  // column of the first of these 4 within the KV tile
+  for (int q = 0; q < W; q += 4) {
+    const int c = cb + q;  // column of the first of these 4 within the KV tile
     float bb[4];
     if (MODE == kModeConst) {
 #pragma unroll
@@ -273,21 +275,53 @@ __device__ __forceinline__ void silu_seg(const uint32_t (&s)[32], uint32_t (&pk)
   }
 }
 
-// S (TMEM, this warp's 32 columns of its rows) -> P (TMEM, bf16).
-template <int MODE, int TM>
-__device__ __forceinline__ void seg_epilogue(uint32_t s_addr, uint32_t p_addr, int h,
-                                             const RowCtx& rc, const float4* pos4,
-                                             const float* time_h, const int* ts32,
-                                             const long long* ts) {
-  uint32_t s[32];
-  uint32_t pk[16];
-  tmem_ld32(s_addr, s);
-  tmem_wait_ld_regs(s);
-  silu_seg<MODE, TM>(s, pk, h, rc, pos4, time_h, ts32, ts);
-  tmem_st16(p_addr, pk);
+__device__ __forceinline__ void tmem_wait_ld_regs16(uint32_t (&r)[16]) {
+  __syncwarp();
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
 }
 
-// Mode and bias of one (query tile, 32-row quarter, 32-column half) segment of a KV tile,
+// Each thread of a warp writes 8 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// This warp's 48 columns of S (TMEM) -> P (bf16, TMEM), written over the first 24 of those
+// columns: the 32-column chunk is read before its 16 P columns are written, and the 16-column
+// chunk's 8 P columns land in the already-read first chunk too.  (Loading both chunks at once
+// needs 16 more registers than the epilogue warps have.)
+template <int MODE, int TM>
+__device__ __forceinline__ void seg_epilogue(uint32_t seg_addr, int h, const RowCtx& rc,
+                                             const float4* pos4, const float* time_h,
+                                             const int* ts32, const long long* ts) {
+  {
+    uint32_t s[32];
+    uint32_t pk[16];
+    tmem_ld32(seg_addr, s);
+    tmem_wait_ld_regs(s);
+    silu_chunk<MODE, TM, 32>(s, pk, kSeg * h, rc, pos4, time_h, ts32, ts);
+    tmem_st16(seg_addr, pk);
+  }
+  {
+    uint32_t s[16];
+    uint32_t pk[8];
+    tmem_ld16(seg_addr + 32, s);
+    tmem_wait_ld_regs16(s);
+    silu_chunk<MODE, TM, 16>(s, pk, kSeg * h + 32, rc, pos4, time_h, ts32, ts);
+    tmem_st8(seg_addr + 16, pk);
+  }
+}
+
+// Mode and bias of one (query tile, 32-row quarter, 48-column half) segment of a KV tile,
 // decided by the classifier warp from the quarter's row ranges, so exact for every row:
 // all entries masked; some entry masked or a candidate row meeting candidate keys (general);
 // every key beyond the position clamp and every (row, key) pair in one time bucket (constant);
@@ -303,7 +337,7 @@ __device__ __forceinline__ int2 classify_quarter(const QuarterRows& q, int c0, i
                                                  long long tmin, long long tmax,
                                                  const float4* pos4, int P2,
                                                  const float* time_h) {
-  const int last = c0 + 31;
+  const int last = c0 + kSeg - 1;
   int mode;
   if (q.i1 < q.i0 || c0 > q.i1) {
     mode = kModeZero;
@@ -325,6 +359,43 @@ __device__ __forceinline__ int2 classify_quarter(const QuarterRows& q, int c0, i
     else if (mode == kModeConst) mode = kModeElem;
   }
   if (mode == kModeConst) hb += pos4[P2 + 3].x;  // beyond the clamp: the table's last entry
+  return make_int2(mode | (tconst ? 8 : 0), __float_as_int(hb));
+}
+
+// classify_quarter with the timestamps given relative to a common reference, all within
+// +-2^30 of it, so the time buckets come from 32-bit differences: floor(log2(max(1, d))) is
+// 31 minus the leading zero count of d, clamped to nb-1.
+__device__ __forceinline__ int bucket32(int d, int nbm1) {
+  const int b = d < 1 ? 0 : 31 - __clz(d);
+  return b < nbm1 ? b : nbm1;
+}
+
+__device__ __forceinline__ int2 classify_quarter32(int i0, int i1, int pmin, int tlo, int thi,
+                                                   int c0, int n, int P, bool use_pos,
+                                                   bool use_time, int NB, int tmin, int tmax,
+                                                   const float4* pos4, int P2,
+                                                   const float* time_h) {
+  const int last = c0 + kSeg - 1;
+  int mode;
+  if (i1 < i0 || c0 > i1) {
+    mode = kModeZero;
+  } else if (i1 >= n && last >= n) {
+    mode = kModeGeneral;
+  } else if (last > i0) {
+    mode = kModeCausal;
+  } else {
+    mode = (use_pos && pmin - last < P) ? kModeElem : kModeConst;
+  }
+  bool tconst = true;
+  float hb = 0.f;
+  if (use_time && mode != kModeZero && mode != kModeGeneral) {
+    const int b_lo = bucket32(tlo - tmax, NB - 1);
+    const int b_hi = bucket32(thi - tmin, NB - 1);
+    tconst = b_lo == b_hi;
+    if (tconst) hb = time_h[b_lo];
+    else if (mode == kModeConst) mode = kModeElem;
+  }
+  if (mode == kModeConst) hb += pos4[P2 + 3].x;
   return make_int2(mode | (tconst ? 8 : 0), __float_as_int(hb));
 }
 
@@ -407,9 +478,10 @@ __device__ __forceinline__ void tma_load_1d(void* smem_dst, const CUtensorMap* m
 // does no address arithmetic between MMAs.
 struct IssuerCtx {
   uint64_t dq[2], dk0, dv0;        // dq per item slot
-  uint32_t s_col0, p_col0, o_col;  // buffer 1 lies 64 (S) or 32 (P) columns further
+  uint32_t buf0, o_col;            // score buffer 1 lies 96 columns after buffer 0
   uint64_t* s_full0;               // buffer 1's barriers follow buffer 0's
   uint64_t* p_full0;
+  uint64_t* pv_done0;
   uint64_t* o_full;
   uint64_t* o_empty;
   uint64_t* kv_full;
@@ -424,17 +496,21 @@ __device__ __forceinline__ void issue_s(const IssuerCtx& c, uint64_t dq, int bs,
   const uint64_t dk = c.dk0 + static_cast<uint64_t>(st) * kStageDesc;
 #pragma unroll
   for (int kk = 0; kk < kD / 16; ++kk)
-    mma_bf16_ss(c.s_col0 + 64u * bs, dq + 2 * kk, dk + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+    mma_bf16_ss(c.buf0 + 96u * bs, dq + 2 * kk, dk + 2 * kk, idesc, kk > 0 ? 1u : 0u);
   mma_commit(c.s_full0 + bs);
 }
 
+// O (+)= P V over the tile's 96 keys: P of keys 16kk.. is at column 8kk of the buffer for the
+// first half and at 48 + 8 (kk - 3) for the second.
 __device__ __forceinline__ void issue_pv(const IssuerCtx& c, int b, int st, bool acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, kD, 0, 1);
   const uint64_t dv = c.dv0 + static_cast<uint64_t>(st) * kStageDesc;
+  const uint32_t pb = c.buf0 + 96u * b;
 #pragma unroll
   for (int kk = 0; kk < kKV / 16; ++kk)
-    mma_bf16_ts(c.o_col, c.p_col0 + 32u * b + kk * 8, dv + 128 * kk, idesc,
+    mma_bf16_ts(c.o_col, pb + (kk < 3 ? 8 * kk : 48 + 8 * (kk - 3)), dv + 128 * kk, idesc,
                 (acc || kk > 0) ? 1u : 0u);
+  mma_commit(c.pv_done0 + b);
 }
 
 // 20 warps launch with 96 registers each (5 warps per SM sub-partition); after set-up
@@ -485,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sm.s_full[a][b], 1);
         mbar_init(&sm.p_full[a][b], 8);  // one elected lane per epilogue warp of tile a
+        mbar_init(&sm.pv_done[a][b], 1);
       }
       mbar_init(&sm.o_full[a], 1);
       mbar_init(&sm.o_empty[a], 8);
@@ -571,10 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         c.dq[1] = smem_desc_sw128(smem_u32(sm.q[1][a]), 16, 1024);
         c.dk0 = smem_desc_sw128(smem_u32(sm.k[0]), 16, 1024);
         c.dv0 = smem_desc_sw128(smem_u32(sm.v[0]), kKVBytes, 1024);
-        c.s_col0 = tmem + col_s(a, 0);
-        c.p_col0 = tmem + col_p(a, 0);
+        c.buf0 = tmem + col_buf(a, 0);
         c.s_full0 = &sm.s_full[a][0];
         c.p_full0 = &sm.p_full[a][0];
+        c.pv_done0 = &sm.pv_done[a][0];
         c.o_col = tmem + col_o(a);
         c.o_full = &sm.o_full[a];
         c.o_empty = &sm.o_empty[a];
@@ -603,6 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int u = gu + (kk < nh ? kk : cb + (kk - nh));
             // cls_ready follows kv_full: the classifier waited for the tile's load
             ok = mbar_wait(&sm.cls_ready[u % kStages], (u / kStages) & 1, abort_flag, g.status);
+            // the buffer's previous P has been read by its PV
+            if (ok && gs >= 2) ok = mbar_wait(c.pv_done0 + (gs & 1), ((gs - 2) >> 1) & 1, abort_flag, g.status);
             if (!ok) break;
             tc_fence_after();
             issue_s(c, dq, gs & 1, u % kStages);
@@ -627,7 +706,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   st2 -= kStages;
                   ph2 ^= 1;
                 }
-                ok = mbar_wait(&sm.cls_ready[st2], ph2, abort_flag, g.status);
+                ok = mbar_wait(&sm.cls_ready[st2], ph2, abort_flag, g.status) &&
+                     mbar_wait(c.pv_done0 + (gs & 1), ((gs - 2) >> 1) & 1, abort_flag, g.status);
                 if (!ok) break;
                 tc_fence_after();
                 issue_s(c, dq, gs & 1, st2);
@@ -657,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ============================================================ classifier warp
-      // For every KV tile the CTA loads: int32 copies of its timestamps, each 32-column half's
+      // For every KV tile the CTA loads: int32 copies of its timestamps, each 48-column half's
       // timestamp range over its in-sequence columns, and the mode and constant bias of the 16
       // (query tile, row quarter, half) segments, published on cls_ready[stage].  The issuers
       // wait for it before the tile's S, so an epilogue that has S has these too.  A stage is
@@ -671,8 +751,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int L = it.len;
         const int n = hist_len(L, g.mask, g.num_candidates);
         const PairPlan plan = make_plan(it.qtile, L, n);
-        // row ranges of the 8 (query tile, quarter) groups: lane c < 8 keeps group c's
-        QuarterRows qr;
+        // Row ranges of the 8 (query tile, quarter) groups.  Timestamps are taken relative to
+        // t_ref (the item's first row) when every one the item touches lies within +-2^30 of it
+        // (32-bit reductions), else the 64-bit path below runs.
+        // lane s < 16 owns segment s = (query tile s >> 3, quarter s >> 1 & 3, half s & 1)
+        const int grp = (lane >> 1) & 7;
+        const int g_i0 = (plan.q[0] + (grp >> 2)) * kQ + 32 * (grp & 3);
+        const int g_i1 = min(g_i0 + 31, L - 1);
+        const int g_pmin = min(g_i0, n);
+        long long t_ref = 0;
+        bool rel32 = false;
+        int g_tlo = 0, g_thi = 0;   // relative 32-bit row range of this lane's group
+        QuarterRows qr;             // 64-bit row ranges (used when !rel32): lane c < 8: group c
         {
           const int c = lane & 7;
           qr.i0 = (plan.q[0] + (c >> 2)) * kQ + 32 * (c & 3);
@@ -681,45 +771,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           qr.tlo = qr.thi = 0;
         }
         if (use_time) {
-          long long tg[8];  // all 8 loads in flight together
+          // (t_ref is the first row of query tile 0; pass 1 checks the 32-bit range, pass 2
+          // reduces; the row timestamps are read twice, the second time from cache)
+          t_ref = g.ts[it.row0 + plan.q[0] * kQ];
+          bool fits = true;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const int i = (plan.q[0] + (c >> 2)) * kQ + 32 * (c & 3) + lane;
-            tg[c] = i < L ? g.ts[it.row0 + i] : 0;
+            const long long r64 = (i < L ? __ldg(&g.ts[it.row0 + i]) : t_ref) - t_ref;
+            fits = fits && r64 < (1ll << 30) && r64 > -(1ll << 30);
           }
-#pragma unroll
+          rel32 = __all_sync(0xffffffffu, fits);
+#pragma unroll 2
           for (int c = 0; c < 8; ++c) {
             const int i = (plan.q[0] + (c >> 2)) * kQ + 32 * (c & 3) + lane;
             const bool v = i < L;
-            long long mn = v ? tg[c] : LLONG_MAX, mx = v ? tg[c] : LLONG_MIN;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-              const long long omn = __shfl_xor_sync(0xffffffffu, mn, off);
-              const long long omx = __shfl_xor_sync(0xffffffffu, mx, off);
-              mn = omn < mn ? omn : mn;
-              mx = omx > mx ? omx : mx;
-            }
-            if ((lane & 7) == c) {
-              qr.tlo = mn;
-              qr.thi = mx;
-            }
-          }
-        }
-        for (int u = 0; u < plan.nU; ++u, ++gu) {
-          const int st = gu % kStages;
-          ok = warp_wait(&sm.kv_full[st], (gu / kStages) & 1, abort_flag, g.status);
-          if (!ok) break;
-          const int c0t = plan.tile_of(u) * kKV;
-          long long hmin[2] = {0, 0}, hmax[2] = {0, 0};
-          if (use_time) {
-            const long long* ts_tile = sm.ts[st] + ((it.row0 + c0t) & 1);
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-              const int c = lane + 32 * hf;
-              const long long tv = ts_tile[c];
-              sm.ts32[st][c] = static_cast<int>(tv);
-              const bool in_seq = c0t + c < L;  // the sequence's own columns
-              long long mn = in_seq ? tv : LLONG_MAX, mx = in_seq ? tv : LLONG_MIN;
+            const long long tv = v ? __ldg(&g.ts[it.row0 + i]) : t_ref;
+            if (rel32) {
+              const int r = static_cast<int>(tv - t_ref);
+              const int mn = __reduce_min_sync(0xffffffffu, v ? r : INT_MAX);
+              const int mx = __reduce_max_sync(0xffffffffu, v ? r : INT_MIN);
+              if (grp == c) {
+                g_tlo = mn;
+                g_thi = mx;
+              }
+            } else {
+              long long mn = v ? tv : LLONG_MAX, mx = v ? tv : LLONG_MIN;
 #pragma unroll
               for (int off = 16; off > 0; off >>= 1) {
                 const long long omn = __shfl_xor_sync(0xffffffffu, mn, off);
@@ -727,28 +804,113 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mn = omn < mn ? omn : mn;
                 mx = omx > mx ? omx : mx;
               }
-              hmin[hf] = mn;
-              hmax[hf] = mx;
-            }
-            if (lane < 2) {
-              sm.tmin[st][lane] = lane == 0 ? hmin[0] : hmin[1];
-              sm.tmax[st][lane] = lane == 0 ? hmax[0] : hmax[1];
+              if ((lane & 7) == c) {
+                qr.tlo = mn;
+                qr.thi = mx;
+              }
             }
           }
-          // lane s < 16 classifies segment s = (query tile, quarter, half) = (s >> 3, s >> 1 & 3,
-          // s & 1); group (tile, quarter) = s >> 1 is held by lane s >> 1
-          const int grp = (lane >> 1) & 7;
-          QuarterRows mine;
-          mine.i0 = __shfl_sync(0xffffffffu, qr.i0, grp);
-          mine.i1 = __shfl_sync(0xffffffffu, qr.i1, grp);
-          mine.pmin = __shfl_sync(0xffffffffu, qr.pmin, grp);
-          mine.tlo = __shfl_sync(0xffffffffu, qr.tlo, grp);
-          mine.thi = __shfl_sync(0xffffffffu, qr.thi, grp);
-          if (lane < 16) {
-            const int hf = lane & 1;
-            sm.cls[st][lane] = classify_quarter(mine, c0t + 32 * hf, n, use_pos ? g.P : 0,
-                                                use_pos, use_time, g.NB, hf ? hmin[1] : hmin[0],
-                                                hf ? hmax[1] : hmax[0], pos4, P2, sm.rab_time_h);
+        }
+        QuarterRows mine;  // 64-bit path: this lane's group
+        mine.i0 = g_i0;
+        mine.i1 = g_i1;
+        mine.pmin = g_pmin;
+        mine.tlo = __shfl_sync(0xffffffffu, qr.tlo, grp);
+        mine.thi = __shfl_sync(0xffffffffu, qr.thi, grp);
+        for (int u = 0; u < plan.nU; ++u, ++gu) {
+          const int st = gu % kStages;
+          ok = warp_wait(&sm.kv_full[st], (gu / kStages) & 1, abort_flag, g.status);
+          if (!ok) break;
+          const int c0t = plan.tile_of(u) * kKV;
+          const int hf = lane & 1;
+          if (!use_time) {
+            if (lane < 16)
+              sm.cls[st][lane] = classify_quarter32(g_i0, g_i1, g_pmin, 0, 0, c0t + kSeg * hf, n,
+                                                    use_pos ? g.P : 0, use_pos, false, g.NB, 0, 0,
+                                                    pos4, P2, sm.rab_time_h);
+          } else {
+            const long long* ts_tile = sm.ts[st] + ((it.row0 + c0t) & 1);
+            // lane l holds columns l, l + 32, l + 64; half 0 is columns 0..47, half 1 48..95
+            long long tv[3];
+            bool in_seq[3], fits = rel32;
+#pragma unroll
+            for (int r3 = 0; r3 < 3; ++r3) {
+              const int c = lane + 32 * r3;
+              tv[r3] = ts_tile[c];
+              sm.ts32[st][c] = static_cast<int>(tv[r3]);
+              in_seq[r3] = c0t + c < L;  // the sequence's own columns
+              const long long r64 = tv[r3] - t_ref;
+              fits = fits && (!in_seq[r3] || (r64 < (1ll << 30) && r64 > -(1ll << 30)));
+            }
+            if (__all_sync(0xffffffffu, fits)) {
+              int mn0 = INT_MAX, mx0 = INT_MIN, mn1 = INT_MAX, mx1 = INT_MIN;
+#pragma unroll
+              for (int r3 = 0; r3 < 3; ++r3) {
+                const int c = lane + 32 * r3;
+                const int r = static_cast<int>(tv[r3] - t_ref);
+                if (in_seq[r3]) {
+                  if (c < kSeg) {
+                    mn0 = min(mn0, r);
+                    mx0 = max(mx0, r);
+                  } else {
+                    mn1 = min(mn1, r);
+                    mx1 = max(mx1, r);
+                  }
+                }
+              }
+              mn0 = __reduce_min_sync(0xffffffffu, mn0);
+              mx0 = __reduce_max_sync(0xffffffffu, mx0);
+              mn1 = __reduce_min_sync(0xffffffffu, mn1);
+              mx1 = __reduce_max_sync(0xffffffffu, mx1);
+              if (lane < 2) {  // the epilogue's per-row refinement reads absolute values
+                sm.tmin[st][lane] = t_ref + (lane == 0 ? mn0 : mn1);
+                sm.tmax[st][lane] = t_ref + (lane == 0 ? mx0 : mx1);
+              }
+              if (lane < 16)
+                sm.cls[st][lane] = classify_quarter32(g_i0, g_i1, g_pmin, g_tlo, g_thi,
+                                                      c0t + kSeg * hf, n, use_pos ? g.P : 0,
+                                                      use_pos, true, g.NB, hf ? mn1 : mn0,
+                                                      hf ? mx1 : mx0, pos4, P2, sm.rab_time_h);
+            } else {
+              long long mn0 = LLONG_MAX, mx0 = LLONG_MIN, mn1 = LLONG_MAX, mx1 = LLONG_MIN;
+#pragma unroll
+              for (int r3 = 0; r3 < 3; ++r3) {
+                const int c = lane + 32 * r3;
+                if (in_seq[r3]) {
+                  if (c < kSeg) {
+                    mn0 = tv[r3] < mn0 ? tv[r3] : mn0;
+                    mx0 = tv[r3] > mx0 ? tv[r3] : mx0;
+                  } else {
+                    mn1 = tv[r3] < mn1 ? tv[r3] : mn1;
+                    mx1 = tv[r3] > mx1 ? tv[r3] : mx1;
+                  }
+                }
+              }
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) {
+                const long long a0 = __shfl_xor_sync(0xffffffffu, mn0, off);
+                const long long b0 = __shfl_xor_sync(0xffffffffu, mx0, off);
+                const long long a1 = __shfl_xor_sync(0xffffffffu, mn1, off);
+                const long long b1 = __shfl_xor_sync(0xffffffffu, mx1, off);
+                mn0 = a0 < mn0 ? a0 : mn0;
+                mx0 = b0 > mx0 ? b0 : mx0;
+                mn1 = a1 < mn1 ? a1 : mn1;
+                mx1 = b1 > mx1 ? b1 : mx1;
+              }
+              if (lane < 2) {
+                sm.tmin[st][lane] = lane == 0 ? mn0 : mn1;
+                sm.tmax[st][lane] = lane == 0 ? mx0 : mx1;
+              }
+              if (!rel32) {  // the row ranges are 64-bit too
+              } else {
+                mine.tlo = t_ref + g_tlo;
+                mine.thi = t_ref + g_thi;
+              }
+              if (lane < 16)
+                sm.cls[st][lane] = classify_quarter(mine, c0t + kSeg * hf, n, use_pos ? g.P : 0,
+                                                    use_pos, true, g.NB, hf ? mn1 : mn0,
+                                                    hf ? mx1 : mx0, pos4, P2, sm.rab_time_h);
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.cls_ready[st]);
@@ -758,8 +920,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     setmaxnreg_inc<104>();
     // ============================================================ epilogue warpgroups
-    // Warpgroup 1 + 2 a + h handles query tile a, columns 32 h .. 32 h + 31 of every S tile
-    // (and of O); warp w reads TMEM lanes 32 (w % 4) .. + 31: one query row per thread.
+    // Warpgroup 1 + 2 a + h handles query tile a, columns 48 h .. 48 h + 47 of every score tile
+    // and columns 32 h .. 32 h + 31 of O; warp w reads TMEM lanes 32 (w % 4) .. + 31: one query
+    // row per thread.
     const int e = warp - 4;
     const int a = e >> 3;
     const int h = (e >> 2) & 1;
@@ -815,37 +978,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         rc = segment_ctx(rc, sm.cls[st][8 * a + 2 * quad + h], c0t, h, ti, row_valid, use_time,
                          g.NB, &sm.tmin[st][h], &sm.tmax[st][h], sm.rab_time_h);
-        // S(k) was issued after PV(k-2) by the same thread, so PV(k-2) has completed, and all
-        // eight warps of tile a finished tile k-2 (its P preceded S(k)): its stage is free
+        // S(k) was issued after PV(k-2) had completed (same buffer), and all eight warps of
+        // tile a finished tile k-2 (its P preceded that PV): tile k-2's stage is free
         if (k >= 2 && lead) mbar_arrive(&sm.kv_empty[(gu + plan.uidx(a, k - 2)) % kStages]);
         tc_fence_after();
-        const uint32_t s_addr = lane_addr + col_s(a, b) + 32 * h;
-        const uint32_t p_addr = lane_addr + col_p(a, b) + 16 * h;
+        const uint32_t seg_addr = lane_addr + col_buf(a, b) + kSeg * h;
         const int* ts32 = sm.ts32[st];
         // warp-uniform choice (the epilogues hold .sync.aligned TMEM loads / stores)
         if (rc.mode == kModeConst) {
-          seg_epilogue<kModeConst, 0>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+          seg_epilogue<kModeConst, 0>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         } else if (rc.mode == kModeElem) {
           if (rc.time_mode == 0)
-            seg_epilogue<kModeElem, 0>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+            seg_epilogue<kModeElem, 0>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
           else if (rc.time_mode == 1)
-            seg_epilogue<kModeElem, 1>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+            seg_epilogue<kModeElem, 1>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
           else
-            seg_epilogue<kModeElem, 2>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+            seg_epilogue<kModeElem, 2>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         } else if (rc.mode == kModeCausal) {
           if (rc.time_mode == 0)
-            seg_epilogue<kModeCausal, 0>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+            seg_epilogue<kModeCausal, 0>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
           else if (rc.time_mode == 1)
-            seg_epilogue<kModeCausal, 1>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+            seg_epilogue<kModeCausal, 1>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
           else
-            seg_epilogue<kModeCausal, 2>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+            seg_epilogue<kModeCausal, 2>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         } else if (rc.mode == kModeZero) {
           uint32_t pk[16];
 #pragma unroll
           for (int z = 0; z < 16; ++z) pk[z] = 0u;
-          tmem_st16(p_addr, pk);
+          tmem_st16(seg_addr, pk);
+          uint32_t pk8[8];
+#pragma unroll
+          for (int z = 0; z < 8; ++z) pk8[z] = 0u;
+          tmem_st8(seg_addr + 16, pk8);
         } else {  // M-FALCON candidates, or 64-bit time differences
-          seg_epilogue<kModeGeneral, 3>(s_addr, p_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+          seg_epilogue<kModeGeneral, 3>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         }
         tmem_wait_st();
         tc_fence_before();
