@@ -295,29 +295,21 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
       : "memory");
 }
 
-// This warp's 48 columns of S (TMEM) -> P (bf16, TMEM), written over the first 24 of those
-// columns: the 32-column chunk is read before its 16 P columns are written, and the 16-column
-// chunk's 8 P columns land in the already-read first chunk too.  (Loading both chunks at once
-// needs 16 more registers than the epilogue warps have.)
+// This warp's 48 columns of S (TMEM) -> P (bf16, TMEM) in three 16-column chunks; the P of
+// chunk c (8 columns of bf16 pairs) is written over columns 8c .. 8c+7, which belong to chunk
+// 0 or 1 and have been read already.  One 16-column body per mode keeps the code small.
 template <int MODE, int TM>
 __device__ __forceinline__ void seg_epilogue(uint32_t seg_addr, int h, const RowCtx& rc,
                                              const float4* pos4, const float* time_h,
                                              const int* ts32, const long long* ts) {
-  {
-    uint32_t s[32];
-    uint32_t pk[16];
-    tmem_ld32(seg_addr, s);
-    tmem_wait_ld_regs(s);
-    silu_chunk<MODE, TM, 32>(s, pk, kSeg * h, rc, pos4, time_h, ts32, ts);
-    tmem_st16(seg_addr, pk);
-  }
-  {
+#pragma unroll 1
+  for (int c = 0; c < kSeg / 16; ++c) {
     uint32_t s[16];
     uint32_t pk[8];
-    tmem_ld16(seg_addr + 32, s);
+    tmem_ld16(seg_addr + 16 * c, s);
     tmem_wait_ld_regs16(s);
-    silu_chunk<MODE, TM, 16>(s, pk, kSeg * h + 32, rc, pos4, time_h, ts32, ts);
-    tmem_st8(seg_addr + 16, pk);
+    silu_chunk<MODE, TM, 16>(s, pk, kSeg * h + 16 * c, rc, pos4, time_h, ts32, ts);
+    tmem_st8(seg_addr + 8 * c, pk);
   }
 }
 
@@ -994,13 +986,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             seg_epilogue<kModeElem, 1>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
           else
             seg_epilogue<kModeElem, 2>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
-        } else if (rc.mode == kModeCausal) {
-          if (rc.time_mode == 0)
-            seg_epilogue<kModeCausal, 0>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
-          else if (rc.time_mode == 1)
-            seg_epilogue<kModeCausal, 1>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
-          else
-            seg_epilogue<kModeCausal, 2>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        } else if (rc.mode == kModeCausal && rc.time_mode == 0) {
+          seg_epilogue<kModeCausal, 0>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         } else if (rc.mode == kModeZero) {
           uint32_t pk[16];
 #pragma unroll
@@ -1010,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int z = 0; z < 8; ++z) pk8[z] = 0u;
           tmem_st8(seg_addr + 16, pk8);
-        } else {  // M-FALCON candidates, or 64-bit time differences
+        } else {  // M-FALCON candidates, the diagonal with a varying time term, 64-bit times
           seg_epilogue<kModeGeneral, 3>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         }
         tmem_wait_st();
