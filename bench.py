@@ -76,19 +76,22 @@ def load_peaks():
 
 
 def attn_traffic_bytes():
-    """DRAM bytes per attention launch from the committed ncu summary, if the kernel source is
-    unchanged since the counters were taken (else None)."""
-    summ = os.path.join(ROOT, "profiles", "attn_fwd_pair_stack4.json")
+    """DRAM bytes per attention launch from the committed ncu summary (its `traffic_record`
+    line), if the kernel source is unchanged since the counters were taken (else None)."""
+    summ = os.path.join(ROOT, "profiles", "attn_fwd_pair_stack4_b2.md")
     src = os.path.join(ROOT, "hstu_sequential_transducer_jagged_b200", "csrc", "attn_fwd_pair.cu")
     if not os.path.exists(summ):
         return None
+    rec = {}
     with open(summ) as f:
-        rec = json.load(f)
+        for line in f:
+            if line.strip().startswith("traffic_record "):
+                rec = dict(kv.split("=", 1) for kv in line.split()[1:])
     with open(src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()
-    if rec.get("kernel_source_sha256") != digest:
+    if rec.get("kernel_source_sha256") != digest or "dram_bytes_per_launch" not in rec:
         return None
-    return rec.get("dram_bytes_per_launch")
+    return int(rec["dram_bytes_per_launch"])
 
 
 class ClockSampler:
