@@ -164,6 +164,22 @@ def oracle_layer_sample(wl, seconds_min=12.0, max_reps=12):
     return (e - s) * reps / el, sample, len(os.sched_getaffinity(0))
 
 
+def reduce_over_ranks(values_max, values_sum, device):
+    """Across the ranks of the default process group: the maximum of each of values_max (the
+    ranks' device times: the job is as slow as its slowest rank) and the sum of each of
+    values_sum (tokens: weak scaling, every rank its own batch).  Every rank calls it in the
+    same order with lists of the same lengths."""
+    import torch
+    import torch.distributed as dist
+    vmax = torch.tensor(list(values_max), device=device, dtype=torch.float64)
+    vsum = torch.tensor(list(values_sum), device=device, dtype=torch.float64)
+    if vmax.numel():
+        dist.all_reduce(vmax, op=dist.ReduceOp.MAX)
+    if vsum.numel():
+        dist.all_reduce(vsum, op=dist.ReduceOp.SUM)
+    return [float(v) for v in vmax.tolist()], [float(v) for v in vsum.tolist()]
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
@@ -376,12 +392,7 @@ def main():
     attn_ms = [a.elapsed_time(b) for row in attn_ev for a, b in row]
     total_ms = float(sum(step_ms))
     if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        tok = torch.tensor([float(T)], device=dev, dtype=torch.float64)
-        dist.all_reduce(tok, op=dist.ReduceOp.SUM)
-        tokens_all = float(tok.item())
+        (total_ms,), (tokens_all,) = reduce_over_ranks([total_ms], [float(T)], dev)
     else:
         tokens_all = float(T)
     ms_per_step = total_ms / K
@@ -425,9 +436,7 @@ def main():
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
         if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+            (e2e_ms,), _ = reduce_over_ranks([e2e_ms], [], dev)
         h2d = xh.numel() * xh.element_size() + offh.numel() * 4 + tsh.numel() * 8
         d2h = yh.numel() * yh.element_size()
         e2e = {"value": tokens_all * L * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
