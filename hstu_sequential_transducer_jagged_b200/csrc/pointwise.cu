@@ -26,11 +26,20 @@ __device__ __forceinline__ int item_cost(int qt0, int group, int L, int n) {
   return cost;
 }
 
+// Histogram bins live in shared memory when they fit (the usual case), else in the global
+// workspace.  Warps take sequences, lanes take a sequence's items.
+constexpr int kWorklistSmemBins = 4096;
+
 __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B, int T,
                                       int max_len, int mask, int m, int group,
                                       WorkItem* __restrict__ items, int32_t* __restrict__ count,
-                                      int32_t* __restrict__ hist, int max_cost, int32_t* status) {
+                                      int32_t* __restrict__ hist_global, int max_cost,
+                                      int32_t* status) {
   __shared__ int bad;
+  __shared__ int hist_smem[kWorklistSmemBins];
+  int32_t* hist = max_cost < kWorklistSmemBins ? hist_smem : hist_global;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
   if (threadIdx.x == 0) bad = 0;
   for (int c = threadIdx.x; c <= max_cost; c += blockDim.x) hist[c] = 0;
   __syncthreads();
@@ -47,11 +56,12 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
     }
     return;
   }
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+  for (int b = warp; b < B; b += nwarps) {
     const int L = offsets[b + 1] - offsets[b];
     const int n = hist_len(L, mask, m);
     const int nt = (L + kTileRows - 1) / kTileRows;
-    for (int qt = 0; qt < nt; qt += group) atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
+    for (int qt = lane * group; qt < nt; qt += 32 * group)
+      atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {  // exclusive scan in decreasing cost
@@ -64,11 +74,11 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
     *count = run;
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+  for (int b = warp; b < B; b += nwarps) {
     const int L = offsets[b + 1] - offsets[b];
     const int n = hist_len(L, mask, m);
     const int nt = (L + kTileRows - 1) / kTileRows;
-    for (int qt = 0; qt < nt; qt += group) {
+    for (int qt = lane * group; qt < nt; qt += 32 * group) {
       const int pos = atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
       WorkItem it;
       it.seq = b;
