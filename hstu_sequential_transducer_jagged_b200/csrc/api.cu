@@ -223,8 +223,9 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
                                 const void* v, int64_t ld_v, void* o, int64_t ld_o,
                                 cudaStream_t s) {
   const bool tc = attn_uses_tc(D, dtype, q, ld_q, k, ld_k, v, ld_v, o, ld_o);
-  // the paired kernel keeps the position tables in shared memory (P <= 2048) and loads the
-  // timestamps with TMA (16-byte aligned base)
+  // the paired kernel keeps the position table in shared memory (it fits for P up to about
+  // 1100 next to its tiles: the shared-memory check below decides) and loads the timestamps
+  // with TMA (16-byte aligned base)
   const bool use_time = g.ts != nullptr && g.rab_time != nullptr;
   const bool pair = tc && D == 64 && (g.rab_pos == nullptr || g.P <= 2048) &&
                     (!use_time || aligned16(g.ts)) &&

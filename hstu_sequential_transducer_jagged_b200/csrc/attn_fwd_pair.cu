@@ -90,18 +90,18 @@ static_assert(kTsStride >= kTsBox, "timestamp stage holds one box");
 static_assert(offsetof(PairSmem, ts) % 128 == 0, "timestamp buffer alignment");
 static_assert(sizeof(PairSmem) % 16 == 0, "the position table follows the struct");
 static_assert(kKVBytes % 1024 == 0, "K / V stages keep the 1024-byte swizzle alignment");
-static_assert(kKV == 2 * kSeg && kSeg == 48, "two 48-column halves: a 32- and a 16-column chunk");
+static_assert(kKV == 2 * kSeg && kSeg % 16 == 0, "two halves of 16-column chunks");
 
 // KV tiles (96 rows) a 128-row query tile visits: history tiles 0..nh-1 (keys j < min(qe, n)),
 // then nd (0..3) tiles from d0 on that hold the candidate rows' own keys beyond the history.
-struct KvRange64 {
+struct KvRangeP {
   int nh, d0, nd;
 };
 
-__device__ __forceinline__ KvRange64 kv_range64(int qt, int L, int n) {
+__device__ __forceinline__ KvRangeP kv_range_pair(int qt, int L, int n) {
   const int qs = qt * kQ;
   const int qe = min(qs + kQ, L);
-  KvRange64 r;
+  KvRangeP r;
   r.nh = (min(qe, n) + kKV - 1) / kKV;
   r.d0 = 0;
   r.nd = 0;
@@ -118,7 +118,7 @@ __device__ __forceinline__ KvRange64 kv_range64(int qt, int L, int n) {
 struct PairPlan {
   int q[2];
   bool valid[2];
-  KvRange64 r[2];
+  KvRangeP r[2];
   int nhm;
   int base[2];  // U index of each query tile's first candidate tile
   int nU;
@@ -129,13 +129,13 @@ struct PairPlan {
     return r[1].d0 + (u - base[1]);
   }
   // (selects instead of indexing by a runtime a keep the plan in registers)
-  __device__ __forceinline__ KvRange64 range(int a) const { return a == 0 ? r[0] : r[1]; }
+  __device__ __forceinline__ KvRangeP range(int a) const { return a == 0 ? r[0] : r[1]; }
   __device__ __forceinline__ int count(int a) const {
-    const KvRange64 ra = range(a);
+    const KvRangeP ra = range(a);
     return (a == 0 ? valid[0] : valid[1]) ? ra.nh + ra.nd : 0;
   }
   __device__ __forceinline__ int uidx(int a, int k) const {
-    const KvRange64 ra = range(a);
+    const KvRangeP ra = range(a);
     return k < ra.nh ? k : (a == 0 ? base[0] : base[1]) + (k - ra.nh);
   }
 };
@@ -146,9 +146,9 @@ __device__ __forceinline__ PairPlan make_plan(int qt0, int L, int n) {
   p.q[1] = qt0 + 1;
   p.valid[0] = qt0 * kQ < L;
   p.valid[1] = (qt0 + 1) * kQ < L;
-  p.r[0] = kv_range64(p.q[0], L, n);
+  p.r[0] = kv_range_pair(p.q[0], L, n);
   if (p.valid[1]) {
-    p.r[1] = kv_range64(p.q[1], L, n);
+    p.r[1] = kv_range_pair(p.q[1], L, n);
   } else {
     p.r[1].nh = 0;
     p.r[1].d0 = 0;
@@ -211,7 +211,7 @@ struct RowCtx {
   int pi_plus_p, P2, nbm1;
   int i, n, c0t;     // query row, history length, first column of the KV tile
   bool row_valid;
-  int mode;          // kModeConst, kModeElem, kModeGeneral or kModeZero
+  int mode;          // kModeConst, kModeElem, kModeCausal, kModeGeneral or kModeZero
 };
 
 constexpr int kModeConst = 0;    // one bias value per row
@@ -314,10 +314,11 @@ __device__ __forceinline__ void seg_epilogue(uint32_t seg_addr, int h, const Row
 }
 
 // Mode and bias of one (query tile, 32-row quarter, 48-column half) segment of a KV tile,
-// decided by the classifier warp from the quarter's row ranges, so exact for every row:
-// all entries masked; some entry masked or a candidate row meeting candidate keys (general);
-// every key beyond the position clamp and every (row, key) pair in one time bucket (constant);
-// else per element.  cls.x = mode | time-constant flag << 2, cls.y = 0.5 x the constant terms.
+// decided by the classifier warp from the quarter's row ranges, so exact for every row: all
+// entries masked (zero); a candidate row meeting candidate keys (general); keys past some row
+// (causal diagonal); every key beyond the position clamp and every (row, key) pair in one time
+// bucket (constant); else per element.  cls.x = mode | time-constant flag << 3, cls.y = 0.5 x
+// the constant terms.
 struct QuarterRows {
   int i0, i1;            // first and last valid row (i1 < i0: none)
   int pmin;              // smallest position among them
@@ -657,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const PairPlan plan =
               make_plan(it.qtile, it.len, hist_len(it.len, g.mask, g.num_candidates));
           // this query tile's KV tiles in load order: [0, nh) and [cb, ce)
-          const KvRange64 rg = plan.range(a);
+          const KvRangeP rg = plan.range(a);
           const int cnt = plan.count(a);
           const int nh = cnt > 0 ? rg.nh : 0;
           const int cb = a == 0 ? plan.base[0] : plan.base[1];
