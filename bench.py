@@ -263,6 +263,67 @@ def run_attention_only(args, lib, Bd, desc, ly, x, y, ws, stream, wl):
                       "attn_tflops": fl / (ms / 1e3) / 1e12}), flush=True)
 
 
+def run_attention_bwd(args, lib, Bd, dev):
+    """Time the attention forward and backward alone on the attention forward+backward workload
+    (B=64, L~U{512..2048}, H=8, d=64) through the C ABI with preallocated buffers.  FLOPs are
+    the unmasked pairs' algorithmic work: 4 d per pair forward, 8 d per pair backward (the
+    backward's recomputation of S is not counted)."""
+    import torch
+    wl = W.make("attn_fwdbwd_bf16_b64", seed=args.seed)
+    bf = torch.bfloat16
+    q, k, v, d_o = (torch.from_numpy(a).to(bf).to(dev) for a in (wl.q, wl.k, wl.v, wl.d_o))
+    off = torch.from_numpy(wl.seq_offsets).to(dev)
+    ts = torch.from_numpy(wl.timestamps).to(dev)
+    rp = torch.from_numpy(wl.rab_pos).to(dev)
+    rt = torch.from_numpy(wl.rab_time).to(dev)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    d_pos, d_time = torch.empty_like(rp), torch.empty_like(rt)
+    desc = Bd.attn_desc(seq_offsets=off, total_tokens=wl.total_tokens,
+                        max_seq_len=int(wl.lengths.max()), timestamps=ts,
+                        num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, ld_q=q.stride(0),
+                        ld_k=k.stride(0), ld_v=v.stride(0), ld_o=o.stride(0), rab_pos=rp,
+                        max_pos_dist=wl.max_pos_dist, rab_time=rt,
+                        num_time_buckets=wl.num_time_buckets, alpha=wl.alpha)
+    ws = Bd.Workspace(lib.hstu_attention_backward_workspace_size(ctypes.byref(desc)), dev)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def fwd():
+        st = lib.hstu_attention_forward(ctypes.byref(desc), P(q), P(k), P(v), P(o), ws.ptr,
+                                        ws.nbytes, sp)
+        if st != 0:
+            raise Bd.HstuError(st, "hstu_attention_forward")
+
+    def bwd():
+        st = lib.hstu_attention_backward(ctypes.byref(desc), P(q), P(k), P(v), P(d_o), P(dq),
+                                         P(dk), P(dv), P(d_pos), P(d_time), ws.ptr, ws.nbytes, sp)
+        if st != 0:
+            raise Bd.HstuError(st, "hstu_attention_backward")
+
+    res = {}
+    for name, fn in (("fwd", fwd), ("bwd", bwd)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        res[name] = a.elapsed_time(b) / args.steps
+    if ws.sync_status() != 0:
+        raise RuntimeError("device status word set")
+    pairs = attention_pairs(wl) * wl.num_heads
+    print(json.dumps({"mode": "attn_bwd", "workload": wl.name, "tokens": wl.total_tokens,
+                      "fwd_ms": res["fwd"],
+                      "fwd_tflops": 4.0 * wl.d_qk * pairs / (res["fwd"] / 1e3) / 1e12,
+                      "bwd_ms": res["bwd"],
+                      "bwd_tflops": 8.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -272,8 +333,9 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--mode", default="stack", choices=["stack", "attn"],
-                    help="attn: time only the attention stage of layer 0 (profiling aid)")
+    ap.add_argument("--mode", default="stack", choices=["stack", "attn", "attn_bwd"],
+                    help="attn: time only the attention stage of layer 0 (profiling aid); "
+                         "attn_bwd: attention forward and backward on the B=64 workload")
     ap.add_argument("--batch", type=int, default=0,
                     help="use only the first B sequences of the workload (profiling aid)")
     args = ap.parse_args()
@@ -297,6 +359,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     lib = Bd.lib()
+    if args.mode == "attn_bwd":
+        run_attention_bwd(args, lib, Bd, dev)
+        return
 
     # CPU oracle baseline first (rank 0, one GPU), before any other GPU work
     cpu = None
