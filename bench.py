@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 from hstu_sequential_transducer_jagged_b200 import workloads as W  # noqa: E402
 
 WORKLOAD = "stack4_bf16_b8_inter"
+NOMINAL_BF16_TFLOPS = 2250.0  # dense bf16 tensor-core peak of a B200 (vendor figure, context)
 METRIC = "HSTU jagged causal attention TFLOP/s & layer tokens/s on 1 B200 (% of peak)"
 UNIT = "layer-tokens/s"
 L2_FLUSH_BYTES = 256 << 20
@@ -463,6 +464,24 @@ def main():
     ms_per_step = total_ms / K
     value = tokens_all * L * K / (total_ms / 1e3)
 
+    # ---- L2-warm reference (informational): a few steps back to back with no flush between
+    warm_k = min(K, 10)
+    warm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(warm_k)]
+    warm_attn = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(L)] for _ in range(warm_k)]
+    for k in range(warm_k):
+        warm_ev[k][0].record(stream)
+        run_stack(warm_attn[k])
+        warm_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    l2_warm = {
+        "ms_per_step": float(np.mean([a.elapsed_time(b) for a, b in warm_ev])),
+        "attn_ms_per_layer": float(np.mean([a.elapsed_time(b) for row in warm_attn
+                                            for a, b in row])),
+        "steps": warm_k,
+    }
+
     # ---- end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if args.e2e_steps > 0:
@@ -518,6 +537,14 @@ def main():
     attn_avg_ms = float(np.mean(attn_ms))
     attn_tflops = aflops / (attn_avg_ms / 1e3) / 1e12
     traffic = attn_traffic_bytes()
+    # The SiLU's tanh costs one MUFU operation per score and the MUFU pipe takes 16 per clock per
+    # SM, so the attention cannot exceed 16 x 4 d FLOP per clock per SM (at the sampled clock).
+    sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ceil_tflops = 16 * 4 * wl.d_qk * n_sms * sm_mhz * 1e6 / 1e12
+    epi_ceiling = {"value": ceil_tflops, "unit": "TFLOP/s",
+                   "basis": f"one MUFU tanh per score, 16 per clock per SM, {n_sms} SMs at "
+                            f"{sm_mhz:.0f} MHz", "attn_frac": attn_tflops / ceil_tflops}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -536,6 +563,9 @@ def main():
                      "peak_source": f"{peaks['source']} bf16 (burst)",
                      "traffic": traffic,
                      "algorithmic_flops_per_launch": aflops},
+        "attn_frac_of_nominal": attn_tflops / NOMINAL_BF16_TFLOPS,
+        "epilogue_ceiling": epi_ceiling,
+        "l2_warm": l2_warm,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
