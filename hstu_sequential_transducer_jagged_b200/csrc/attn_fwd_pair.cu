@@ -989,6 +989,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             seg_epilogue<kModeElem, 2>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         } else if (rc.mode == kModeCausal && rc.time_mode == 0) {
           seg_epilogue<kModeCausal, 0>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        } else if (rc.mode == kModeCausal && rc.time_mode == 1) {
+          seg_epilogue<kModeCausal, 1>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
+        } else if (rc.mode == kModeCausal && rc.time_mode == 2) {
+          seg_epilogue<kModeCausal, 2>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         } else if (rc.mode == kModeZero) {
           uint32_t pk[16];
 #pragma unroll
@@ -998,7 +1002,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int z = 0; z < 8; ++z) pk8[z] = 0u;
           tmem_st8(seg_addr + 16, pk8);
-        } else {  // M-FALCON candidates, the diagonal with a varying time term, 64-bit times
+        } else {  // M-FALCON candidates, or 64-bit time differences
           seg_epilogue<kModeGeneral, 3>(seg_addr, h, rc, pos4, sm.rab_time_h, ts32, ts_tile);
         }
         tmem_wait_st();
