@@ -68,3 +68,21 @@ def test_reference_arm_is_rank0_only(capsys):
 
     bench.run_reference(Args, rank=1)   # returns at once, prints nothing
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the reference arm (the fp64 oracle on the host cores) on rank 0: one JSON line with the
+    # contract's keys; one short step keeps this test to seconds
+    import json
+    import subprocess
+    proc = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                           "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                          timeout=600, cwd=ROOT)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    line = json.loads(proc.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 1
+    for key in ("metric", "unit", "n_gpus", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
