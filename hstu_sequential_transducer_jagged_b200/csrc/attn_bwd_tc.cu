@@ -1,0 +1,481 @@
+// attn_bwd_tc.cu — jagged HSTU pointwise attention backward for head width 64 on the
+// 5th-generation tensor cores.  Compiled into the library but not yet reachable from the C ABI:
+// hstu_attention_backward keeps the SIMT kernels until this one has passed its parity run on
+// hardware.
+//
+// With S = alpha Q Kᵀ + rab on visible pairs, P = SiLU(S), O = P V and the output gradient dO
+// (chain rule through "万亿参数推荐大模型：HSTU 架构如何超越传统 Self-Attention" §2.1, second formula):
+//   dV = Pᵀ dO,  dP = dO Vᵀ,  dS = dP ⊙ SiLU'(S),  SiLU'(x) = σ(x) (1 + x (1 - σ(x))),
+//   dQ = alpha dS K,  dK = alpha dSᵀ Q,
+//   d rab_pos[k] = Σ dS over pairs with clamped distance index k, d rab_time[b] likewise per time
+//   bucket (the N×N rab backward that "6.2 HSTU的工程突破" §6.2.3 names as the RAB's cost).
+//
+// Key/value-stationary: a CTA takes a (sequence, head, 128-row key tile) item and walks the
+// query tiles from the diagonal to the end of the sequence.  Per query tile:
+//   Sᵀ = K Qᵀ and dPᵀ = V dOᵀ                       (smem x smem MMAs, M = keys, N = queries)
+//   epilogue (one key row per thread): x = alpha s + bias, σ = 1/2 + tanh(x/2)/2, P = x σ,
+//     dS = dP σ (1 + x (1 - σ)), 0 where the mask hides the pair; Pᵀ and (alpha dS)ᵀ as bf16
+//     over the first halves of the Sᵀ / dPᵀ columns, (alpha dS)ᵀ also to shared memory (the
+//     MN-major A operand of dQ); bias-table gradients summed in registers along runs of one
+//     table index and added to shared-memory bins when the index changes
+//   dV += Pᵀ dO,  dK += (alpha dS)ᵀ Q                 (tensor-memory A operand)
+//   dQ  = (alpha dS) K -> tensor memory -> 4 drain warps add it (16-byte vector atomics) to an
+//     fp32 accumulator in global memory, converted to bf16 after the kernel.
+// TMEM columns: Sᵀ 0..127, dPᵀ 128..255, dV 256..319, dK 320..383, dQ 384..447.
+// Warps: 0 TMA producer, 1 MMA issuer (and the TMEM allocation), 2-3 idle, 4-11 epilogue (lane
+// quarter w % 4, query half (w - 4) / 4), 12-15 dQ drain (lane quarter w % 4).
+// Items are visited in the reverse of the forward's longest-first order (which sorts by the
+// number of key tiles a query tile visits), so that key tiles near the start of long sequences,
+// which walk the most query tiles, start first.
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace hstu {
+namespace {
+
+constexpr int kD = 64;
+constexpr int kT = 128;
+constexpr int kQStages = 2;
+constexpr int kThreads = 512;
+constexpr int kTileBytes = kT * kD * 2;   // 16 KB
+constexpr int kTsStride = 144;            // 1152 bytes per stage (TMA destination 128-aligned)
+constexpr int kTsBox = 130;
+constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+
+struct BwdSmem {
+  alignas(1024) uint8_t k[kTileBytes];
+  alignas(1024) uint8_t v[kTileBytes];
+  alignas(1024) uint8_t q[kQStages][kTileBytes];
+  alignas(1024) uint8_t dO[kQStages][kTileBytes];
+  alignas(1024) uint8_t ds[2 * kTileBytes];      // [query half][key row][64 queries] SW128
+  alignas(128) long long tq[kQStages][kTsStride];  // timestamps of the query tile
+  uint64_t kv_full, kv_empty;
+  uint64_t qd_full[kQStages], qd_empty[kQStages];
+  uint64_t s_full, p_full, mm_done, dq_full, dq_empty, acc_full, acc_empty, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  // followed by float bins[2P+1 + NB]
+};
+
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
+  __syncwarp();
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* status) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+__device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Items: (sequence, 128-row key tile) from the work list built with one tile per item, times heads.
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_ts, AttnGeom g,
+                       __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out,
+                       int64_t ld_kv, float* __restrict__ dq_acc, int64_t ld_dq,
+                       float* __restrict__ d_pos, float* __restrict__ d_time) {
+  const int nitems = *g.item_count;
+  const int total = nitems * g.H;
+  if (static_cast<int>(blockIdx.x) >= total) return;
+  extern __shared__ uint8_t smem_raw[];
+  BwdSmem& sm = *reinterpret_cast<BwdSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* bins = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(BwdSmem));
+  const bool use_pos = g.rab_pos != nullptr;
+  const bool use_time = g.ts != nullptr && g.rab_time != nullptr;
+  const int npos = use_pos ? 2 * g.P + 1 : 0;
+  const int nbins = npos + (use_time ? g.NB : 0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int stride = static_cast<int>(gridDim.x);
+
+  // bins[0, nbins): gradient bins; then copies of the two bias tables
+  float* tab_pos = bins + nbins;
+  float* tab_time = tab_pos + npos;
+  for (int e = threadIdx.x; e < nbins; e += kThreads) {
+    bins[e] = 0.f;
+    tab_pos[e] = e < npos ? g.rab_pos[e] : g.rab_time[e - npos];
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.kv_full, 1);
+    mbar_init(&sm.kv_empty, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&sm.qd_full[s], 1);
+      mbar_init(&sm.qd_empty[s], 1);
+    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.mm_done, 1);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dq_empty, 4);
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.acc_empty, 8);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int gs = 0, jj = 0, kv_issued = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < total; w += stride, ++jj) {
+        const WorkItem it = g.items[nitems - 1 - w / g.H];
+        const int head = w % g.H, kt = it.qtile, L = it.len;
+        const int nt = (L + kT - 1) / kT;
+        if (jj > 0 && !mbar_wait(&sm.kv_empty, (jj - 1) & 1, abort_flag, g.status)) {
+          ok = false;
+          break;
+        }
+        ++kv_issued;
+        mbar_arrive_expect_tx(&sm.kv_full, 2 * kTileBytes);
+        tma_load_2d(sm.k, &tm_k, &sm.kv_full, head * kD, it.row0 + kt * kT);
+        tma_load_2d(sm.v, &tm_v, &sm.kv_full, head * kD, it.row0 + kt * kT);
+        for (int qt = kt; qt < nt; ++qt, ++gs) {
+          const int st = gs % kQStages;
+          if (gs >= kQStages &&
+              !mbar_wait(&sm.qd_empty[st], ((gs / kQStages) - 1) & 1, abort_flag, g.status)) {
+            ok = false;
+            break;
+          }
+          const int r0 = it.row0 + qt * kT;
+          mbar_arrive_expect_tx(&sm.qd_full[st], 2 * kTileBytes + (use_time ? kTsBox * 8 : 0));
+          tma_load_2d(sm.q[st], &tm_q, &sm.qd_full[st], head * kD, r0);
+          tma_load_2d(sm.dO[st], &tm_do, &sm.qd_full[st], head * kD, r0);
+          if (use_time) tma_load_1d(sm.tq[st], &tm_ts, &sm.qd_full[st], r0 & ~1);
+        }
+      }
+      if (!ok) {  // leave no TMA write in flight into shared memory about to be released
+        if (kv_issued > 0) mbar_wait(&sm.kv_full, (kv_issued - 1) & 1, nullptr, nullptr);
+        for (int u = gs > kQStages ? gs - kQStages : 0; u < gs; ++u)
+          mbar_wait(&sm.qd_full[u % kQStages], (u / kQStages) & 1, nullptr, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);     // S^T, dP^T
+      constexpr uint32_t id_kv = idesc_bf16_f32(128, kD, 0, 1);     // dV, dK (B MN-major)
+      constexpr uint32_t id_q = idesc_bf16_f32(128, kD, 1, 1);      // dQ (A and B MN-major)
+      const uint32_t kb = smem_u32(sm.k), vb = smem_u32(sm.v), dsb = smem_u32(sm.ds);
+      int gs = 0, jj = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < total; w += stride, ++jj) {
+        const WorkItem it = g.items[nitems - 1 - w / g.H];
+        const int kt = it.qtile, L = it.len;
+        const int nt = (L + kT - 1) / kT;
+        ok = mbar_wait(&sm.kv_full, jj & 1, abort_flag, g.status);
+        for (int qt = kt; ok && qt < nt; ++qt, ++gs) {
+          const int st = gs % kQStages;
+          const bool first = qt == kt;
+          ok = mbar_wait(&sm.qd_full[st], (gs / kQStages) & 1, abort_flag, g.status);
+          // the previous step's MMAs read P^T / dS^T (aliased with S^T / dP^T) and the dS tile
+          if (ok && gs > 0) ok = mbar_wait(&sm.mm_done, (gs - 1) & 1, abort_flag, g.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qb = smem_u32(sm.q[st]), ob = smem_u32(sm.dO[st]);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            mma_bf16_ss(tmem + kColST, smem_desc_sw128(kb + kk * 32, 16, 1024),
+                        smem_desc_sw128(qb + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            mma_bf16_ss(tmem + kColDPT, smem_desc_sw128(vb + kk * 32, 16, 1024),
+                        smem_desc_sw128(ob + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sm.s_full);
+          ok = mbar_wait(&sm.p_full, gs & 1, abort_flag, g.status);
+          if (ok && first && jj > 0) ok = mbar_wait(&sm.acc_empty, (jj - 1) & 1, abort_flag, g.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk) {  // 16 queries per step; P^T / dS^T columns
+            const uint32_t pc = kk < 4 ? 8 * kk : 64 + 8 * (kk - 4);
+            mma_bf16_ts(tmem + kColDV, tmem + kColST + pc, smem_desc_sw128(ob + kk * 2048, kTileBytes, 1024),
+                        id_kv, (!first || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + kColDK, tmem + kColDPT + pc, smem_desc_sw128(qb + kk * 2048, kTileBytes, 1024),
+                        id_kv, (!first || kk > 0) ? 1u : 0u);
+          }
+          if (gs > 0) ok = mbar_wait(&sm.dq_empty, (gs - 1) & 1, abort_flag, g.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk)  // 16 keys per step
+            mma_bf16_ss(tmem + kColDQ, smem_desc_sw128(dsb + kk * 2048, kTileBytes, 1024),
+                        smem_desc_sw128(kb + kk * 2048, kTileBytes, 1024), id_q, kk > 0 ? 1u : 0u);
+          mma_commit(&sm.dq_full);
+          mma_commit(&sm.mm_done);
+          mma_commit(&sm.qd_empty[st]);
+        }
+        if (!ok) break;
+        mma_commit(&sm.acc_full);
+        mma_commit(&sm.kv_empty);
+      }
+      if (!ok) {
+        mma_commit(&sm.drain);
+        mbar_wait(&sm.drain, 0, nullptr, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3, hq = (warp - 4) >> 2;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float alpha = g.alpha;
+    // Bias-gradient runs: along one key row the table index changes only where the clamped
+    // distance or the time bucket changes, so each thread sums a run in registers and adds it
+    // to the shared-memory bin when the index moves on.
+    int run_p = -1, run_t = -1;
+    float acc_p = 0.f, acc_t = 0.f;
+    int gs = 0, jj = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < total; w += stride, ++jj) {
+      const WorkItem it = g.items[nitems - 1 - w / g.H];
+      const int head = w % g.H, kt = it.qtile, L = it.len;
+      const int n = hist_len(L, g.mask, g.num_candidates);
+      const int nt = (L + kT - 1) / kT;
+      const int jrow = kt * kT + quad * 32 + lane;  // this thread's key row
+      const bool jvalid = jrow < L;
+      const int pj = jrow < n ? jrow : n;
+      const long long tj = (use_time && jvalid) ? g.ts[it.row0 + jrow] : 0;
+      for (int qt = kt; ok && qt < nt; ++qt, ++gs) {
+        const int st = gs % kQStages;
+        ok = warp_wait(&sm.s_full, gs & 1, abort_flag, g.status);
+        // the query timestamps came with the Q stage: observe its completion too
+        if (ok && use_time) ok = warp_wait(&sm.qd_full[st], (gs / kQStages) & 1, abort_flag, g.status);
+        if (!ok) break;
+        tc_fence_after();
+        const long long* tq = sm.tq[st] + ((it.row0 + qt * kT) & 1);
+        uint8_t* ds_row = sm.ds + hq * kTileBytes + (quad * 32 + lane) * 128;
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {  // 32 query columns per chunk
+          const uint32_t col = 64 * hq + 32 * ch;
+          uint32_t s[32], dp[32];
+          tmem_ld32(lane_addr + kColST + col, s);
+          tmem_ld32(lane_addr + kColDPT + col, dp);
+          tmem_wait_ld32(s);
+          tmem_wait_ld32(dp);
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int c = 64 * hq + 32 * ch + e + u;
+              const int i = qt * kT + c;
+              float bias = 0.f;
+              int pidx = 0, bidx = 0;
+              if (use_pos) {
+                const int pi = i < n ? i : n;
+                int d = pi - pj;
+                d = d < -g.P ? -g.P : (d > g.P ? g.P : d);
+                pidx = d + g.P;
+                bias += tab_pos[pidx];
+              }
+              if (use_time) {
+                bidx = time_bucket64(tq[c] - tj, g.NB);
+                bias += tab_time[bidx];
+              }
+              const bool vis = jvalid && i < L && jrow <= i && (jrow < n || jrow == i);
+              const float x = fmaf(alpha, __uint_as_float(s[e + u]), bias);
+              const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
+              const float p = x * sg;
+              const float dsv = vis ? __uint_as_float(dp[e + u]) * sg * fmaf(x, 1.f - sg, 1.f) : 0.f;
+              pv[u] = vis ? p : 0.f;
+              dv2[u] = alpha * dsv;
+              if (vis && use_pos) {
+                if (pidx != run_p) {
+                  if (run_p >= 0) atomicAdd(&bins[run_p], acc_p);
+                  run_p = pidx;
+                  acc_p = 0.f;
+                }
+                acc_p += dsv;
+              }
+              if (vis && use_time) {
+                if (bidx != run_t) {
+                  if (run_t >= 0) atomicAdd(&bins[npos + run_t], acc_t);
+                  run_t = bidx;
+                  acc_t = 0.f;
+                }
+                acc_t += dsv;
+              }
+            }
+            pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+            dk[e >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+          }
+          // P^T / (a dS)^T over the already-read first half of this warp's 64 columns
+          tmem_st16(lane_addr + kColST + 64 * hq + 16 * ch, pk);
+          tmem_st16(lane_addr + kColDPT + 64 * hq + 16 * ch, dk);
+          // (a dS)^T row to shared memory: chunk cc (8 queries) of this half at cc ^ (row & 7)
+          const int rr = quad * 32 + lane;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int chunk = 4 * ch + cc;
+            uint4 val = make_uint4(dk[4 * cc], dk[4 * cc + 1], dk[4 * cc + 2], dk[4 * cc + 3]);
+            *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (rr & 7)) * 16)) = val;
+          }
+        }
+        tmem_wait_st();
+        fence_async_smem();  // the dS tile is read by the dQ MMA (async proxy)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full);
+      }
+      if (!ok) break;
+      // the item's dV, dK: this warp's 32 of the 64 columns of each
+      ok = warp_wait(&sm.acc_full, jj & 1, abort_flag, g.status);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t a[32];
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        tmem_ld32(lane_addr + (which ? kColDK : kColDV) + 32 * hq, a);
+        tmem_wait_ld32(a);
+        if (jvalid) {
+          __nv_bfloat16* dst = (which ? dk_out : dv_out) +
+                               static_cast<int64_t>(it.row0 + jrow) * ld_kv + head * kD + 32 * hq;
+#pragma unroll
+          for (int w4 = 0; w4 < 4; ++w4) {
+            uint4 vv;
+            vv.x = pack_bf16x2(__uint_as_float(a[8 * w4 + 0]), __uint_as_float(a[8 * w4 + 1]));
+            vv.y = pack_bf16x2(__uint_as_float(a[8 * w4 + 2]), __uint_as_float(a[8 * w4 + 3]));
+            vv.z = pack_bf16x2(__uint_as_float(a[8 * w4 + 4]), __uint_as_float(a[8 * w4 + 5]));
+            vv.w = pack_bf16x2(__uint_as_float(a[8 * w4 + 6]), __uint_as_float(a[8 * w4 + 7]));
+            reinterpret_cast<uint4*>(dst)[w4] = vv;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty);
+    }
+    if (run_p >= 0) atomicAdd(&bins[run_p], acc_p);
+    if (run_t >= 0) atomicAdd(&bins[npos + run_t], acc_t);
+  } else if (warp >= 12) {
+    // ---------------------------------------------------------------- dQ drain
+    const int quad = warp & 3;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    int gs = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < total; w += stride) {
+      const WorkItem it = g.items[nitems - 1 - w / g.H];
+      const int head = w % g.H, kt = it.qtile, L = it.len;
+      const int nt = (L + kT - 1) / kT;
+      for (int qt = kt; ok && qt < nt; ++qt, ++gs) {
+        ok = warp_wait(&sm.dq_full, gs & 1, abort_flag, g.status);
+        if (!ok) break;
+        tc_fence_after();
+        const int i = qt * kT + quad * 32 + lane;
+        uint32_t a[32];
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          tmem_ld32(lane_addr + kColDQ + 32 * ch, a);
+          tmem_wait_ld32(a);
+          if (i < L) {
+            float* dst = dq_acc + static_cast<int64_t>(it.row0 + i) * ld_dq + head * kD + 32 * ch;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              atomicAdd(reinterpret_cast<float4*>(dst + e),
+                        make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]),
+                                    __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3])));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.dq_empty);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  for (int e = threadIdx.x; e < nbins; e += kThreads) {
+    const float v = bins[e];
+    if (v != 0.f) atomicAdd(e < npos ? &d_pos[e] : &d_time[e - npos], v);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+}  // namespace hstu
+
+// ---------------------------------------------------------------------------- host side
+namespace hstu {
+namespace {
+__global__ void f32_to_bf16_rows(const float* __restrict__ src, int64_t ld_src,
+                                 __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int rows,
+                                 int cols) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(rows) * cols;
+  if (idx >= n) return;
+  const int r = static_cast<int>(idx / cols), c = static_cast<int>(idx % cols);
+  dst[r * ld_dst + c] = __float2bfloat16_rn(src[r * ld_src + c]);
+}
+}  // namespace
+
+size_t attn_bwd_tc_smem(int P, int NB) {
+  return sizeof(BwdSmem) + 1024 + 2 * sizeof(float) * (2 * P + 1 + NB);
+}
+
+cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const CUtensorMap& tdo,
+                               const CUtensorMap& tts, const AttnGeom& g,
+                               __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                               int64_t ld, float* dq_acc, float* d_pos, float* d_time,
+                               int grid, cudaStream_t stream) {
+  const size_t smem = attn_bwd_tc_smem(g.rab_pos ? g.P : 0, g.rab_time ? g.NB : 0);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(dq_acc, 0, sizeof(float) * g.T * g.H * 64, stream);
+  if (e == cudaSuccess && d_pos) e = cudaMemsetAsync(d_pos, 0, sizeof(float) * (2 * g.P + 1), stream);
+  if (e == cudaSuccess && d_time) e = cudaMemsetAsync(d_time, 0, sizeof(float) * g.NB, stream);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  attn_bwd_tc_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, dv, ld,
+                                                       dq_acc, static_cast<int64_t>(g.H) * 64,
+                                                       d_pos, d_time);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t n = static_cast<int64_t>(g.T) * g.H * 64;
+  f32_to_bf16_rows<<<static_cast<int>((n + 255) / 256), 256, 0, stream>>>(
+      dq_acc, static_cast<int64_t>(g.H) * 64, dq, ld, g.T, g.H * 64);
+  return cudaGetLastError();
+}
+}  // namespace hstu
