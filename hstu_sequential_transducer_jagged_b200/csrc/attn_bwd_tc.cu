@@ -97,8 +97,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_do,
                        const __grid_constant__ CUtensorMap tm_ts, AttnGeom g,
-                       __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out,
-                       int64_t ld_kv, float* __restrict__ dq_acc, int64_t ld_dq,
+                       __nv_bfloat16* __restrict__ dk_out, int64_t ld_dk,
+                       __nv_bfloat16* __restrict__ dv_out, int64_t ld_dv,
+                       float* __restrict__ dq_acc, int64_t ld_acc,
                        float* __restrict__ d_pos, float* __restrict__ d_time) {
   const int nitems = *g.item_count;
   const int total = nitems * g.H;
@@ -367,7 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld32(a);
         if (jvalid) {
           __nv_bfloat16* dst = (which ? dk_out : dv_out) +
-                               static_cast<int64_t>(it.row0 + jrow) * ld_kv + head * kD + 32 * hq;
+                               static_cast<int64_t>(it.row0 + jrow) * (which ? ld_dk : ld_dv) +
+                               head * kD + 32 * hq;
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
             uint4 vv;
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(lane_addr + kColDQ + 32 * ch, a);
           tmem_wait_ld32(a);
           if (i < L) {
-            float* dst = dq_acc + static_cast<int64_t>(it.row0 + i) * ld_dq + head * kD + 32 * ch;
+            float* dst = dq_acc + static_cast<int64_t>(it.row0 + i) * ld_acc + head * kD + 32 * ch;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               atomicAdd(reinterpret_cast<float4*>(dst + e),
@@ -438,14 +440,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------- host side
 namespace hstu {
 namespace {
+// dQ accumulator (fp32, row stride ld_src) -> bf16 rows; 8 columns per thread (cols and ld_dst
+// multiples of 8, dst 16-byte aligned: checked by the caller).
 __global__ void f32_to_bf16_rows(const float* __restrict__ src, int64_t ld_src,
                                  __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int rows,
                                  int cols) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(rows) * cols;
-  if (idx >= n) return;
-  const int r = static_cast<int>(idx / cols), c = static_cast<int>(idx % cols);
-  dst[r * ld_dst + c] = __float2bfloat16_rn(src[r * ld_src + c]);
+  const int per_row = cols / 8;
+  if (idx >= static_cast<int64_t>(rows) * per_row) return;
+  const int64_t r = idx / per_row;
+  const int c = static_cast<int>(idx % per_row) * 8;
+  const float4 a = *reinterpret_cast<const float4*>(src + r * ld_src + c);
+  const float4 b = *reinterpret_cast<const float4*>(src + r * ld_src + c + 4);
+  uint4 o;
+  o.x = pack_bf16x2(a.x, a.y);
+  o.y = pack_bf16x2(a.z, a.w);
+  o.z = pack_bf16x2(b.x, b.y);
+  o.w = pack_bf16x2(b.z, b.w);
+  *reinterpret_cast<uint4*>(dst + r * ld_dst + c) = o;
 }
 }  // namespace
 
@@ -453,29 +465,34 @@ size_t attn_bwd_tc_smem(int P, int NB) {
   return sizeof(BwdSmem) + 1024 + 2 * sizeof(float) * (2 * P + 1 + NB);
 }
 
+// Launches the backward over the work list in g (one 128-row tile per item): tq / tk / tv / tdo
+// are 64 x 128 boxes (128-byte swizzle) over Q, K, V, dO; tts a 130-element int64 box over the
+// timestamps (used when g.ts and g.rab_time are set).  dq_acc: fp32 [T, H*64], zeroed here.
+// grid: at most one CTA per SM (persistent).  Returns cudaErrorInvalidValue when the bias
+// tables do not fit in shared memory.
 cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdo,
                                const CUtensorMap& tts, const AttnGeom& g,
-                               __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
-                               int64_t ld, float* dq_acc, float* d_pos, float* d_time,
-                               int grid, cudaStream_t stream) {
+                               __nv_bfloat16* dq, int64_t ld_dq, __nv_bfloat16* dk,
+                               int64_t ld_dk, __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc,
+                               float* d_pos, float* d_time, int grid, cudaStream_t stream) {
   const size_t smem = attn_bwd_tc_smem(g.rab_pos ? g.P : 0, g.rab_time ? g.NB : 0);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  // d_pos / d_time are accumulated into: the caller zeroes them
   cudaError_t e = cudaMemsetAsync(dq_acc, 0, sizeof(float) * g.T * g.H * 64, stream);
-  if (e == cudaSuccess && d_pos) e = cudaMemsetAsync(d_pos, 0, sizeof(float) * (2 * g.P + 1), stream);
-  if (e == cudaSuccess && d_time) e = cudaMemsetAsync(d_time, 0, sizeof(float) * g.NB, stream);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_tc_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, dv, ld,
-                                                       dq_acc, static_cast<int64_t>(g.H) * 64,
-                                                       d_pos, d_time);
+  attn_bwd_tc_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, ld_dk, dv,
+                                                       ld_dv, dq_acc,
+                                                       static_cast<int64_t>(g.H) * 64, d_pos,
+                                                       d_time);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t n = static_cast<int64_t>(g.T) * g.H * 64;
+  const int64_t n = static_cast<int64_t>(g.T) * g.H * 8;  // 8 columns per thread
   f32_to_bf16_rows<<<static_cast<int>((n + 255) / 256), 256, 0, stream>>>(
-      dq_acc, static_cast<int64_t>(g.H) * 64, dq, ld, g.T, g.H * 64);
+      dq_acc, static_cast<int64_t>(g.H) * 64, dq, ld_dq, g.T, g.H * 64);
   return cudaGetLastError();
 }
 }  // namespace hstu
