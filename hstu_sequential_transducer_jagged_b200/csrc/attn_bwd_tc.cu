@@ -27,6 +27,8 @@
 // Items are visited in the reverse of the forward's longest-first order (which sorts by the
 // number of key tiles a query tile visits), so that key tiles near the start of long sequences,
 // which walk the most query tiles, start first.
+#include <climits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -90,7 +92,164 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Bias-gradient run: sums dS in registers while the table index stays the same and adds the
+// sum to the shared-memory bin when the index moves on.
+struct BinRun {
+  int idx;
+  float acc;
+  __device__ __forceinline__ void add(float* bins, int i, float v) {
+    if (i != idx) {
+      if (idx >= 0) atomicAdd(&bins[idx], acc);
+      idx = i;
+      acc = 0.f;
+    }
+    acc += v;
+  }
+  __device__ __forceinline__ void flush(float* bins) {
+    if (idx >= 0) atomicAdd(&bins[idx], acc);
+    idx = -1;
+    acc = 0.f;
+  }
+};
+
+// Per-thread constants of one item: the thread's key row and the tables.
+struct BwdRow {
+  int jrow, pj, n, L;
+  bool jvalid;
+  long long tj;
+};
+struct BwdTabs {
+  const float* pos;   // rab_pos copy in shared memory
+  const float* time;  // rab_time copy
+  float* bins_pos;    // gradient bins
+  float* bins_time;
+  float alpha;
+  int P, NB;
+  bool use_pos, use_time;
+};
+
+// Classes of a 32-query x 32-key block of one warp (warp-uniform): every pair hidden; every pair
+// visible with one position bin and one time bucket; every pair visible with one time bucket;
+// anything else (per-element mask, bias and bins).
+constexpr int kChunkGeneral = 0, kChunkTimeConst = 1, kChunkConst = 2, kChunkZero = 3;
+
+__device__ __forceinline__ long long warp_min64(long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const long long o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = o < v ? o : v;
+  }
+  return v;
+}
+__device__ __forceinline__ long long warp_max64(long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const long long o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = o > v ? o : v;
+  }
+  return v;
+}
+
+// Class of the block of queries i0 .. i0+31 and keys j0 .. j0+31.  tq_c: the block's query
+// timestamps (lane l reads entry l); tj_lo / tj_hi: the warp's key timestamp range.  For the two
+// constant classes it returns the constant bias terms (summed in the per-element path's order:
+// position, then time) and their bins.  Exact for every pair: the bucket rule is monotone in the
+// time difference and the position clamp in the distance.
+__device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const BwdTabs& t,
+                                           const long long* tq_c, long long tj_lo,
+                                           long long tj_hi, float& cbias, int& cpidx,
+                                           int& ctidx) {
+  const int j1 = j0 + 31;
+  if (i0 >= L || j0 >= L || i0 + 31 < j0) return kChunkZero;
+  if (!(i0 >= j1 && i0 + 31 < L && j1 < n)) return kChunkGeneral;  // not every pair visible
+  float tterm = 0.f;
+  ctidx = 0;
+  if (t.use_time) {
+    const long long tq = tq_c[threadIdx.x & 31];
+    const long long tq_lo = warp_min64(tq), tq_hi = warp_max64(tq);
+    const int b_lo = time_bucket64(tq_lo - tj_hi, t.NB);
+    const int b_hi = time_bucket64(tq_hi - tj_lo, t.NB);
+    if (b_lo != b_hi) return kChunkGeneral;
+    ctidx = b_lo;
+    tterm = t.time[b_lo];
+  }
+  cpidx = 0;
+  if (t.use_pos) {
+    // keys are history tokens (position = index); queries past the history sit at n
+    const int dmin = (i0 < n ? i0 : n) - j1;
+    if (dmin < t.P) {
+      cbias = tterm;
+      return kChunkTimeConst;
+    }
+    cpidx = 2 * t.P;  // every distance at or beyond the clamp
+    cbias = t.pos[cpidx] + tterm;
+    return kChunkConst;
+  }
+  cbias = tterm;
+  return kChunkConst;
+}
+
+// One 32-column block of a key row: P and alpha dS (bf16 pairs) from S and dP, and the bias
+// gradients.  i_first: query index of the block's first column; tq_c: its timestamps.
+template <int V>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
+                                          uint32_t (&pk)[16], uint32_t (&dk)[16], int i_first,
+                                          const long long* tq_c, const BwdRow& r,
+                                          const BwdTabs& t, float cbias, int cpidx, int ctidx,
+                                          BinRun& run_p, BinRun& run_t) {
+  float sum = 0.f;  // constant classes: the block's dS total for the constant bins
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pv[2], dsa[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i_first + e + u;
+      float bias;
+      int pidx = 0, bidx = 0;
+      if (V == kChunkConst) {
+        bias = cbias;
+      } else {
+        bias = 0.f;
+        if (t.use_pos) {
+          const int pi = i < r.n ? i : r.n;
+          int d = pi - r.pj;
+          d = d < -t.P ? -t.P : (d > t.P ? t.P : d);
+          pidx = d + t.P;
+          bias += t.pos[pidx];
+        }
+        if (V == kChunkTimeConst) {
+          bias += cbias;
+        } else if (t.use_time) {
+          bidx = time_bucket64(tq_c[e + u] - r.tj, t.NB);
+          bias += t.time[bidx];
+        }
+      }
+      const float x = fmaf(t.alpha, __uint_as_float(s[e + u]), bias);
+      const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
+      float p = x * sg;
+      float dsv = __uint_as_float(dp[e + u]) * sg * fmaf(x, 1.f - sg, 1.f);
+      if (V == kChunkGeneral) {
+        const bool vis = r.jvalid && i < r.L && r.jrow <= i && (r.jrow < r.n || r.jrow == i);
+        p = vis ? p : 0.f;
+        dsv = vis ? dsv : 0.f;
+        if (vis && t.use_pos) run_p.add(t.bins_pos, pidx, dsv);
+        if (vis && t.use_time) run_t.add(t.bins_time, bidx, dsv);
+      } else {
+        if (V == kChunkTimeConst && t.use_pos) run_p.add(t.bins_pos, pidx, dsv);
+        sum += dsv;
+      }
+      pv[u] = p;
+      dsa[u] = t.alpha * dsv;
+    }
+    pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+    dk[e >> 1] = pack_bf16x2(dsa[0], dsa[1]);
+  }
+  if (V == kChunkConst && t.use_pos) run_p.add(t.bins_pos, cpidx, sum);
+  if (V != kChunkGeneral && t.use_time) run_t.add(t.bins_time, ctidx, sum);
+}
+
 // Items: (sequence, 128-row key tile) from the work list built with one tile per item, times heads.
+template <bool kFast>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -260,8 +419,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Bias-gradient runs: along one key row the table index changes only where the clamped
     // distance or the time bucket changes, so each thread sums a run in registers and adds it
     // to the shared-memory bin when the index moves on.
-    int run_p = -1, run_t = -1;
-    float acc_p = 0.f, acc_t = 0.f;
+    BinRun run_p{-1, 0.f}, run_t{-1, 0.f};
+    BwdTabs tabs;
+    tabs.pos = tab_pos;
+    tabs.time = tab_time;
+    tabs.bins_pos = bins;
+    tabs.bins_time = bins + npos;
+    tabs.alpha = alpha;
+    tabs.P = g.P;
+    tabs.NB = g.NB;
+    tabs.use_pos = use_pos;
+    tabs.use_time = use_time;
     int gs = 0, jj = 0;
     bool ok = true;
     for (int w = blockIdx.x; ok && w < total; w += stride, ++jj) {
@@ -269,10 +437,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int head = w % g.H, kt = it.qtile, L = it.len;
       const int n = hist_len(L, g.mask, g.num_candidates);
       const int nt = (L + kT - 1) / kT;
-      const int jrow = kt * kT + quad * 32 + lane;  // this thread's key row
+      const int j0 = kt * kT + quad * 32;  // this warp's first key row
+      const int jrow = j0 + lane;          // this thread's key row
       const bool jvalid = jrow < L;
-      const int pj = jrow < n ? jrow : n;
-      const long long tj = (use_time && jvalid) ? g.ts[it.row0 + jrow] : 0;
+      BwdRow row;
+      row.jrow = jrow;
+      row.jvalid = jvalid;
+      row.pj = jrow < n ? jrow : n;
+      row.n = n;
+      row.L = L;
+      row.tj = (use_time && jvalid) ? g.ts[it.row0 + jrow] : 0;
+      long long tj_lo = 0, tj_hi = 0;  // the warp's key timestamp range (valid keys)
+      if (kFast && use_time) {
+        tj_lo = warp_min64(jvalid ? row.tj : LLONG_MAX);
+        tj_hi = warp_max64(jvalid ? row.tj : LLONG_MIN);
+      }
       for (int qt = kt; ok && qt < nt; ++qt, ++gs) {
         const int st = gs % kQStages;
         ok = warp_wait(&sm.s_full, gs & 1, abort_flag, g.status);
@@ -285,58 +464,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int ch = 0; ch < 2; ++ch) {  // 32 query columns per chunk
           const uint32_t col = 64 * hq + 32 * ch;
-          uint32_t s[32], dp[32];
-          tmem_ld32(lane_addr + kColST + col, s);
-          tmem_ld32(lane_addr + kColDPT + col, dp);
-          tmem_wait_ld32(s);
-          tmem_wait_ld32(dp);
+          const int i0 = qt * kT + static_cast<int>(col);
+          const long long* tq_c = tq + col;
+          float cbias = 0.f;
+          int cpidx = 0, ctidx = 0;
+          const int cls = kFast ? chunk_class(i0, j0, L, n, tabs, tq_c, tj_lo, tj_hi, cbias,
+                                              cpidx, ctidx)
+                                : kChunkGeneral;
           uint32_t pk[16], dk[16];
+          if (cls == kChunkZero) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2], dv2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int c = 64 * hq + 32 * ch + e + u;
-              const int i = qt * kT + c;
-              float bias = 0.f;
-              int pidx = 0, bidx = 0;
-              if (use_pos) {
-                const int pi = i < n ? i : n;
-                int d = pi - pj;
-                d = d < -g.P ? -g.P : (d > g.P ? g.P : d);
-                pidx = d + g.P;
-                bias += tab_pos[pidx];
-              }
-              if (use_time) {
-                bidx = time_bucket64(tq[c] - tj, g.NB);
-                bias += tab_time[bidx];
-              }
-              const bool vis = jvalid && i < L && jrow <= i && (jrow < n || jrow == i);
-              const float x = fmaf(alpha, __uint_as_float(s[e + u]), bias);
-              const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
-              const float p = x * sg;
-              const float dsv = vis ? __uint_as_float(dp[e + u]) * sg * fmaf(x, 1.f - sg, 1.f) : 0.f;
-              pv[u] = vis ? p : 0.f;
-              dv2[u] = alpha * dsv;
-              if (vis && use_pos) {
-                if (pidx != run_p) {
-                  if (run_p >= 0) atomicAdd(&bins[run_p], acc_p);
-                  run_p = pidx;
-                  acc_p = 0.f;
-                }
-                acc_p += dsv;
-              }
-              if (vis && use_time) {
-                if (bidx != run_t) {
-                  if (run_t >= 0) atomicAdd(&bins[npos + run_t], acc_t);
-                  run_t = bidx;
-                  acc_t = 0.f;
-                }
-                acc_t += dsv;
-              }
-            }
-            pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-            dk[e >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+            for (int z = 0; z < 16; ++z) pk[z] = dk[z] = 0u;
+          } else {
+            uint32_t s[32], dp[32];
+            tmem_ld32(lane_addr + kColST + col, s);
+            tmem_ld32(lane_addr + kColDPT + col, dp);
+            tmem_wait_ld32(s);
+            tmem_wait_ld32(dp);
+            if (cls == kChunkConst)
+              bwd_chunk<kChunkConst>(s, dp, pk, dk, i0, tq_c, row, tabs, cbias, cpidx, ctidx,
+                                     run_p, run_t);
+            else if (cls == kChunkTimeConst)
+              bwd_chunk<kChunkTimeConst>(s, dp, pk, dk, i0, tq_c, row, tabs, cbias, cpidx,
+                                         ctidx, run_p, run_t);
+            else
+              bwd_chunk<kChunkGeneral>(s, dp, pk, dk, i0, tq_c, row, tabs, cbias, cpidx, ctidx,
+                                       run_p, run_t);
           }
           // P^T / (a dS)^T over the already-read first half of this warp's 64 columns
           tmem_st16(lane_addr + kColST + 64 * hq + 16 * ch, pk);
@@ -385,8 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty);
     }
-    if (run_p >= 0) atomicAdd(&bins[run_p], acc_p);
-    if (run_t >= 0) atomicAdd(&bins[npos + run_t], acc_t);
+    run_p.flush(tabs.bins_pos);
+    run_t.flush(tabs.bins_time);
   } else if (warp >= 12) {
     // ---------------------------------------------------------------- dQ drain
     const int quad = warp & 3;
@@ -468,26 +621,29 @@ size_t attn_bwd_tc_smem(int P, int NB) {
 // Launches the backward over the work list in g (one 128-row tile per item): tq / tk / tv / tdo
 // are 64 x 128 boxes (128-byte swizzle) over Q, K, V, dO; tts a 130-element int64 box over the
 // timestamps (used when g.ts and g.rab_time are set).  dq_acc: fp32 [T, H*64], zeroed here.
-// grid: at most one CTA per SM (persistent).  Returns cudaErrorInvalidValue when the bias
-// tables do not fit in shared memory.
+// grid: at most one CTA per SM (persistent).  fast: classify each 32 x 32 block of a warp
+// (hidden, visible with constant bias terms, visible with a constant time term) and skip the
+// per-element work these make unnecessary; otherwise every element takes the per-element path.
+// Both give the same P and dS values.  Returns cudaErrorInvalidValue when the bias tables do
+// not fit in shared memory.
 cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdo,
                                const CUtensorMap& tts, const AttnGeom& g,
                                __nv_bfloat16* dq, int64_t ld_dq, __nv_bfloat16* dk,
                                int64_t ld_dk, __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc,
-                               float* d_pos, float* d_time, int grid, cudaStream_t stream) {
+                               float* d_pos, float* d_time, int grid, bool fast,
+                               cudaStream_t stream) {
   const size_t smem = attn_bwd_tc_smem(g.rab_pos ? g.P : 0, g.rab_time ? g.NB : 0);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   // d_pos / d_time are accumulated into: the caller zeroes them
   cudaError_t e = cudaMemsetAsync(dq_acc, 0, sizeof(float) * g.T * g.H * 64, stream);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+  auto kernel = fast ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  attn_bwd_tc_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, ld_dk, dv,
-                                                       ld_dv, dq_acc,
-                                                       static_cast<int64_t>(g.H) * 64, d_pos,
-                                                       d_time);
+  kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, ld_dk, dv, ld_dv, dq_acc,
+                                           static_cast<int64_t>(g.H) * 64, d_pos, d_time);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(g.T) * g.H * 8;  // 8 columns per thread
