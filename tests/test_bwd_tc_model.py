@@ -1,0 +1,70 @@
+"""The tensor-core backward's data movement, modelled on the CPU (tests/bwd_tc_model.py),
+against the oracle's chain rule for the attention backward ("6.2 HSTU的工程突破" §6.2.3 names the
+rab gradient it includes).
+
+The model uses the kernel's own address arithmetic for every shared- and tensor-memory access
+and the canonical operand layouts for what the MMAs read.  So it checks that each operand lands
+where its reader expects it, for both epilogue forms (per element, and classified 32 x 32
+blocks), before the kernel runs on hardware.  Each planted layout mistake must make it fail.
+"""
+import numpy as np
+import pytest
+
+from oracle import hstu_oracle as O
+from hstu_sequential_transducer_jagged_b200 import workloads as W
+import bwd_tc_model as M  # noqa: E402  (tests/ is on sys.path under pytest)
+
+ROW_TOL, ABS_TOL, FRO_TOL = 2e-2, 1e-3, 5e-3
+
+
+def within(got, ref, bf16_out):
+    g = M.bits_to_f32(M.bf16_bits(got)) if bf16_out else got
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    bound = ROW_TOL * (np.abs(r).max(axis=-1, keepdims=True) if r.ndim > 1
+                       else np.abs(r).max()) + ABS_TOL
+    fro = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+    return bool((np.abs(g - r) <= bound).all() and fro <= FRO_TOL)
+
+
+def oracle(case):
+    return O.attention_backward(case.q, case.k, case.v, case.d_o, case.seq_offsets,
+                                case.timestamps, case.rab_pos, case.rab_time,
+                                num_heads=case.num_heads, d_qk=case.d_qk, d_v=case.d_v,
+                                max_pos_dist=case.max_pos_dist,
+                                num_time_buckets=case.num_time_buckets, alpha=case.alpha,
+                                mask=case.mask, num_candidates=case.num_candidates)
+
+
+CASES = {
+    "causal": lambda: W.random_attention_case(30, [200, 1, 129, 77], H=2, d=64, P=20, NB=16,
+                                              gap_mean=20.0, qkv_std=0.5),
+    "mfalcon": lambda: W.random_attention_case(80, [200, 1, 129, 77], H=2, d=64, P=20, NB=16,
+                                               mask=W.MASK_MFALCON, num_candidates=50,
+                                               gap_mean=20.0, qkv_std=0.5),
+    "far pairs": lambda: W.random_attention_case(31, [700, 300], H=1, d=64, P=64, NB=32,
+                                                 gap_mean=600.0, qkv_std=0.5),
+}
+
+
+@pytest.mark.parametrize("fast", [False, True])
+@pytest.mark.parametrize("name", list(CASES))
+def test_model_matches_oracle(name, fast):
+    case = CASES[name]()
+    got = M.run(case, fast)
+    ref = oracle(case)
+    for nm, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got, ref):
+        assert within(g, r, nm in ("dq", "dk", "dv")), f"{name} fast={fast}: {nm}"
+
+
+@pytest.mark.parametrize("knob", [dict(ds_swizzle=False), dict(dq_lbo=8192),
+                                  dict(split_pc=False), dict(p_col_step=32)])
+def test_planted_layout_mistakes_fail(knob):
+    case = CASES["causal"]()
+    with np.errstate(all="ignore"):  # misplaced operands read garbage
+        got = M.run(case, True, knob)
+    ref = oracle(case)
+    with np.errstate(all="ignore"):
+        assert not all(within(g, r, nm in ("dq", "dk", "dv"))
+                       for nm, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got,
+                                           ref))
