@@ -29,7 +29,7 @@ EXPORTED = [
     "hstu_jagged_padded_copy",
     "hstu_debug_time_buckets", "hstu_workspace_init", "hstu_sync_status",
     "hstu_status_string", "hstu_version", "hstu_last_error_string",
-    "hstu_attention_forward_static_ws",
+    "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout",
 ]
 
 
@@ -96,6 +96,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_version": (ctypes.c_char_p, []),
         "hstu_last_error_string": (ctypes.c_char_p, []),
         "hstu_attention_forward_static_ws": (i32, [adp, vp, vp, vp, vp, vp, vp]),
+        "hstu_debug_wait_timeout": (i32, [vp, sz, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -306,6 +307,12 @@ def layer_forward(x, w1, w2, seq_offsets, max_seq_len, timestamps=None, rab_pos=
                                     _ptr(b2), _ptr(out), ws.ptr, ws.nbytes, _stream_ptr(stream)),
            "hstu_layer_forward")
     return out
+
+
+def debug_wait_timeout(ws: Workspace, stream=None) -> None:
+    """Launch the bounded-wait probe; ws.sync_status() then reports HSTU_ERR_TIMEOUT (5)."""
+    _check(lib().hstu_debug_wait_timeout(ws.ptr, ws.nbytes, _stream_ptr(stream)),
+           "hstu_debug_wait_timeout")
 
 
 def debug_time_buckets(dt: torch.Tensor, nb: int, stream=None) -> torch.Tensor:

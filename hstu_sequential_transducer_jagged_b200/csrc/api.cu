@@ -40,6 +40,7 @@ cudaError_t launch_jagged_padded(const int32_t* offsets, int B, int max_len, con
                                  cudaStream_t stream);
 cudaError_t launch_time_buckets(const int64_t* dt, int n, int32_t* out, int nb,
                                 cudaStream_t stream);
+cudaError_t launch_wait_timeout_probe(int32_t* status, cudaStream_t stream);
 cudaError_t launch_attn_fwd_simt(int dtype, int D, const AttnGeom& g, const void* q, int64_t ld_q,
                                  const void* k, int64_t ld_k, const void* v, int64_t ld_v,
                                  void* o, int64_t ld_o, int grid, cudaStream_t stream);
@@ -477,6 +478,13 @@ hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out
   if (n == 0) return HSTU_OK;
   if (dt == nullptr || out == nullptr) return HSTU_ERR_INVALID_ARG;
   cudaError_t e = launch_time_buckets(dt, n, out, nb, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+}
+
+hstu_status_t hstu_debug_wait_timeout(void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (check_ws(ws, ws_bytes, kStatusBytes) != HSTU_OK) return HSTU_ERR_WORKSPACE;
+  cudaError_t e = launch_wait_timeout_probe(static_cast<int32_t*>(ws),
+                                            reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 

@@ -263,6 +263,27 @@ cudaError_t launch_jagged_padded(const int32_t* offsets, int B, int max_len, con
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------- bounded-wait probe
+// One mbarrier whose phase nothing completes, waited on with the bounded wait every kernel of
+// the library uses: the wait gives up after its limit, writes the timeout code into the status
+// word and the kernel returns, so the failure reaches the host and the context stays usable.
+__global__ void wait_timeout_probe_kernel(int32_t* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status);
+}
+
+cudaError_t launch_wait_timeout_probe(int32_t* status, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------------- time buckets
 __global__ void time_bucket_kernel(const int64_t* __restrict__ dt, int n, int32_t* __restrict__ out,
                                    int nb) {

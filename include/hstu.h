@@ -201,6 +201,15 @@ hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_se
                                       int64_t padded_row_stride_bytes, int64_t row_bytes,
                                       int32_t to_padded, hstu_stream_t stream);
 
+/* Failure-path check of the status word: launches one CTA that waits, with the bounded wait
+ * every kernel of the library uses, on a barrier phase that nothing completes.  The wait gives
+ * up after its limit (2 s), writes HSTU_ERR_TIMEOUT into the status word of ws and the kernel
+ * returns; the next hstu_sync_status(ws) reports HSTU_ERR_TIMEOUT and clears the word, and the
+ * context stays usable.  ws: device workspace of at least 256 bytes, 256-byte aligned, owned by
+ * the caller.  Returns HSTU_ERR_WORKSPACE for a missing, misaligned or short ws (nothing is
+ * launched), HSTU_ERR_CUDA if the launch fails, else HSTU_OK (asynchronous on stream). */
+hstu_status_t hstu_debug_wait_timeout(void* ws, size_t ws_bytes, hstu_stream_t stream);
+
 /* Debug export of the time-bias bucket rule: out[i] = clamp(floor(log2(max(1, dt[i]))), 0,
  * nb-1), computed on the device by the same code the attention kernels inline, so it can be
  * compared bit-exactly with an integer reference.  dt, out: device [n]. */

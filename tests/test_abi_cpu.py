@@ -157,3 +157,9 @@ def test_static_scratch_call_rejects_on_the_host(lib):
                                                 None) == 3
     msg = lib.hstu_last_error_string().decode()
     assert str(need) in msg and str(limit) in msg
+
+
+def test_wait_timeout_probe_rejects_bad_workspace(lib):
+    assert lib.hstu_debug_wait_timeout(None, 256, None) == 3
+    assert lib.hstu_debug_wait_timeout(ctypes.c_void_p((1 << 20) + 8), 256, None) == 3
+    assert lib.hstu_debug_wait_timeout(FAKE, 100, None) == 3
