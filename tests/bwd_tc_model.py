@@ -109,6 +109,31 @@ def time_bucket64(dt, nb):
     return O.time_bucket(np.asarray(dt, dtype=np.int64), nb)
 
 
+def chunk_class(i0, j0, L, n, P, NB, tq_c, tj, jvalid, tabp, tabt, use_pos=True,
+                use_time=True):
+    """The epilogue's class of the block of queries i0 .. i0+31 and keys j0 .. j0+31 (as in the
+    kernel's chunk_class): ("zero" | "const" | "timeconst" | "general", constant bias, position
+    bin, time bucket)."""
+    j1 = j0 + 31
+    if i0 >= L or j0 >= L or i0 + 31 < j0:
+        return "zero", np.float32(0), 0, 0
+    if not (i0 >= j1 and i0 + 31 < L and j1 < n):
+        return "general", np.float32(0), 0, 0
+    tterm, ctidx = np.float32(0), 0
+    if use_time:
+        tj_lo, tj_hi = tj[jvalid].min(), tj[jvalid].max()
+        b_lo = int(time_bucket64(tq_c[:32].min() - tj_hi, NB))
+        b_hi = int(time_bucket64(tq_c[:32].max() - tj_lo, NB))
+        if b_lo != b_hi:
+            return "general", np.float32(0), 0, 0
+        ctidx, tterm = b_lo, tabt[b_lo]
+    if use_pos:
+        if min(i0, n) - j1 < P:
+            return "timeconst", np.float32(tterm), 0, ctidx
+        return "const", np.float32(tabp[2 * P] + tterm), 2 * P, ctidx
+    return "const", np.float32(tterm), 0, ctidx
+
+
 DEFAULT_KNOBS = dict(ds_swizzle=True, dq_lbo=kTileBytes, split_pc=True, p_col_step=16)
 
 
@@ -198,21 +223,8 @@ def run(case, fast, knobs=None):
                             tq_c = tq[col:col + 32]
                             cls, cbias, cpidx, ctidx = "general", np.float32(0), 0, 0
                             if fast:
-                                j1 = j0 + 31
-                                if i0 >= L or j0 >= L or i0 + 31 < j0:
-                                    cls = "zero"
-                                elif i0 >= j1 and i0 + 31 < L and j1 < n:
-                                    tj_lo, tj_hi = tj[jvalid].min(), tj[jvalid].max()
-                                    b_lo = int(time_bucket64(tq_c.min() - tj_hi, NB))
-                                    b_hi = int(time_bucket64(tq_c.max() - tj_lo, NB))
-                                    if b_lo == b_hi:
-                                        ctidx, tterm = b_lo, tabt[b_lo]
-                                        dmin = min(i0, n) - j1
-                                        if dmin < P:
-                                            cls, cbias = "timeconst", np.float32(tterm)
-                                        else:
-                                            cls, cpidx = "const", 2 * P
-                                            cbias = np.float32(tabp[cpidx] + tterm)
+                                cls, cbias, cpidx, ctidx = chunk_class(i0, j0, L, n, P, NB, tq_c,
+                                                                       tj, jvalid, tabp, tabt)
                             if cls == "zero":
                                 pk = np.zeros((32, 16), dtype=np.uint32)
                                 dk_ = np.zeros((32, 16), dtype=np.uint32)

@@ -68,3 +68,52 @@ def test_planted_layout_mistakes_fail(knob):
         assert not all(within(g, r, nm in ("dq", "dk", "dv"))
                        for nm, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got,
                                            ref))
+
+
+def test_block_classes_exact():
+    """Brute force over random blocks: every pair of a constant block is visible and has the
+    claimed position bin and time bucket; every pair of a zero block is hidden (causal and
+    M-FALCON masks, sorted and shuffled timestamps, gaps from 1 s to 10^7 s)."""
+    rng = np.random.default_rng(1)
+    seen = set()
+    for _ in range(400):
+        L = int(rng.integers(1, 700))
+        mfal = bool(rng.random() < 0.4)
+        m = int(rng.integers(0, min(L, 200) + 1)) if mfal else 0
+        mask = O.MASK_MFALCON if mfal else O.MASK_CAUSAL
+        n = max(L - m, 0) if mfal else L
+        P, NB = int(rng.choice([4, 20, 64, 300])), int(rng.choice([8, 16, 64]))
+        ts = np.floor(np.cumsum(rng.exponential(float(rng.choice([1.0, 600.0, 1e7])), L)))
+        ts = ts.astype(np.int64)
+        if mfal and n > 0:
+            ts[n:] = ts[n - 1]
+        if rng.random() < 0.2:
+            rng.shuffle(ts)
+        ok = O.allowed_pairs(L, mask, m)
+        pidx = O.position_index(O.positions(L, mask, m)[:, None] - O.positions(L, mask, m)[None, :], P)
+        tidx = O.time_bucket(ts[:, None] - ts[None, :], NB)
+        tpad = np.concatenate([ts, np.zeros(256, np.int64)])
+        tabp, tabt = np.zeros(2 * P + 1, np.float32), np.zeros(NB, np.float32)
+        nt = (L + 127) // 128
+        for _ in range(4):
+            kt = int(rng.integers(0, nt))
+            qt = int(rng.integers(kt, nt))
+            i0 = qt * 128 + int(rng.choice([0, 32, 64, 96]))
+            j0 = kt * 128 + 32 * int(rng.integers(0, 4))
+            jrow = j0 + np.arange(32)
+            cls, _, cp, ct = M.chunk_class(i0, j0, L, n, P, NB, tpad[i0:i0 + 32],
+                                           tpad[np.minimum(jrow, len(tpad) - 1)], jrow < L,
+                                           tabp, tabt)
+            seen.add(cls)
+            ii, jj = np.meshgrid(np.arange(i0, i0 + 32), jrow, indexing="ij")
+            inside = (ii < L) & (jj < L)
+            vis = np.zeros_like(inside)
+            vis[inside] = ok[ii[inside], jj[inside]]
+            if cls == "zero":
+                assert not vis.any()
+            elif cls in ("const", "timeconst"):
+                assert vis.all()
+                assert (tidx[ii, jj] == ct).all()
+                if cls == "const":
+                    assert (pidx[ii, jj] == cp).all()
+    assert seen == {"zero", "general", "const", "timeconst"}
