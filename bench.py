@@ -321,7 +321,11 @@ def run_attention_bwd(args, lib, Bd, dev):
                       "fwd_ms": res["fwd"],
                       "fwd_tflops": 4.0 * wl.d_qk * pairs / (res["fwd"] / 1e3) / 1e12,
                       "bwd_ms": res["bwd"],
-                      "bwd_tflops": 8.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12}),
+                      "bwd_tflops": 8.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12,
+                      # the recomputation of S = QK^T (2 d per pair), reported apart
+                      "bwd_recompute_gflop": 2.0 * wl.d_qk * pairs / 1e9,
+                      "bwd_tflops_incl_recompute":
+                          10.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12}),
           flush=True)
 
 
