@@ -219,6 +219,38 @@ def test_attention_timestamp_shift_invariance_and_linearity_in_v():
     np.testing.assert_allclose(a, 2.0 * base + b, rtol=1e-12, atol=1e-12)
 
 
+def test_attention_keeps_interaction_intensity():
+    """The worked example of "HSTU：Scaling Law 的首次探索" §7.1.4, innovation 1: user A clicks
+    technology 10 times and entertainment once, user B 100 and 10 times.  A softmax gives both
+    the same 90 % / 10 % mixture; pointwise aggregation keeps B's tenfold intensity.  With the
+    same key and value per interest, no bias terms and a final query token whose own key is zero
+    (its own term is SiLU(0) = 0), B's output there is exactly ten times A's, while the weights
+    normalised to sum 1 (what a softmax would use) are the same for both users."""
+    rng = np.random.default_rng(3)
+    d = 8
+    k_tech, k_ent, v_tech, v_ent, q = (rng.normal(size=d) for _ in range(5))
+
+    def user(n_tech, n_ent):
+        L = n_tech + n_ent + 1
+        K = np.vstack([np.tile(k_tech, (n_tech, 1)), np.tile(k_ent, (n_ent, 1)), np.zeros(d)])
+        V = np.vstack([np.tile(v_tech, (n_tech, 1)), np.tile(v_ent, (n_ent, 1)),
+                       rng.normal(size=d)])
+        Q = np.zeros((L, d))
+        Q[-1] = q
+        out = O.attention_forward(Q, K, V, np.array([0, L]), None, None, None, num_heads=1,
+                                  d_qk=d, d_v=d, max_pos_dist=0, num_time_buckets=1,
+                                  rows=np.array([L - 1]))
+        w = O.silu(np.array([q @ k_tech, q @ k_ent]))
+        mix = np.array([n_tech, n_ent]) * w
+        return out[L - 1], mix / mix.sum()
+
+    out_a, mix_a = user(10, 1)
+    out_b, mix_b = user(100, 10)
+    assert np.allclose(out_b, 10.0 * out_a, rtol=1e-12, atol=0)
+    assert np.allclose(mix_a, mix_b, rtol=1e-12, atol=0)
+    assert not np.allclose(out_b, out_a)
+
+
 def test_attention_rows_subset_equals_full():
     case = W.random_attention_case(7, [20, 3, 17], H=2, d=4, P=6, NB=10, bf16=False)
     full = O.attention_forward(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
