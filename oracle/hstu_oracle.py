@@ -358,3 +358,70 @@ def stack_forward(x, layers, seq_offsets, timestamps, *, num_heads, d_qk, d_v, m
         if round_between is not None:
             h = np.asarray(round_between(h), dtype=np.float64)
     return h
+
+
+# --------------------------------------------------------------------------------------------
+# the layer's backward, for training the stack end to end ([FunRec 7.1] §7.1.3: the whole
+# user sequence is trained in one causal pass; [Review §2.1] the three layer formulas): the
+# chain rule through Y = X + f2(Norm(A(X)V(X)) ⊙ U(X)), written out step by step in fp64
+# --------------------------------------------------------------------------------------------
+
+def layer_norm_backward(a, d_out, eps=1e-5, gamma=None):
+    """Gradient of Σ d_out ⊙ Norm(a) with respect to a, gamma and beta (last axis normalised).
+
+    With n = (a - mean) / sqrt(var + eps) and out = n ⊙ gamma + beta: dn = d_out ⊙ gamma;
+    da = (dn - mean(dn) - n ⊙ mean(dn ⊙ n)) / sqrt(var + eps); dgamma = Σ_rows d_out ⊙ n;
+    dbeta = Σ_rows d_out.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    d_out = np.asarray(d_out, dtype=np.float64)
+    mu = a.mean(axis=-1, keepdims=True)
+    xc = a - mu
+    rstd = 1.0 / np.sqrt((xc ** 2).mean(axis=-1, keepdims=True) + eps)
+    n = xc * rstd
+    dn = d_out if gamma is None else d_out * np.asarray(gamma, dtype=np.float64)
+    da = rstd * (dn - dn.mean(axis=-1, keepdims=True) - n * (dn * n).mean(axis=-1, keepdims=True))
+    return da, (d_out * n).sum(axis=0), d_out.sum(axis=0)
+
+
+def layer_backward(x, w1, w2, seq_offsets, timestamps, rab_pos, rab_time, d_y, *, num_heads,
+                   d_qk, d_v, max_pos_dist, num_time_buckets, alpha=1.0, mask=MASK_CAUSAL,
+                   num_candidates=0, b1=None, b2=None, ln_eps=1e-5, ln_gamma=None,
+                   ln_beta=None):
+    """Gradients of L = Σ d_y ⊙ Y for one layer, Y = layer_forward(...).
+
+    Forward: pre = X W1 + b1, Z = SiLU(pre) = [U | V | Q | K], AV = A(X)V(X),
+    G = Norm(AV) ⊙ U, Y = X + G W2 + b2.  Backward, in reverse order:
+      dW2 = Gᵀ dY, db2 = Σ dY, dG = dY W2ᵀ;
+      dU = dG ⊙ Norm(AV), dNorm = dG ⊙ U, (dAV, dgamma, dbeta) = Norm backward;
+      (dQ, dK, dV, d rab_pos, d rab_time) = attention backward of dAV;
+      dZ = [dU | dV | dQ | dK], dpre = dZ ⊙ SiLU'(pre);
+      dW1 = Xᵀ dpre, db1 = Σ dpre, dX = dY (residual edge) + dpre W1ᵀ.
+    Returns a dict with dx, dw1, db1, dw2, db2, d_rab_pos, d_rab_time, d_ln_gamma, d_ln_beta.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w1 = np.asarray(w1, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64)
+    dy = np.asarray(d_y, dtype=np.float64)
+    pre = linear(x, w1, b1)
+    z = silu(pre)
+    u, v, q, k = split_uvqk(z, num_heads, d_qk, d_v)
+    av = attention_forward(q, k, v, seq_offsets, timestamps, rab_pos, rab_time,
+                           num_heads=num_heads, d_qk=d_qk, d_v=d_v, max_pos_dist=max_pos_dist,
+                           num_time_buckets=num_time_buckets, alpha=alpha, mask=mask,
+                           num_candidates=num_candidates)
+    nrm = layer_norm(av, ln_eps, ln_gamma, ln_beta)
+    g = nrm * u
+    dw2 = g.T @ dy
+    db2 = dy.sum(axis=0)
+    dg = dy @ w2.T
+    du = dg * nrm
+    d_av, d_gamma, d_beta = layer_norm_backward(av, dg * u, ln_eps, ln_gamma)
+    dq, dk, dv, d_pos, d_time = attention_backward(
+        q, k, v, d_av, seq_offsets, timestamps, rab_pos, rab_time, num_heads=num_heads,
+        d_qk=d_qk, d_v=d_v, max_pos_dist=max_pos_dist, num_time_buckets=num_time_buckets,
+        alpha=alpha, mask=mask, num_candidates=num_candidates)
+    dz = np.concatenate([du, dv, dq, dk], axis=1)
+    dpre = dz * silu_grad(pre)
+    return dict(dx=dy + dpre @ w1.T, dw1=x.T @ dpre, db1=dpre.sum(axis=0), dw2=dw2, db2=db2,
+                d_rab_pos=d_pos, d_rab_time=d_time, d_ln_gamma=d_gamma, d_ln_beta=d_beta)

@@ -452,3 +452,68 @@ def test_layer_rows_equals_full_and_stack_composes():
     ref = O.layer_forward(full, l2.w1, l2.w2, c.seq_offsets, c.timestamps, l2.rab_pos,
                           l2.rab_time, **_layer_kw(c))
     np.testing.assert_allclose(st, ref, rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------------------------------- layer backward
+def _tiny_layer(seed=7, mask=O.MASK_CAUSAL, m=0):
+    rng = np.random.default_rng(seed)
+    H, d, dm = 2, 3, 5
+    offsets = np.array([0, 4, 5, 9])
+    T = int(offsets[-1])
+    ts = np.concatenate([np.cumsum(rng.integers(0, 9, size=int(b - a)))
+                         for a, b in zip(offsets[:-1], offsets[1:])]).astype(np.int64)
+    p = dict(x=rng.normal(size=(T, dm)), w1=0.5 * rng.normal(size=(dm, 4 * H * d)),
+             w2=0.5 * rng.normal(size=(H * d, dm)), b1=0.1 * rng.normal(size=4 * H * d),
+             b2=0.1 * rng.normal(size=dm), rab_pos=0.3 * rng.normal(size=2 * 2 + 1),
+             rab_time=0.3 * rng.normal(size=4), ln_gamma=1 + 0.2 * rng.normal(size=H * d),
+             ln_beta=0.1 * rng.normal(size=H * d))
+    kw = dict(num_heads=H, d_qk=d, d_v=d, max_pos_dist=2, num_time_buckets=4, alpha=0.7,
+              mask=mask, num_candidates=m, ln_eps=1e-5)
+    return p, offsets, ts, kw, rng.normal(size=(T, dm))
+
+
+def _layer_loss(p, offsets, ts, kw, dy):
+    y = O.layer_forward(p["x"], p["w1"], p["w2"], offsets, ts, p["rab_pos"], p["rab_time"],
+                        b1=p["b1"], b2=p["b2"], ln_gamma=p["ln_gamma"], ln_beta=p["ln_beta"],
+                        **kw)
+    return float((dy * y).sum())
+
+
+@pytest.mark.parametrize("mask,m", [(O.MASK_CAUSAL, 0), (O.MASK_MFALCON, 2)])
+def test_layer_backward_finite_differences(mask, m):
+    """Every gradient of the layer (input, both projections and biases, both bias tables, the
+    LayerNorm affine) against central finite differences of Σ dY ⊙ Y in fp64."""
+    p, offsets, ts, kw, dy = _tiny_layer(mask=mask, m=m)
+    g = O.layer_backward(p["x"], p["w1"], p["w2"], offsets, ts, p["rab_pos"], p["rab_time"], dy,
+                         b1=p["b1"], b2=p["b2"], ln_gamma=p["ln_gamma"], ln_beta=p["ln_beta"],
+                         **kw)
+    names = dict(x="dx", w1="dw1", w2="dw2", b1="db1", b2="db2", rab_pos="d_rab_pos",
+                 rab_time="d_rab_time", ln_gamma="d_ln_gamma", ln_beta="d_ln_beta")
+    h = 1e-6
+    for key, gname in names.items():
+        arr = p[key]
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + h
+            lp = _layer_loss(p, offsets, ts, kw, dy)
+            arr[idx] = old - h
+            lm = _layer_loss(p, offsets, ts, kw, dy)
+            arr[idx] = old
+            num[idx] = (lp - lm) / (2 * h)
+        scale = max(np.abs(num).max(), 1e-3)
+        assert np.abs(g[gname] - num).max() <= 1e-6 * scale + 1e-8, key
+
+
+def test_layer_backward_zero_w2_passes_dy_through():
+    """With W2 = 0 the branch contributes nothing: dX = dY exactly (the residual edge), and
+    every gradient upstream of f2 vanishes while dW2 = Gᵀ dY does not."""
+    p, offsets, ts, kw, dy = _tiny_layer(seed=8)
+    p["w2"][:] = 0.0
+    g = O.layer_backward(p["x"], p["w1"], p["w2"], offsets, ts, p["rab_pos"], p["rab_time"], dy,
+                         b1=p["b1"], b2=p["b2"], ln_gamma=p["ln_gamma"], ln_beta=p["ln_beta"],
+                         **kw)
+    assert np.array_equal(g["dx"], dy)
+    for name in ("dw1", "db1", "d_rab_pos", "d_rab_time", "d_ln_gamma", "d_ln_beta"):
+        assert not np.any(g[name]), name
+    assert np.abs(g["dw2"]).max() > 0
