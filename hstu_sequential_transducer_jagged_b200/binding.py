@@ -29,7 +29,7 @@ EXPORTED = [
     "hstu_jagged_padded_copy",
     "hstu_debug_time_buckets", "hstu_workspace_init", "hstu_sync_status",
     "hstu_status_string", "hstu_version", "hstu_last_error_string",
-    "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout",
+    "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout", "hstu_alibi_tables",
 ]
 
 
@@ -97,6 +97,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_last_error_string": (ctypes.c_char_p, []),
         "hstu_attention_forward_static_ws": (i32, [adp, vp, vp, vp, vp, vp, vp]),
         "hstu_debug_wait_timeout": (i32, [vp, sz, vp]),
+        "hstu_alibi_tables": (i32, [ctypes.c_float, ctypes.c_float, i32, i32, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -307,6 +308,18 @@ def layer_forward(x, w1, w2, seq_offsets, max_seq_len, timestamps=None, rab_pos=
                                     _ptr(b2), _ptr(out), ws.ptr, ws.nbytes, _stream_ptr(stream)),
            "hstu_layer_forward")
     return out
+
+
+def alibi_tables(m_p: float, m_t: float, max_pos_dist: int, num_time_buckets: int):
+    """Host tables (numpy float32) that give the attention the bias -m_p (p_i - p_j) -
+    m_t bucket(t_i - t_j) (exact where |p_i - p_j| <= max_pos_dist)."""
+    import numpy as np
+    pos = np.empty(2 * max_pos_dist + 1, dtype=np.float32)
+    tim = np.empty(num_time_buckets, dtype=np.float32)
+    _check(lib().hstu_alibi_tables(m_p, m_t, max_pos_dist, num_time_buckets,
+                                   pos.ctypes.data_as(ctypes.c_void_p),
+                                   tim.ctypes.data_as(ctypes.c_void_p)), "hstu_alibi_tables")
+    return pos, tim
 
 
 def debug_wait_timeout(ws: Workspace, stream=None) -> None:

@@ -481,6 +481,18 @@ hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
+hstu_status_t hstu_alibi_tables(float m_p, float m_t, int32_t max_pos_dist,
+                                int32_t num_time_buckets, float* rab_pos, float* rab_time) {
+  if (!std::isfinite(m_p) || !std::isfinite(m_t) || max_pos_dist < 0 || num_time_buckets < 1)
+    return HSTU_ERR_INVALID_ARG;
+  if (rab_pos != nullptr)
+    for (int32_t k = 0; k <= 2 * max_pos_dist; ++k)
+      rab_pos[k] = -m_p * static_cast<float>(k - max_pos_dist);
+  if (rab_time != nullptr)
+    for (int32_t b = 0; b < num_time_buckets; ++b) rab_time[b] = -m_t * static_cast<float>(b);
+  return HSTU_OK;
+}
+
 hstu_status_t hstu_debug_wait_timeout(void* ws, size_t ws_bytes, hstu_stream_t stream) {
   if (check_ws(ws, ws_bytes, kStatusBytes) != HSTU_OK) return HSTU_ERR_WORKSPACE;
   cudaError_t e = launch_wait_timeout_probe(static_cast<int32_t*>(ws),

@@ -201,6 +201,17 @@ hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_se
                                       int64_t padded_row_stride_bytes, int64_t row_bytes,
                                       int32_t to_padded, hstu_stream_t stream);
 
+/* Tables for the parameter-free relative bias of "6.2 HSTU的工程突破" §6.2.3, Eq. (6.2.6):
+ * bias(i, j) = -m_p (p_i - p_j) - m_t bucket(t_i - t_j).  The bias is linear in the integer
+ * position difference and in the bucket index, so it is the learned-table bias with
+ * rab_pos[k] = -m_p (k - P) (k = 0 .. 2P) and rab_time[b] = -m_t b (b = 0 .. NB-1): pass these
+ * tables to the attention or layer calls with max_pos_dist = P.  The position term is exact only
+ * where |p_i - p_j| <= P, so take P >= the longest sequence length - 1.  Host arrays owned by the
+ * caller, [2P+1] and [NB] floats; either may be NULL to skip it.  Returns HSTU_ERR_INVALID_ARG
+ * for a non-finite slope, P < 0 or NB < 1; no device work. */
+hstu_status_t hstu_alibi_tables(float m_p, float m_t, int32_t max_pos_dist,
+                                int32_t num_time_buckets, float* rab_pos, float* rab_time);
+
 /* Failure-path check of the status word: launches one CTA that waits, with the bounded wait
  * every kernel of the library uses, on a barrier phase that nothing completes.  The wait gives
  * up after its limit (2 s), writes HSTU_ERR_TIMEOUT into the status word of ws and the kernel

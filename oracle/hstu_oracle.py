@@ -425,3 +425,43 @@ def layer_backward(x, w1, w2, seq_offsets, timestamps, rab_pos, rab_time, d_y, *
     dpre = dz * silu_grad(pre)
     return dict(dx=dy + dpre @ w1.T, dw1=x.T @ dpre, db1=dpre.sum(axis=0), dw2=dw2, db2=db2,
                 d_rab_pos=d_pos, d_rab_time=d_time, d_ln_gamma=d_gamma, d_ln_beta=d_beta)
+
+
+# --------------------------------------------------------------------------------------------
+# the parameter-free relative bias of [GenRank §6.2.3], Eq. (6.2.6), in place of the learned
+# tables: bias_{i,j} = -m_p (p_i - p_j) - m_t bucket(t_i - t_j)  (ALiBi extended to time)
+# --------------------------------------------------------------------------------------------
+
+def alibi_bias_matrix(rows, L, ts, m_p, m_t, num_buckets, mask, num_candidates):
+    """Eq. (6.2.6) for the given query rows and all keys of one sequence (fp64), with the same
+    positions (candidates at n) and the same time-bucket rule as the learned-table bias."""
+    p = positions(L, mask, num_candidates)
+    out = -float(m_p) * (p[rows][:, None] - p[None, :]).astype(np.float64)
+    if ts is not None:
+        ts = np.asarray(ts, dtype=np.int64)
+        out -= float(m_t) * time_bucket(ts[rows][:, None] - ts[None, :], num_buckets)
+    return out
+
+
+def attention_forward_alibi(q, k, v, seq_offsets, timestamps, m_p, m_t, *, num_heads, d_qk,
+                            d_v, num_time_buckets, alpha=1.0, mask=MASK_CAUSAL,
+                            num_candidates=0):
+    """The pointwise attention with Eq. (6.2.6)'s bias inside the SiLU:
+    out_i = Σ_{j allowed} SiLU(alpha <q_i, k_j> + bias_{i,j}) v_j, per head (fp64)."""
+    H = num_heads
+    T = int(seq_offsets[-1])
+    Q, K, V = _heads(q, H, d_qk), _heads(k, H, d_qk), _heads(v, H, d_v)
+    out = np.zeros((T, H, d_v), dtype=np.float64)
+    for b in range(len(seq_offsets) - 1):
+        s, e = int(seq_offsets[b]), int(seq_offsets[b + 1])
+        L = e - s
+        if L == 0:
+            continue
+        rows = np.arange(L)
+        ts = None if timestamps is None else np.asarray(timestamps[s:e], dtype=np.int64)
+        ok = allowed_pairs(L, mask, num_candidates)
+        bias = alibi_bias_matrix(rows, L, ts, m_p, m_t, num_time_buckets, mask, num_candidates)
+        for h in range(H):
+            scores = alpha * (Q[s:e, h, :] @ K[s:e, h, :].T) + bias
+            out[s:e, h, :] = np.where(ok, silu(scores), 0.0) @ V[s:e, h, :]
+    return out.reshape(T, H * d_v)
