@@ -30,7 +30,12 @@ EXPORTED = [
     "hstu_debug_time_buckets", "hstu_workspace_init", "hstu_sync_status",
     "hstu_status_string", "hstu_version", "hstu_last_error_string",
     "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout", "hstu_alibi_tables",
+    "hstu_debug_bias_index",
 ]
+
+# Rules of hstu_debug_bias_index (hstu_bias_rule_t)
+BIAS_RULES = {"bucket64": 0, "bucket_row": 1, "time_elem": 2, "bucket_cls": 3, "threshold": 4,
+              "pos_table": 5, "pos_general": 6, "pos_segment": 7, "pos_direct": 8}
 
 
 class HstuError(RuntimeError):
@@ -90,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_layer_forward_stage": (i32, [ldp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_jagged_padded_copy": (i32, [vp, i32, i32, vp, i64, vp, i64, i64, i32, vp]),
         "hstu_debug_time_buckets": (i32, [vp, i32, vp, i32, vp]),
+        "hstu_debug_bias_index": (i32, [i32, vp, i32, i32, vp, vp]),
         "hstu_workspace_init": (i32, [vp, sz, vp]),
         "hstu_sync_status": (i32, [vp, vp]),
         "hstu_status_string": (ctypes.c_char_p, [i32]),
@@ -332,6 +338,17 @@ def debug_time_buckets(dt: torch.Tensor, nb: int, stream=None) -> torch.Tensor:
     out = torch.empty(dt.shape, dtype=torch.int32, device=dt.device)
     _check(lib().hstu_debug_time_buckets(_ptr(dt), dt.numel(), _ptr(out), nb, _stream_ptr(stream)),
            "hstu_debug_time_buckets")
+    return out
+
+
+def debug_bias_index(rule: str, inputs: torch.Tensor, param: int, stream=None) -> torch.Tensor:
+    """The attention kernels' bias-table index for each input (see hstu_debug_bias_index):
+    inputs is a device int64 tensor [n] for the time rules and [n, 3] for the others."""
+    code = BIAS_RULES[rule]
+    n = inputs.shape[0]
+    out = torch.empty(n, dtype=torch.int32, device=inputs.device)
+    _check(lib().hstu_debug_bias_index(code, _ptr(inputs.contiguous()), n, param, _ptr(out),
+                                       _stream_ptr(stream)), "hstu_debug_bias_index")
     return out
 
 

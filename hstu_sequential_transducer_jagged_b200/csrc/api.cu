@@ -40,6 +40,8 @@ cudaError_t launch_jagged_padded(const int32_t* offsets, int B, int max_len, con
                                  cudaStream_t stream);
 cudaError_t launch_time_buckets(const int64_t* dt, int n, int32_t* out, int nb,
                                 cudaStream_t stream);
+cudaError_t launch_bias_index(int rule, const int64_t* in, int n, int param, int32_t* out,
+                              cudaStream_t stream);
 cudaError_t launch_wait_timeout_probe(int32_t* status, cudaStream_t stream);
 cudaError_t launch_attn_fwd_simt(int dtype, int D, const AttnGeom& g, const void* q, int64_t ld_q,
                                  const void* k, int64_t ld_k, const void* v, int64_t ld_v,
@@ -51,6 +53,14 @@ cudaError_t launch_attn_bwd_simt(int dtype, int D, const AttnGeom& g, const void
                                  const void* k, int64_t ld_k, const void* v, int64_t ld_v,
                                  const void* d_o, int64_t ld_do, void* dq, void* dk, void* dv,
                                  float* d_pos, float* d_time, int grid, cudaStream_t stream);
+cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const CUtensorMap& tdo,
+                               const CUtensorMap& tts, const AttnGeom& g, __nv_bfloat16* dq,
+                               int64_t ld_dq, __nv_bfloat16* dk, int64_t ld_dk,
+                               __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc, float* d_pos,
+                               float* d_time, int grid, bool fast, cudaStream_t stream);
+size_t attn_bwd_tc_smem(int P, int NB);
+int attn_bwd_tc_ts_box();
 }  // namespace hstu
 
 using namespace hstu;
@@ -69,6 +79,8 @@ hstu_status_t cuda_fail(cudaError_t e) {
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;  // status word at 0, work-item count at 4
 constexpr int kMaxSeqLen = 1 << 24;
+// Largest position clamp P: 2P + 1 table entries and every index stay far inside int32.
+constexpr int kMaxPosDist = 1 << 24;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -159,7 +171,7 @@ hstu_status_t check_common(int B, int T, int max_len, const int32_t* offsets, in
   if (H < 1 || dqk < 1 || dv < 1) return HSTU_ERR_INVALID_ARG;
   if (mask != HSTU_MASK_CAUSAL && mask != HSTU_MASK_MFALCON) return HSTU_ERR_INVALID_ARG;
   if (mask == HSTU_MASK_MFALCON && (m < 0 || mb < 1)) return HSTU_ERR_INVALID_ARG;
-  if (rab_pos != nullptr && P < 0) return HSTU_ERR_INVALID_ARG;
+  if (rab_pos != nullptr && (P < 0 || P > kMaxPosDist)) return HSTU_ERR_INVALID_ARG;
   if (rab_time != nullptr && NB < 1) return HSTU_ERR_INVALID_ARG;
   if (!std::isfinite(alpha)) return HSTU_ERR_INVALID_ARG;
   if (dtype != HSTU_BF16 && dtype != HSTU_FP32) return HSTU_ERR_INVALID_ARG;
@@ -294,7 +306,12 @@ size_t hstu_attention_workspace_size(const hstu_attn_desc_t* d) {
 }
 
 size_t hstu_attention_backward_workspace_size(const hstu_attn_desc_t* d) {
-  return hstu_attention_workspace_size(d);
+  if (d == nullptr || d->total_tokens < 0 || d->num_seqs < 0 || d->max_seq_len < 0 ||
+      d->num_heads < 1 || d->d_qk < 1)
+    return 0;
+  // + the fp32 dQ accumulator [T, H * d_qk] of the tensor-core backward
+  return hstu_attention_workspace_size(d) +
+         align_up(sizeof(float) * static_cast<size_t>(d->total_tokens) * d->num_heads * d->d_qk);
 }
 
 hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* d, const void* q, const void* k,
@@ -344,7 +361,7 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
   if (d->rab_pos != nullptr && 2 * static_cast<int64_t>(d->max_pos_dist) + 1 + d->num_time_buckets > 50000)
     return HSTU_ERR_UNSUPPORTED;  // the per-CTA bias-gradient bins live in shared memory
   const WsLayout w = attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len);
-  st = check_ws(ws, ws_bytes, w.total_attn);
+  st = check_ws(ws, ws_bytes, hstu_attention_backward_workspace_size(d));
   if (st != HSTU_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d_rab_pos != nullptr && d->rab_pos != nullptr &&
@@ -364,8 +381,35 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
                                d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
                                d->num_candidates, d->alpha);
   const int grid = max_items(d->total_tokens, d->num_seqs) * d->num_heads;
-  cudaError_t e = launch_attn_bwd_simt(d->dtype, D, g, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o,
-                                       d->ld_o, dq, dk, dv, d_rab_pos, d_rab_time, grid, s);
+  // Head width 64 in bf16 with 16-byte aligned rows runs on the tensor cores (bias-gradient bins
+  // and table copies in shared memory); every other shape on CUDA cores.
+  const bool use_time = d->timestamps != nullptr && d->rab_time != nullptr;
+  const bool tc = D == 64 && attn_uses_tc(D, d->dtype, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o,
+                                          d->ld_o) &&
+                  aligned16(dq) && aligned16(dk) && aligned16(dv) && (!use_time || aligned16(d->timestamps)) &&
+                  attn_bwd_tc_smem(d->rab_pos ? d->max_pos_dist : 0,
+                                   d->rab_time ? d->num_time_buckets : 0) <= 227 * 1024;
+  cudaError_t e;
+  if (tc) {
+    CUtensorMap tq, tk, tv, tdo, tts;
+    std::memset(&tts, 0, sizeof(tts));
+    const int64_t T = d->total_tokens;
+    if (!make_map_bf16(&tq, q, T, cols, d->ld_q, 64, kTileRows) ||
+        !make_map_bf16(&tk, k, T, cols, d->ld_k, 64, kTileRows) ||
+        !make_map_bf16(&tv, v, T, cols, d->ld_v, 64, kTileRows) ||
+        !make_map_bf16(&tdo, d_o, T, cols, d->ld_o, 64, kTileRows) ||
+        (use_time && !make_map_i64_1d(&tts, d->timestamps, T, attn_bwd_tc_ts_box())))
+      return HSTU_ERR_CUDA;
+    float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.total_attn);
+    const int pgrid = grid < num_sms_current() ? grid : num_sms_current();
+    e = launch_attn_bwd_tc(tq, tk, tv, tdo, tts, g, static_cast<__nv_bfloat16*>(dq), d->ld_q,
+                           static_cast<__nv_bfloat16*>(dk), d->ld_k,
+                           static_cast<__nv_bfloat16*>(dv), d->ld_v, dq_acc, d_rab_pos,
+                           d_rab_time, pgrid, true, s);
+  } else {
+    e = launch_attn_bwd_simt(d->dtype, D, g, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o, d->ld_o,
+                             dq, dk, dv, d_rab_pos, d_rab_time, grid, s);
+  }
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
@@ -481,9 +525,23 @@ hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
+hstu_status_t hstu_debug_bias_index(int32_t rule, const int64_t* in, int32_t n, int32_t param,
+                                    int32_t* out, hstu_stream_t stream) {
+  if (rule < HSTU_BIAS_RULE_BUCKET64 || rule > HSTU_BIAS_RULE_POS_DIRECT || n < 0)
+    return HSTU_ERR_INVALID_ARG;
+  const bool time_rule = rule <= HSTU_BIAS_RULE_THRESHOLD;
+  if (time_rule ? (param < 1) : (param < 0 || param > kMaxPosDist)) return HSTU_ERR_INVALID_ARG;
+  if (n == 0) return HSTU_OK;
+  if (in == nullptr || out == nullptr) return HSTU_ERR_INVALID_ARG;
+  cudaError_t e =
+      launch_bias_index(rule, in, n, param, out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+}
+
 hstu_status_t hstu_alibi_tables(float m_p, float m_t, int32_t max_pos_dist,
                                 int32_t num_time_buckets, float* rab_pos, float* rab_time) {
-  if (!std::isfinite(m_p) || !std::isfinite(m_t) || max_pos_dist < 0 || num_time_buckets < 1)
+  if (!std::isfinite(m_p) || !std::isfinite(m_t) || max_pos_dist < 0 ||
+      max_pos_dist > kMaxPosDist || num_time_buckets < 1)
     return HSTU_ERR_INVALID_ARG;
   if (rab_pos != nullptr)
     for (int32_t k = 0; k <= 2 * max_pos_dist; ++k)
@@ -593,6 +651,14 @@ extern "C" hstu_status_t hstu_attention_forward_static_ws(const hstu_attn_desc_t
                                   d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
   if (st != HSTU_OK) return st;
   if (status_out != nullptr && (reinterpret_cast<uintptr_t>(status_out) % 4) != 0)
+    return HSTU_ERR_INVALID_ARG;
+  // the checks hstu_attention_forward makes before it touches the workspace, made here before
+  // the status word of the shared array is cleared
+  const int64_t cols = static_cast<int64_t>(d->num_heads) * d->d_qk;
+  if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
+    return HSTU_ERR_INVALID_ARG;
+  if (d->num_seqs > 0 && d->total_tokens > 0 &&
+      (q == nullptr || k == nullptr || v == nullptr || o == nullptr))
     return HSTU_ERR_INVALID_ARG;
   const size_t need = hstu_attention_workspace_size(d);
   if (need > HSTU_STATIC_SCRATCH_BYTES) {

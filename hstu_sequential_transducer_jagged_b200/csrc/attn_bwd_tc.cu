@@ -1,7 +1,6 @@
 // attn_bwd_tc.cu — jagged HSTU pointwise attention backward for head width 64 on the
-// 5th-generation tensor cores.  Compiled into the library but not yet reachable from the C ABI:
-// hstu_attention_backward keeps the SIMT kernels until this one has passed its parity run on
-// hardware.
+// 5th-generation tensor cores (hstu_attention_backward's path for bf16 with 16-byte aligned rows;
+// other shapes take the CUDA-core kernels).
 //
 // With S = alpha Q Kᵀ + rab on visible pairs, P = SiLU(S), O = P V and the output gradient dO
 // (chain rule through "万亿参数推荐大模型：HSTU 架构如何超越传统 Self-Attention" §2.1, second formula):
@@ -176,8 +175,7 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
   cpidx = 0;
   if (t.use_pos) {
     // keys are history tokens (position = index); queries past the history sit at n
-    const int dmin = (i0 < n ? i0 : n) - j1;
-    if (dmin < t.P) {
+    if (!pos_segment_beyond_clamp(i0 < n ? i0 : n, j1, t.P)) {
       cbias = tterm;
       return kChunkTimeConst;
     }
@@ -212,9 +210,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_
         bias = 0.f;
         if (t.use_pos) {
           const int pi = i < r.n ? i : r.n;
-          int d = pi - r.pj;
-          d = d < -t.P ? -t.P : (d > t.P ? t.P : d);
-          pidx = d + t.P;
+          pidx = pos_index_direct(pi, r.pj, t.P);
           bias += t.pos[pidx];
         }
         if (V == kChunkTimeConst) {
@@ -613,6 +609,8 @@ __global__ void f32_to_bf16_rows(const float* __restrict__ src, int64_t ld_src,
   *reinterpret_cast<uint4*>(dst + r * ld_dst + c) = o;
 }
 }  // namespace
+
+int attn_bwd_tc_ts_box() { return kTsBox; }
 
 size_t attn_bwd_tc_smem(int P, int NB) {
   return sizeof(BwdSmem) + 1024 + 2 * sizeof(float) * (2 * P + 1 + NB);

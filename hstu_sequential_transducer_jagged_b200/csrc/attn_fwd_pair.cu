@@ -47,7 +47,7 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kQ = kTileRows;           // query tile rows (128)
-constexpr int kKV = 96;                 // key/value tile rows
+constexpr int kKV = kPairKvRows;        // key/value tile rows (96)
 constexpr int kSeg = 48;                // columns of a score tile per epilogue warp
 constexpr int kStages = 5;
 constexpr int kThreads = 640;          // 5 warpgroups
@@ -55,7 +55,7 @@ constexpr int kQBytes = kQ * kD * 2;    // 16 KB, 128-byte swizzle
 constexpr int kKVBytes = kKV * kD * 2;  // 12 KB
 constexpr int kTsBox = 98;              // timestamps loaded per KV tile (x rounded down to even)
 constexpr int kTsStride = 112;          // 896-byte stages keep every TMA destination 128-aligned
-constexpr int kTimeSmem = 64;
+constexpr int kTimeSmem = kTimeTableEntries;
 
 __device__ __forceinline__ uint32_t col_buf(int a, int b) { return 96u * (2 * a + b); }
 __device__ __forceinline__ uint32_t col_o(int a) { return 384u + 64u * a; }
@@ -161,8 +161,6 @@ __device__ __forceinline__ PairPlan make_plan(int qt0, int L, int n) {
   return p;
 }
 
-__device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
-
 // Waits for outstanding tcgen05.ld and ties the destination registers to the wait, so the
 // compiler cannot read them before the data has landed.
 __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
@@ -178,20 +176,9 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
       : "memory");
 }
 
-// floor(log2(max(1, d))) clamped to nb-1 for |d| < 2^23 without FLO: 2^23 + d is exact in
-// fp32, so after subtracting 2^23 the exponent field is the bit length of d minus one.
-__device__ __forceinline__ int bucket_small(int d, int nbm1) {
-  d = d < 1 ? 1 : (d > 0x7FFFFF ? 0x7FFFFF : d);
-  const float f = __int_as_float(0x4B000000 | d) - 8388608.0f;
-  const int b = (__float_as_int(f) >> 23) - 127;
-  return b < nbm1 ? b : nbm1;
-}
-
 // 0.5 x rab_time[bucket(d)] for |d| < 2^23 (the table holds clamped entries up to index 63).
 __device__ __forceinline__ float time_term32(const float* time_h, int d) {
-  d = d < 1 ? 1 : (d > 0x7FFFFF ? 0x7FFFFF : d);
-  const float f = __int_as_float(0x4B000000 | d) - 8388608.0f;
-  return time_h[(__float_as_int(f) >> 23) - 127];
+  return time_h[log2_small(d)];
 }
 
 __device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_fast(h), h); }
@@ -237,7 +224,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[W], uint32_t (&pk
       for (int u = 0; u < 4; ++u) bb[u] = rc.half_bias;
     } else if (MODE == kModeElem || MODE == kModeCausal) {
       // exact for every row: beyond the band the clamped table repeats its last entry
-      const float4 pv = pos4[clampi(rc.pbase - c, 0, rc.P2 + 3)];
+      const float4 pv = pos4[pos4_row(rc.pbase, c, rc.P2)];
       bb[0] = rc.half_bias + pv.x;
       bb[1] = rc.half_bias + pv.y;
       bb[2] = rc.half_bias + pv.z;
@@ -246,7 +233,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[W], uint32_t (&pk
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int j = rc.c0t + c + u;  // candidate keys (j >= n) sit at position n
-        bb[u] = pos4[clampi(rc.pi_plus_p - (j < rc.n ? j : rc.n), 0, rc.P2)].x;
+        bb[u] = pos4[pos4_general_row(rc.pi_plus_p, j, rc.n, rc.P2)].x;
       }
     }
     if (TM == 1 || TM == 2) {
@@ -254,7 +241,8 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[W], uint32_t (&pk
       const int d[4] = {rc.ti_lo - tv.x, rc.ti_lo - tv.y, rc.ti_lo - tv.z, rc.ti_lo - tv.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        bb[u] += TM == 1 ? (d[u] >= rc.thr ? rc.t_hi : rc.t_lo) : time_term32(time_h, d[u]);
+        bb[u] += TM == 1 ? (threshold_takes_hi(d[u], rc.thr) ? rc.t_hi : rc.t_lo)
+                         : time_term32(time_h, d[u]);
     } else if (TM == 3) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) bb[u] += time_h[time_bucket64(rc.ti - ts[c + u], rc.nbm1 + 1)];
@@ -339,7 +327,7 @@ __device__ __forceinline__ int2 classify_quarter(const QuarterRows& q, int c0, i
   } else if (last > q.i0) {
     mode = kModeCausal;    // the causal diagonal (keys past the sequence are past it too)
   } else {
-    mode = (use_pos && q.pmin - last < P) ? kModeElem : kModeConst;
+    mode = (use_pos && !pos_segment_beyond_clamp(q.pmin, last, P)) ? kModeElem : kModeConst;
   }
   bool tconst = true;
   float hb = 0.f;
@@ -351,18 +339,12 @@ __device__ __forceinline__ int2 classify_quarter(const QuarterRows& q, int c0, i
     if (tconst) hb = time_h[b_lo];
     else if (mode == kModeConst) mode = kModeElem;
   }
-  if (mode == kModeConst) hb += pos4[P2 + 3].x;  // beyond the clamp: the table's last entry
+  if (mode == kModeConst) hb += pos4[P2 + 3].x;  // beyond the clamp: lane 0 reads entry 2P
   return make_int2(mode | (tconst ? 8 : 0), __float_as_int(hb));
 }
 
 // classify_quarter with the timestamps given relative to a common reference, all within
-// +-2^30 of it, so the time buckets come from 32-bit differences: floor(log2(max(1, d))) is
-// 31 minus the leading zero count of d, clamped to nb-1.
-__device__ __forceinline__ int bucket32(int d, int nbm1) {
-  const int b = d < 1 ? 0 : 31 - __clz(d);
-  return b < nbm1 ? b : nbm1;
-}
-
+// +-2^30 of it, so the time buckets come from 32-bit differences (bucket32).
 __device__ __forceinline__ int2 classify_quarter32(int i0, int i1, int pmin, int tlo, int thi,
                                                    int c0, int n, int P, bool use_pos,
                                                    bool use_time, int NB, int tmin, int tmax,
@@ -377,7 +359,7 @@ __device__ __forceinline__ int2 classify_quarter32(int i0, int i1, int pmin, int
   } else if (last > i0) {
     mode = kModeCausal;
   } else {
-    mode = (use_pos && pmin - last < P) ? kModeElem : kModeConst;
+    mode = (use_pos && !pos_segment_beyond_clamp(pmin, last, P)) ? kModeElem : kModeConst;
   }
   bool tconst = true;
   float hb = 0.f;
@@ -413,7 +395,7 @@ __device__ __forceinline__ RowCtx segment_ctx(RowCtx rc, int2 cls, int c0t, int 
       const bool w_multi = __any_sync(0xffffffffu, row_valid && b_hi > b_lo + 1);
       if (!w_multi) {
         tm = 1;
-        rc.thr = 1 << (b_lo + 1);
+        rc.thr = threshold_of(b_lo);
         rc.t_lo = time_h[b_lo];
         rc.t_hi = time_h[b_hi];
       } else {
@@ -532,14 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (without a position table pos4 holds 4 zero entries, so the per-element path adds 0)
   const int P2 = use_pos ? 2 * g.P : 0;
   for (int x = threadIdx.x; x <= P2 + 3; x += kThreads)
-    pos4[x] = use_pos ? make_float4(0.5f * g.rab_pos[clampi(x, 0, P2)],
-                                    0.5f * g.rab_pos[clampi(x - 1, 0, P2)],
-                                    0.5f * g.rab_pos[clampi(x - 2, 0, P2)],
-                                    0.5f * g.rab_pos[clampi(x - 3, 0, P2)])
+    pos4[x] = use_pos ? make_float4(0.5f * g.rab_pos[pos4_lane_src(x, 0, P2)],
+                                    0.5f * g.rab_pos[pos4_lane_src(x, 1, P2)],
+                                    0.5f * g.rab_pos[pos4_lane_src(x, 2, P2)],
+                                    0.5f * g.rab_pos[pos4_lane_src(x, 3, P2)])
                       : make_float4(0.f, 0.f, 0.f, 0.f);
   if (use_time)
     for (int e = threadIdx.x; e < kTimeSmem; e += kThreads)
-      sm.rab_time_h[e] = 0.5f * g.rab_time[e < g.NB ? e : g.NB - 1];
+      sm.rab_time_h[e] = 0.5f * g.rab_time[time_table_src(e, g.NB)];
   if (threadIdx.x == 0) {
     for (int sl = 0; sl < 2; ++sl) {
       mbar_init(&sm.q_full[sl], 1);

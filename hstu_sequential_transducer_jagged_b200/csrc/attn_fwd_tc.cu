@@ -63,7 +63,6 @@ struct FwdSmem {
   float rab_pos[1];  // variable length tail: 2P+1 entries when the table lives in smem
 };
 
-__device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
 
 // Epilogue for one 32-column chunk of S (this thread's row).  MODE 0: constant bias, no mask;
 // MODE 1: per-element bias, no mask; MODE 2: per-element bias and mask.
@@ -89,7 +88,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p
         float bias = 0.f;
         if (pos_tab != nullptr) {
           const int pj = j < n ? j : n;
-          bias += pos_tab[clampi(pi - pj, -P, P) + P];
+          bias += pos_tab[pos_index_direct(pi, pj, P)];
         }
         if (use_time) bias += time_tab[time_bucket64(ti - ts_tile[c - (c_base & ~127)], NB)];
         h = fmaf(half_alpha, acc, 0.5f * bias);

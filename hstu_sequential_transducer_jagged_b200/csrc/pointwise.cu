@@ -298,4 +298,61 @@ cudaError_t launch_time_buckets(const int64_t* dt, int n, int32_t* out, int nb,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ bias-index rules (debug)
+// One thread per query; each rule calls the bias_index.cuh function the attention kernels call
+// at that point, so the output is what the kernels compute.  Rules and inputs: see
+// hstu_debug_bias_index() in include/hstu.h.
+__global__ void bias_index_kernel(int rule, const int64_t* __restrict__ in, int n, int param,
+                                  int32_t* __restrict__ out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  int r = -1;
+  switch (rule) {
+    case 0: r = time_bucket64(in[i], param); break;
+    case 1: r = bucket_small(static_cast<int>(in[i]), param - 1); break;
+    case 2: r = time_table_src(log2_small(static_cast<int>(in[i])), param); break;
+    case 3: r = bucket32(static_cast<int>(in[i]), param - 1); break;
+    case 4: {  // (dt_lo, dt_hi, dt): the two-bucket choice, -1 if the row spans more buckets
+      const int b_lo = bucket_small(static_cast<int>(in[3 * i]), param - 1);
+      const int b_hi = bucket_small(static_cast<int>(in[3 * i + 1]), param - 1);
+      if (b_hi <= b_lo + 1)
+        r = threshold_takes_hi(static_cast<int>(in[3 * i + 2]), threshold_of(b_lo)) ? b_hi : b_lo;
+      break;
+    }
+    case 5: {  // (p_i, j, -): lane (j mod 4) of the shifted table's entry for key j
+      const int p_i = static_cast<int>(in[3 * i]), j = static_cast<int>(in[3 * i + 1]);
+      const int c0t = j - j % kPairKvRows;         // first key of j's tile
+      const int c = (j - c0t) & ~3;                // the 4-aligned column of the load
+      const int x = pos4_row(p_i + param - c0t, c, 2 * param);
+      r = pos4_lane_src(x, j - c0t - c, 2 * param);
+      break;
+    }
+    case 6: {  // (p_i, j, n): candidate segments, key position min(j, n), lane 0
+      const int x = pos4_general_row(static_cast<int>(in[3 * i]) + param,
+                                     static_cast<int>(in[3 * i + 1]),
+                                     static_cast<int>(in[3 * i + 2]), 2 * param);
+      r = pos4_lane_src(x, 0, 2 * param);
+      break;
+    }
+    case 7:  // (p_min, j_last, -): 2P when the segment's position term is constant, else -1
+      r = pos_segment_beyond_clamp(static_cast<int>(in[3 * i]), static_cast<int>(in[3 * i + 1]),
+                                   param)
+              ? pos4_lane_src(2 * param + 3, 0, 2 * param)
+              : -1;
+      break;
+    case 8:  // (p_i, p_j, -): the direct clamp
+      r = pos_index_direct(static_cast<int>(in[3 * i]), static_cast<int>(in[3 * i + 1]), param);
+      break;
+    default: break;
+  }
+  out[i] = r;
+}
+
+cudaError_t launch_bias_index(int rule, const int64_t* in, int n, int param, int32_t* out,
+                              cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  bias_index_kernel<<<(n + 255) / 256, 256, 0, stream>>>(rule, in, n, param, out);
+  return cudaGetLastError();
+}
+
 }  // namespace hstu

@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "bias_index.cuh"
+
 namespace hstu {
 
 // Status word codes written by kernels (mirror hstu_status_t).
@@ -263,13 +265,6 @@ __device__ __forceinline__ float tanh_fast(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// floor(log2(max(1, dt))) clamped to [0, nb-1], exactly, on the 64-bit difference.
-__device__ __forceinline__ int time_bucket64(long long dt, int nb) {
-  unsigned long long d = dt < 1 ? 1ull : static_cast<unsigned long long>(dt);
-  int b = 63 - __clzll(static_cast<long long>(d));
-  return b < nb - 1 ? b : nb - 1;
 }
 
 }  // namespace hstu

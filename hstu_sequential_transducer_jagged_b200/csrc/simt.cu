@@ -50,9 +50,7 @@ __device__ __forceinline__ PairBias pair_bias(const AttnGeom& g, int i, int j, i
   if (g.rab_pos != nullptr) {
     const int pi = i < n ? i : n;
     const int pj = j < n ? j : n;
-    int dp = pi - pj;
-    dp = dp < -g.P ? -g.P : (dp > g.P ? g.P : dp);
-    b.pidx = dp + g.P;
+    b.pidx = pos_index_direct(pi, pj, g.P);
     b.value += g.rab_pos[b.pidx];
   }
   if (g.ts != nullptr && g.rab_time != nullptr) {

@@ -117,6 +117,8 @@ hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* desc, const void* q
  *     HSTU_ERR_WORKSPACE before any launch, and hstu_last_error_string() gives both sizes.
  *   - Set-up: the first call on each device looks the array's device address up (with that
  *     device current) and caches it; make that first call before any stream capture begins.
+ *     The cached address is never refreshed: after cudaDeviceReset() on a device it is stale,
+ *     so do not use this call on that device again in the same process.
  *   - Sharing: every call on a device uses the same array, which keeps the last call's contents;
  *     each call zeroes the status word on its stream first (the work list is rebuilt in full).
  *     Calls that overlap in time on one device (different streams or host threads without
@@ -208,7 +210,11 @@ hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_se
  * tables to the attention or layer calls with max_pos_dist = P.  The position term is exact only
  * where |p_i - p_j| <= P, so take P >= the longest sequence length - 1.  Host arrays owned by the
  * caller, [2P+1] and [NB] floats; either may be NULL to skip it.  Returns HSTU_ERR_INVALID_ARG
- * for a non-finite slope, P < 0 or NB < 1; no device work. */
+ * for a non-finite slope, P < 0, P > 2^24 or NB < 1; no device work.
+ * Speed note: the paired head-width-64 forward keeps a 4-wide copy of the position table in
+ * shared memory, which fits for P up to about 1100; a larger P (these tables with sequences
+ * longer than that) runs the single-tile tensor-core forward, which reads the table from global
+ * memory and is slower but computes the same result. */
 hstu_status_t hstu_alibi_tables(float m_p, float m_t, int32_t max_pos_dist,
                                 int32_t num_time_buckets, float* rab_pos, float* rab_time);
 
@@ -226,6 +232,53 @@ hstu_status_t hstu_debug_wait_timeout(void* ws, size_t ws_bytes, hstu_stream_t s
  * compared bit-exactly with an integer reference.  dt, out: device [n]. */
 hstu_status_t hstu_debug_time_buckets(const int64_t* dt, int32_t n, int32_t* out, int32_t nb,
                                       hstu_stream_t stream);
+
+/* Debug export of every integer rule the attention kernels use to turn a (query, key) pair into
+ * bias-table indices ("HSTU：Scaling Law 的首次探索" §7.1.4 innovation 2: a bias from the position
+ * and time differences).  The kernels fold these indices into their epilogues in several forms;
+ * this call evaluates each form with the very device functions the kernels call, so that a test
+ * can compare them bit for bit with an integer reference:
+ *   rule HSTU_BIAS_RULE_BUCKET64    in[i] = dt (any int64), param = NB: the 64-bit bucket
+ *                                   clamp(floor(log2(max(1, dt))), 0, NB-1) (M-FALCON segments,
+ *                                   the backward, the single-tile forward).
+ *   rule HSTU_BIAS_RULE_BUCKET_ROW  in[i] = dt with |dt| < 2^23, param = NB: the per-row bucket
+ *                                   bounds of the paired forward (fp32-exponent method).
+ *   rule HSTU_BIAS_RULE_TIME_ELEM   in[i] = dt with |dt| < 2^23, param = NB: the time-table entry
+ *                                   the paired forward's per-element path reads (its 64-entry
+ *                                   table repeats bucket NB-1 past the end).
+ *   rule HSTU_BIAS_RULE_BUCKET_CLS  in[i] = dt with |dt| < 2^31, param = NB: the paired forward's
+ *                                   tile classifier (count of leading zeros on 32 bits).
+ *   rule HSTU_BIAS_RULE_THRESHOLD   in[3i..3i+2] = (dt_lo, dt_hi, dt), dt_lo <= dt <= dt_hi, all
+ *                                   within +-2^23, param = NB: the bucket the two-bucket path
+ *                                   picks for dt in a row whose keys span [dt_lo, dt_hi]; -1 when
+ *                                   the row spans more than two buckets (the kernel then takes
+ *                                   the per-element path).
+ *   rule HSTU_BIAS_RULE_POS_TABLE   in[3i..] = (p_i, j, unused), param = P: the rab_pos index the
+ *                                   paired forward reads for query position p_i and key j through
+ *                                   its 4-wide shifted table (tile of 96 keys, lane j mod 4).
+ *   rule HSTU_BIAS_RULE_POS_GENERAL in[3i..] = (p_i, j, n), param = P: the index of the M-FALCON
+ *                                   candidate segments (key position min(j, n)).
+ *   rule HSTU_BIAS_RULE_POS_SEGMENT in[3i..] = (p_min, j_last, unused), param = P: 2P when the
+ *                                   classifier gives a row segment (smallest query position
+ *                                   p_min, last key j_last) one constant position term, else -1.
+ *   rule HSTU_BIAS_RULE_POS_DIRECT  in[3i..] = (p_i, p_j, unused), param = P: clamp(p_i - p_j,
+ *                                   -P, P) + P as the backward and CUDA-core kernels form it.
+ * in: device int64 [n] (rules 0-3) or [3n] (rules 4-8); out: device int32 [n].  Returns
+ * HSTU_ERR_INVALID_ARG for an unknown rule, n < 0, NB < 1 or P outside [0, 2^24]. */
+typedef enum {
+  HSTU_BIAS_RULE_BUCKET64 = 0,
+  HSTU_BIAS_RULE_BUCKET_ROW = 1,
+  HSTU_BIAS_RULE_TIME_ELEM = 2,
+  HSTU_BIAS_RULE_BUCKET_CLS = 3,
+  HSTU_BIAS_RULE_THRESHOLD = 4,
+  HSTU_BIAS_RULE_POS_TABLE = 5,
+  HSTU_BIAS_RULE_POS_GENERAL = 6,
+  HSTU_BIAS_RULE_POS_SEGMENT = 7,
+  HSTU_BIAS_RULE_POS_DIRECT = 8
+} hstu_bias_rule_t;
+
+hstu_status_t hstu_debug_bias_index(int32_t rule, const int64_t* in, int32_t n, int32_t param,
+                                    int32_t* out, hstu_stream_t stream);
 
 /* Zero the status word at the start of ws (asynchronously, on the stream).  Call once on a new
  * workspace before its first use: the status word must start at zero. */

@@ -123,6 +123,13 @@ def test_layer_rejects_bad_arguments(lib):
                                   ctypes.c_void_p(2 << 20), ok_ws, 1 << 40, None) == 2
 
 
+def test_position_clamp_is_bounded(lib):
+    # 2P + 1 table entries must stay inside int32 arithmetic
+    d = _desc(rab_pos=1 << 20, max_pos_dist=(1 << 24) + 1)
+    st = lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == 1
+
+
 def test_backward_requires_grad_buffers(lib):
     d = _desc(rab_pos=1 << 20, max_pos_dist=4)
     st = lib.hstu_attention_backward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
@@ -134,6 +141,15 @@ def test_misc_entry_points_validate(lib):
     assert lib.hstu_debug_time_buckets(FAKE, -1, FAKE, 8, None) == 1
     assert lib.hstu_debug_time_buckets(FAKE, 4, FAKE, 0, None) == 1
     assert lib.hstu_debug_time_buckets(None, 0, None, 8, None) == 0
+    # bias-index export: unknown rule, n < 0, NB < 1 (time rules), P out of range (position rules)
+    assert lib.hstu_debug_bias_index(9, FAKE, 4, 8, FAKE, None) == 1
+    assert lib.hstu_debug_bias_index(-1, FAKE, 4, 8, FAKE, None) == 1
+    assert lib.hstu_debug_bias_index(0, FAKE, -1, 8, FAKE, None) == 1
+    assert lib.hstu_debug_bias_index(2, FAKE, 4, 0, FAKE, None) == 1
+    assert lib.hstu_debug_bias_index(5, FAKE, 4, -1, FAKE, None) == 1
+    assert lib.hstu_debug_bias_index(5, FAKE, 4, (1 << 24) + 1, FAKE, None) == 1
+    assert lib.hstu_debug_bias_index(5, None, 4, 8, None, None) == 1
+    assert lib.hstu_debug_bias_index(5, None, 0, 8, None, None) == 0
     # row_bytes not a multiple of 16
     assert lib.hstu_jagged_padded_copy(FAKE, 2, 8, FAKE, 32, FAKE, 32, 24, 1, None) == 1
     assert lib.hstu_jagged_padded_copy(FAKE, 0, 8, FAKE, 32, FAKE, 32, 32, 1, None) == 0

@@ -33,6 +33,9 @@ def test_library_tables_reject_bad_arguments(lib):
     assert lib.hstu_alibi_tables(0.1, float("inf"), 3, 4, buf, buf) == 1
     assert lib.hstu_alibi_tables(0.1, 0.1, -1, 4, buf, buf) == 1
     assert lib.hstu_alibi_tables(0.1, 0.1, 3, 0, buf, buf) == 1
+    # 2P would overflow int32 past 2^30: P is bounded by 2^24 (nothing is written)
+    assert lib.hstu_alibi_tables(0.1, 0.1, 2 ** 31 - 1, 4, None, None) == 1
+    assert lib.hstu_alibi_tables(0.1, 0.1, (1 << 24) + 1, 4, None, None) == 1
     assert lib.hstu_alibi_tables(0.1, 0.1, 3, 4, None, None) == 0
 
 

@@ -99,6 +99,77 @@ def test_time_buckets_bit_exact(B):
         assert np.array_equal(got, O.time_bucket(dt, nb)), nb
 
 
+def _edges(kmax, lo=-3):
+    """Differences around every power of two up to 2^kmax, plus zero and negatives."""
+    v = {0, 1, -1, -2, lo}
+    for k in range(1, kmax + 1):
+        v |= {2 ** k - 1, 2 ** k, 2 ** k + 1, -(2 ** k)}
+    return v
+
+
+@pytest.mark.parametrize("nb", [1, 16, 64, 128])
+def test_bias_time_rules_bit_exact(B, nb):
+    """Each time-bucket form the attention kernels evaluate (64-bit, per-row fp32-exponent,
+    per-element table entry, classifier, two-bucket threshold) equals the integer rule of
+    [FunRec 7.1] §7.1.4 innovation 2 with log2 buckets, on every power-of-two edge of its range
+    (the 2^23 and 2^30 switch points included) and on random differences."""
+    rng = np.random.default_rng(nb)
+    small = sorted(x for x in _edges(22) | {2 ** 23 - 1, -(2 ** 23 - 1)} if abs(x) < 2 ** 23)
+    small = np.array(small + list(rng.integers(-2 ** 23 + 1, 2 ** 23, size=4000)), np.int64)
+    cls = sorted(x for x in _edges(30) | {2 ** 31 - 1, -(2 ** 31 - 1), 2 ** 23 - 1, 2 ** 23,
+                                           2 ** 23 + 1} if abs(x) < 2 ** 31)
+    cls = np.array(cls + list(rng.integers(-2 ** 31 + 1, 2 ** 31, size=4000)), np.int64)
+    wide = sorted(_edges(62) | {2 ** 63 - 1, -(2 ** 63) + 1})
+    wide = np.array(wide + list(rng.integers(-2 ** 62, 2 ** 62, size=4000)), np.int64)
+    for rule, vals in (("bucket64", wide), ("bucket_row", small), ("time_elem", small),
+                       ("bucket_cls", cls)):
+        got = B.debug_bias_index(rule, dev(vals), nb).cpu().numpy()
+        assert np.array_equal(got, O.time_bucket(vals, nb)), (rule, nb)
+    # threshold rows: [dt_lo, dt_hi] spans, one dt inside; bounds near powers of two
+    lo = rng.integers(-2 ** 23 + 1, 2 ** 23, size=6000)
+    span = np.where(rng.random(6000) < 0.5, rng.integers(0, 4, size=6000),
+                    rng.integers(0, 2 ** 22, size=6000))
+    edge = np.array(sorted(x for x in _edges(22) if abs(x) < 2 ** 23))
+    lo[:len(edge)] = edge
+    hi = np.minimum(lo + span, 2 ** 23 - 1)
+    dt = lo + (rng.random(6000) * (hi - lo + 1)).astype(np.int64)
+    dt = np.minimum(dt, hi)
+    trip = np.stack([lo, hi, dt], axis=1).astype(np.int64)
+    got = B.debug_bias_index("threshold", dev(trip), nb).cpu().numpy()
+    b_lo, b_hi = O.time_bucket(lo, nb), O.time_bucket(hi, nb)
+    want = np.where(b_hi <= b_lo + 1, O.time_bucket(dt, nb), -1)
+    assert np.array_equal(got, want), nb
+    assert (got >= 0).sum() > 1000  # the threshold path itself was exercised
+
+
+@pytest.mark.parametrize("P", [0, 1, 5, 96, 1024, 3000])
+def test_bias_position_rules_bit_exact(B, P):
+    """Each position-index form (the 4-wide shifted table of the paired forward with its lane
+    offset, the M-FALCON candidate form, the constant-segment decision, the direct clamp)
+    equals clamp(p_i - p_j, -P, P) + P on distances -P-1 .. P+1 and at every tile offset."""
+    rng = np.random.default_rng(P)
+    p_i = rng.integers(0, 12000, size=8000)
+    dist = np.concatenate([np.array([-P - 2, -P - 1, -P, -P + 1, -1, 0, 1, P - 1, P, P + 1,
+                                     P + 2, P + 3, P + 4]),
+                           rng.integers(-P - 300, P + 300, size=8000 - 13)])
+    p_i[:13] = 5000
+    j = np.clip(p_i - dist, 0, None)
+    # every residue of j modulo the 96-key tile and the 4-wide lanes, near the clamp
+    j[13:13 + 192] = 6000 + np.arange(192)
+    p_i[13:13 + 192] = 6000 + 96 + P - 1
+    n = rng.integers(0, 12000, size=8000)
+    trip = np.stack([p_i, j, n], axis=1).astype(np.int64)
+    got = B.debug_bias_index("pos_table", dev(trip), P).cpu().numpy()
+    assert np.array_equal(got, O.position_index(p_i - j, P)), "pos_table"
+    got = B.debug_bias_index("pos_general", dev(trip), P).cpu().numpy()
+    assert np.array_equal(got, O.position_index(p_i - np.minimum(j, n), P)), "pos_general"
+    got = B.debug_bias_index("pos_direct", dev(trip), P).cpu().numpy()
+    assert np.array_equal(got, O.position_index(p_i - j, P)), "pos_direct"
+    got = B.debug_bias_index("pos_segment", dev(trip), P).cpu().numpy()
+    idx = O.position_index(p_i - j, P)
+    assert np.array_equal(got, np.where(idx == 2 * P, 2 * P, -1)), "pos_segment"
+
+
 # --------------------------------------------------------------------- attention forward
 CAUSAL_LENGTHS = [1, 127, 128, 129, 0, 300, 513, 64]
 
