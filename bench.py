@@ -141,28 +141,47 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_layer_sample(wl, seconds_min=12.0, max_reps=12):
-    """The fp64 oracle on a bounded sample of the workload: one layer over its shortest
-    sequence, repeated until seconds_min of CPU work.  Returns (tokens/s, sample, threads)."""
-    from oracle import hstu_oracle as O
-    b = int(np.argmin(wl.lengths))
+def _oracle_layer_once(wl, b, O):
     s, e = int(wl.seq_offsets[b]), int(wl.seq_offsets[b + 1])
-    off = np.array([0, e - s])
     lp = wl.layers[0]
     kw = dict(num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, max_pos_dist=wl.max_pos_dist,
               num_time_buckets=wl.num_time_buckets, alpha=wl.alpha, mask=wl.mask,
               num_candidates=wl.num_candidates)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        O.layer_forward(wl.x[s:e], lp.w1, lp.w2, off, wl.timestamps[s:e], lp.rab_pos,
-                        lp.rab_time, **kw)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds_min or reps >= max_reps:
-            break
-    sample = (f"one fp64 oracle layer over sequence {b} ({e - s} tokens, the shortest) of "
-              f"{wl.name} seed 0, {reps} rep(s), {el:.1f} s")
-    return (e - s) * reps / el, sample, len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    O.layer_forward(wl.x[s:e], lp.w1, lp.w2, np.array([0, e - s]), wl.timestamps[s:e],
+                    lp.rab_pos, lp.rab_time, **kw)
+    return time.perf_counter() - t0
+
+
+def oracle_cost_model(wl):
+    """The fp64 oracle's cost of one layer over the whole workload, scaled from a sample.
+
+    The oracle's layer costs a L + b L^2 seconds for a sequence of L tokens (the two linear
+    layers and the LayerNorm grow with L, the attention with its L(L+1)/2 pairs).  It is timed on
+    the workload's shortest and its median-length sequence, a and b are fitted through the two
+    points, and the fit is summed over every sequence.  Returns (seconds per layer over the
+    whole workload, fit, sample description, threads)."""
+    from oracle import hstu_oracle as O
+    order = np.argsort(wl.lengths)
+    b_short, b_mid = int(order[0]), int(order[len(order) // 2])
+    t_short = _oracle_layer_once(wl, b_short, O)
+    t_mid = _oracle_layer_once(wl, b_mid, O)
+    l1, l2 = float(wl.lengths[b_short]), float(wl.lengths[b_mid])
+    if l2 > l1:
+        # t = a L + b L^2 through (l1, t_short) and (l2, t_mid)
+        bq = (t_mid / l2 - t_short / l1) / (l2 - l1)
+        a = t_short / l1 - bq * l1
+        if a < 0 or bq < 0:  # noisy timings: fall back to pure pair scaling
+            a, bq = 0.0, t_mid / (l2 * l2)
+    else:
+        a, bq = 0.0, t_short / (l1 * l1)
+    Ls = wl.lengths.astype(np.float64)
+    full = float(np.sum(a * Ls + bq * Ls * Ls))
+    sample = (f"fp64 oracle, one layer over sequences {b_short} ({int(l1)} tokens) and {b_mid} "
+              f"({int(l2)} tokens) of {wl.name} seed 0 ({t_short + t_mid:.1f} s of CPU work); "
+              f"t(L) = a L + b L^2 fitted through them and summed over all {wl.num_seqs} "
+              f"sequences ({wl.total_tokens} tokens): {full:.0f} s per layer")
+    return full, (a, bq), sample, len(os.sched_getaffinity(0))
 
 
 def reduce_over_ranks(values_max, values_sum, device):
@@ -182,35 +201,32 @@ def reduce_over_ranks(values_max, values_sum, device):
 
 
 def run_reference(args, rank):
+    """The reference arm: the fp64 CPU oracle (the pages give no implementation to run).  The
+    warm-up fits the oracle's cost model (oracle_cost_model); each timed step runs one oracle layer
+    over the workload's shortest sequence and is scaled to the whole workload by that model."""
     if rank != 0:
         return
     wl = W.make(WORKLOAD, seed=args.seed)
     from oracle import hstu_oracle as O
+    full, (a, bq), fit_sample, cores = oracle_cost_model(wl)
     b = int(np.argmin(wl.lengths))
-    s, e = int(wl.seq_offsets[b]), int(wl.seq_offsets[b + 1])
-    off = np.array([0, e - s])
-    lp = wl.layers[0]
-    kw = dict(num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, max_pos_dist=wl.max_pos_dist,
-              num_time_buckets=wl.num_time_buckets, alpha=wl.alpha, mask=wl.mask,
-              num_candidates=wl.num_candidates)
-
-    def step():
-        O.layer_forward(wl.x[s:e], lp.w1, lp.w2, off, wl.timestamps[s:e], lp.rab_pos,
-                        lp.rab_time, **kw)
-
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
+    Lb = float(wl.lengths[b])
+    scale = full / (a * Lb + bq * Lb * Lb)
+    for _ in range(max(args.warmup - 2, 0)):
+        _oracle_layer_once(wl, b, O)
+    el = 0.0
     for _ in range(args.steps):
-        step()
-    el = time.perf_counter() - t0
-    value = (e - s) * args.steps / el
-    cores = len(os.sched_getaffinity(0))
-    sample = f"one fp64 oracle layer over sequence {b} ({e - s} tokens, the shortest) per step"
+        el += _oracle_layer_once(wl, b, O)
+    # one step = one layer over the whole workload, predicted from the timed sample
+    step_s = el / args.steps * scale
+    value = wl.total_tokens / step_s
+    sample = (f"each step: one fp64 oracle layer over sequence {b} ({int(Lb)} tokens, the "
+              f"shortest), scaled x{scale:.1f} to all {wl.num_seqs} sequences by the cost model "
+              f"of the warm-up ({fit_sample})")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * step_s, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "description": wl.description, "seed": args.seed},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -264,13 +280,13 @@ def run_attention_only(args, lib, Bd, desc, ly, x, y, ws, stream, wl):
                       "attn_tflops": fl / (ms / 1e3) / 1e12}), flush=True)
 
 
-def run_attention_bwd(args, lib, Bd, dev):
-    """Time the attention forward and backward alone on the attention forward+backward workload
-    (B=64, L~U{512..2048}, H=8, d=64) through the C ABI with preallocated buffers.  FLOPs are
-    the unmasked pairs' algorithmic work: 4 d per pair forward, 8 d per pair backward (the
-    backward's recomputation of S is not counted)."""
+def time_attention_fwd_bwd(lib, Bd, dev, steps, warmup, seed=0):
+    """The attention forward and backward alone on the attention forward+backward workload
+    (B=64, L~U{512..2048}, H=8, d=64) through the C ABI with preallocated buffers, L2 flushed
+    between timed calls.  FLOPs are the unmasked pairs' algorithmic work: 4 d per pair forward,
+    8 d per pair backward (the backward's recomputation of S is reported apart)."""
     import torch
-    wl = W.make("attn_fwdbwd_bf16_b64", seed=args.seed)
+    wl = W.make("attn_fwdbwd_bf16_b64", seed=seed)
     bf = torch.bfloat16
     q, k, v, d_o = (torch.from_numpy(a).to(bf).to(dev) for a in (wl.q, wl.k, wl.v, wl.d_o))
     off = torch.from_numpy(wl.seq_offsets).to(dev)
@@ -288,7 +304,8 @@ def run_attention_bwd(args, lib, Bd, dev):
     ws = Bd.Workspace(lib.hstu_attention_backward_workspace_size(ctypes.byref(desc)), dev)
     stream = torch.cuda.current_stream()
     sp = ctypes.c_void_p(stream.cuda_stream)
-    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def fwd():
         st = lib.hstu_attention_forward(ctypes.byref(desc), P(q), P(k), P(v), P(o), ws.ptr,
@@ -304,29 +321,122 @@ def run_attention_bwd(args, lib, Bd, dev):
 
     res = {}
     for name, fn in (("fwd", fwd), ("bwd", bwd)):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             fn()
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.steps):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
             fn()
-        b.record(stream)
+            b.record(stream)
         torch.cuda.synchronize()
-        res[name] = a.elapsed_time(b) / args.steps
+        res[name] = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     if ws.sync_status() != 0:
         raise RuntimeError("device status word set")
     pairs = attention_pairs(wl) * wl.num_heads
-    print(json.dumps({"mode": "attn_bwd", "workload": wl.name, "tokens": wl.total_tokens,
-                      "fwd_ms": res["fwd"],
-                      "fwd_tflops": 4.0 * wl.d_qk * pairs / (res["fwd"] / 1e3) / 1e12,
-                      "bwd_ms": res["bwd"],
-                      "bwd_tflops": 8.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12,
-                      # the recomputation of S = QK^T (2 d per pair), reported apart
-                      "bwd_recompute_gflop": 2.0 * wl.d_qk * pairs / 1e9,
-                      "bwd_tflops_incl_recompute":
-                          10.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12}),
-          flush=True)
+    return {"workload": wl.name, "tokens": wl.total_tokens, "steps": steps,
+            "fwd_ms": res["fwd"], "fwd_tflops": 4.0 * wl.d_qk * pairs / (res["fwd"] / 1e3) / 1e12,
+            "bwd_ms": res["bwd"], "bwd_tflops": 8.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12,
+            "bwd_recompute_gflop": 2.0 * wl.d_qk * pairs / 1e9,
+            "bwd_tflops_incl_recompute": 10.0 * wl.d_qk * pairs / (res["bwd"] / 1e3) / 1e12,
+            "tokens_per_s_fwd_bwd": wl.total_tokens / ((res["fwd"] + res["bwd"]) / 1e3),
+            "l2": "256 MB buffer written before each timed call (outside its events)"}
+
+
+def run_attention_bwd(args, lib, Bd, dev):
+    r = time_attention_fwd_bwd(lib, Bd, dev, args.steps, args.warmup, args.seed)
+    r["mode"] = "attn_bwd"
+    print(json.dumps(r), flush=True)
+
+
+def time_layer_stack(lib, Bd, dev, name, steps, warmup, seed=0):
+    """A layer-stack workload through hstu_layer_forward_stage, with CUDA events around every
+    attention stage; L2 flushed between steps.  Returns tokens/s and the attention's TFLOP/s."""
+    import torch
+    wl = W.make(name, seed=seed)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    x = torch.from_numpy(wl.x).to(dt).to(dev)
+    off = torch.from_numpy(wl.seq_offsets).to(dev)
+    ts = torch.from_numpy(wl.timestamps).to(dev)
+    layers = [dict(w1=torch.from_numpy(lp.w1).to(dt).to(dev), w2=torch.from_numpy(lp.w2).to(dt).to(dev),
+                   rp=torch.from_numpy(lp.rab_pos).to(dev), rt=torch.from_numpy(lp.rab_time).to(dev))
+              for lp in wl.layers]
+    descs = [Bd.layer_desc(seq_offsets=off, total_tokens=wl.total_tokens,
+                           max_seq_len=wl.max_seq_len, timestamps=ts, d_model=wl.d_model,
+                           num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, mask=wl.mask,
+                           num_candidates=wl.num_candidates, microbatch=wl.microbatch or 1,
+                           rab_pos=ly["rp"], max_pos_dist=wl.max_pos_dist, rab_time=ly["rt"],
+                           num_time_buckets=wl.num_time_buckets, alpha=wl.alpha,
+                           ln_eps=wl.ln_eps, dtype=Bd._dtype_code(x)) for ly in layers]
+    ws = Bd.Workspace(lib.hstu_layer_workspace_size(ctypes.byref(descs[0])), dev)
+    bufs = [torch.empty_like(x), torch.empty_like(x)]
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    L = len(layers)
+
+    def run(attn_ev=None):
+        cur = x
+        for l in range(L):
+            out = bufs[l % 2]
+            for stage in (1, 2, 3):
+                if attn_ev is not None and stage == 2:
+                    attn_ev[l][0].record(stream)
+                st = lib.hstu_layer_forward_stage(
+                    ctypes.byref(descs[l]), stage, ctypes.c_void_p(cur.data_ptr()),
+                    ctypes.c_void_p(layers[l]["w1"].data_ptr()), None,
+                    ctypes.c_void_p(layers[l]["w2"].data_ptr()), None,
+                    ctypes.c_void_p(out.data_ptr()), ws.ptr, ws.nbytes, sp)
+                if st != 0:
+                    raise Bd.HstuError(st, f"{name} layer {l} stage {stage}")
+                if attn_ev is not None and stage == 2:
+                    attn_ev[l][1].record(stream)
+            cur = out
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+    attn_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(L)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        step_ev[k][0].record(stream)
+        run(attn_ev[k])
+        step_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    if ws.sync_status() != 0:
+        raise RuntimeError(f"{name}: device status word set")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in step_ev]))
+    attn_ms = float(np.mean([a.elapsed_time(b) for row in attn_ev for a, b in row]))
+    aflops = attention_flops(wl)
+    return {"workload": wl.name, "dtype": wl.dtype, "tokens": wl.total_tokens, "layers": L,
+            "steps": steps, "ms_per_step": ms,
+            "layer_tokens_per_s": wl.total_tokens * L / (ms / 1e3),
+            "attn_ms_per_layer": attn_ms, "attn_tflops": aflops / (attn_ms / 1e3) / 1e12,
+            "stack_tflops": L * (aflops + gemm_flops(wl)) / (ms / 1e3) / 1e12,
+            "l2": "256 MB buffer written between steps (outside the step events)"}
+
+
+def measure_other_configs(lib, Bd, dev, peaks):
+    """The other four workloads, each timed on its own (they are parity cases of the same
+    kernels; the headline line is the 4-layer stack)."""
+    pk = peaks["bf16_tflops"]
+    out = {}
+    for name, steps in (("layer_fp32_b4", 200), ("layer_bf16_b32_geo", 200),
+                        ("mfalcon_bf16_b16", 30)):
+        r = time_layer_stack(lib, Bd, dev, name, steps, 5)
+        if r["dtype"] == "bf16":
+            r["attn_frac_of_bf16_peak"] = r["attn_tflops"] / pk
+        out[name] = r
+    r = time_attention_fwd_bwd(lib, Bd, dev, 30, 3)
+    r["fwd_frac_of_bf16_peak"] = r["fwd_tflops"] / pk
+    r["bwd_frac_of_bf16_peak"] = r["bwd_tflops"] / pk
+    out[r["workload"]] = r
+    return out
 
 
 def run_e2e_pipelined(K, L, layers, wl, xh, offh, tsh, yh_serial, x, off, ts, stream, ws, world,
@@ -409,12 +519,14 @@ def run_e2e_pipelined(K, L, layers, wl, xh, offh, tsh, yh_serial, x, off, ts, st
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)  # about 1 s of device time
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other four workloads (timed after the headline line)")
     ap.add_argument("--mode", default="stack", choices=["stack", "attn", "attn_bwd"],
                     help="attn: time only the attention stage of layer 0 (profiling aid); "
                          "attn_bwd: attention forward and backward on the B=64 workload")
@@ -449,8 +561,9 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wl0 = W.make(WORKLOAD, seed=args.seed)
-        v, sample, cores = oracle_layer_sample(wl0)
-        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        full, _, sample, cores = oracle_cost_model(wl0)
+        cpu = {"value": wl0.total_tokens / full, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": sample}
         del wl0
 
     wl = W.make(WORKLOAD, seed=args.seed + rank)
@@ -625,12 +738,16 @@ def main():
                 e2e["api"] += ("; step i+1's host-to-device copy and step i-1's device-to-host "
                                "copy overlap step i's layers (two copy streams, double buffers)")
 
+    peaks = load_peaks()
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = measure_other_configs(lib, Bd, dev, peaks)
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
 
-    peaks = load_peaks()
     aflops = attention_flops(wl)
     attn_avg_ms = float(np.mean(attn_ms))
     attn_tflops = aflops / (attn_avg_ms / 1e3) / 1e12
@@ -666,6 +783,7 @@ def main():
         "l2_warm": l2_warm,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "configs": configs,
         "clocks": clocks,
         "gpu_launches": 5 * L * K,
         "wall_s_timed_region": wall,

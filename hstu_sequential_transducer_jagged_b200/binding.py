@@ -30,7 +30,7 @@ EXPORTED = [
     "hstu_debug_time_buckets", "hstu_workspace_init", "hstu_sync_status",
     "hstu_status_string", "hstu_version", "hstu_last_error_string",
     "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout", "hstu_alibi_tables",
-    "hstu_debug_bias_index",
+    "hstu_debug_bias_index", "hstu_layer_backward_workspace_size", "hstu_layer_backward",
 ]
 
 # Rules of hstu_debug_bias_index (hstu_bias_rule_t)
@@ -93,6 +93,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_layer_workspace_size": (sz, [ldp]),
         "hstu_layer_forward": (i32, [ldp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_layer_forward_stage": (i32, [ldp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "hstu_layer_backward_workspace_size": (sz, [ldp]),
+        "hstu_layer_backward": (i32, [ldp] + [vp] * 15 + [vp, sz, vp]),
         "hstu_jagged_padded_copy": (i32, [vp, i32, i32, vp, i64, vp, i64, i64, i32, vp]),
         "hstu_debug_time_buckets": (i32, [vp, i32, vp, i32, vp]),
         "hstu_debug_bias_index": (i32, [i32, vp, i32, i32, vp, vp]),
@@ -313,6 +315,41 @@ def layer_forward(x, w1, w2, seq_offsets, max_seq_len, timestamps=None, rab_pos=
     _check(lib().hstu_layer_forward(ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2),
                                     _ptr(b2), _ptr(out), ws.ptr, ws.nbytes, _stream_ptr(stream)),
            "hstu_layer_forward")
+    return out
+
+
+def layer_backward(x, w1, w2, d_y, seq_offsets, max_seq_len, timestamps=None, rab_pos=None,
+                   rab_time=None, *, num_heads, d_qk, d_v, max_pos_dist=0, num_time_buckets=1,
+                   alpha=1.0, mask=MASK_CAUSAL, num_candidates=0, microbatch=128, b1=None,
+                   b2=None, ln_eps=1e-5, ln_gamma=None, ln_beta=None,
+                   ws: Optional[Workspace] = None, stream=None):
+    """Gradients of Σ d_y ⊙ Y through one layer (hstu_layer_backward): a dict with dx (bf16,
+    like x) and the fp32 dw1, db1, dw2, db2, d_rab_pos, d_rab_time, d_ln_gamma, d_ln_beta
+    (None where the matching parameter is None)."""
+    T, d_model = x.shape
+    n1, hv = w1.shape[1], w2.shape[0]
+    f32 = dict(dtype=torch.float32, device=x.device)
+    out = dict(dx=torch.empty_like(x), dw1=torch.empty((d_model, n1), **f32),
+               dw2=torch.empty((hv, d_model), **f32),
+               db1=None if b1 is None else torch.empty(n1, **f32),
+               db2=None if b2 is None else torch.empty(d_model, **f32),
+               d_rab_pos=None if rab_pos is None else torch.empty_like(rab_pos),
+               d_rab_time=None if rab_time is None else torch.empty_like(rab_time),
+               d_ln_gamma=None if ln_gamma is None else torch.empty(hv, **f32),
+               d_ln_beta=None if ln_beta is None else torch.empty(hv, **f32))
+    desc = layer_desc(seq_offsets=seq_offsets, total_tokens=T, max_seq_len=max_seq_len,
+                      timestamps=timestamps, d_model=d_model, num_heads=num_heads, d_qk=d_qk,
+                      d_v=d_v, mask=mask, num_candidates=num_candidates, microbatch=microbatch,
+                      rab_pos=rab_pos, max_pos_dist=max_pos_dist, rab_time=rab_time,
+                      num_time_buckets=num_time_buckets, alpha=alpha, ln_eps=ln_eps,
+                      ln_gamma=ln_gamma, ln_beta=ln_beta, dtype=_dtype_code(x))
+    need = lib().hstu_layer_backward_workspace_size(ctypes.byref(desc))
+    ws = workspace(need, x.device) if ws is None else ws.ensure(need)
+    _check(lib().hstu_layer_backward(
+        ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(d_y),
+        _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["db1"]), _ptr(out["dw2"]), _ptr(out["db2"]),
+        _ptr(out["d_rab_pos"]), _ptr(out["d_rab_time"]), _ptr(out["d_ln_gamma"]),
+        _ptr(out["d_ln_beta"]), ws.ptr, ws.nbytes, _stream_ptr(stream)), "hstu_layer_backward")
     return out
 
 

@@ -16,10 +16,8 @@ namespace hstu {
 cudaError_t launch_attn_fwd_tc(int D, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const AttnGeom& g, __nv_bfloat16* out,
                                int64_t ld_o, int grid, cudaStream_t stream);
-cudaError_t launch_gemm_bf16_tc(int epi, const CUtensorMap& ta, const CUtensorMap& tb, int M,
-                                int N, int K, const float* bias, const __nv_bfloat16* resid,
-                                int64_t ld_r, __nv_bfloat16* C, int64_t ldc, int* status,
-                                cudaStream_t stream);
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);
+int gemm_tc_mn_tiles(int M, int N);
 cudaError_t launch_build_worklist(const int32_t* offsets, int B, int T, int max_len, int mask,
                                   int m, int group, WorkItem* items, int32_t* count,
                                   int32_t* hist, int max_cost, int32_t* status,
@@ -60,6 +58,17 @@ cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc, float* d_pos,
                                float* d_time, int grid, bool fast, cudaStream_t stream);
 size_t attn_bwd_tc_smem(int P, int NB);
+cudaError_t launch_ln_gate_bwd(const __nv_bfloat16* av, int64_t ld_av, const __nv_bfloat16* u,
+                               int64_t ld_u, const __nv_bfloat16* dg, int64_t ld_dg,
+                               const float* gamma, const float* beta, float eps,
+                               __nv_bfloat16* d_av, int64_t ld_dav, __nv_bfloat16* d_u,
+                               int64_t ld_du, float* d_gamma, float* d_beta, int rows, int F,
+                               int num_sms, cudaStream_t stream);
+cudaError_t launch_silu_grad_mul(const __nv_bfloat16* z, int64_t ld_z, const __nv_bfloat16* da,
+                                 int64_t ld_da, __nv_bfloat16* dz, int64_t ld_dz, int rows,
+                                 int cols, int num_sms, cudaStream_t stream);
+cudaError_t launch_colsum(const __nv_bfloat16* m, int64_t ld, int rows, int cols, float* out,
+                          cudaStream_t stream);
 int attn_bwd_tc_ts_box();
 }  // namespace hstu
 
@@ -288,12 +297,123 @@ hstu_status_t gemm(int dtype, int epi, const void* A, int64_t lda, const void* B
     CUtensorMap ta, tb;
     if (!make_map_bf16(&ta, A, M, K, lda, 64, 128) || !make_map_bf16(&tb, Bm, K, N, ldb, 64, 64))
       return HSTU_ERR_CUDA;
-    e = launch_gemm_bf16_tc(epi, ta, tb, M, N, K, bias, static_cast<const __nv_bfloat16*>(R), ldr,
-                            static_cast<__nv_bfloat16*>(C), ldc, status, s);
+    GemmArgs ga{};
+    ga.ta = &ta;
+    ga.tb = &tb;
+    ga.M = M;
+    ga.N = N;
+    ga.K = K;
+    ga.k_splits = 1;
+    ga.epi = epi;
+    ga.a_mn = 0;
+    ga.b_mn = 1;
+    ga.bias = bias;
+    ga.resid = static_cast<const __nv_bfloat16*>(R);
+    ga.ld_r = ldr;
+    ga.C = static_cast<__nv_bfloat16*>(C);
+    ga.ldc = ldc;
+    ga.status = status;
+    e = launch_gemm_tc(ga, s);
   } else {
     e = launch_gemm_simt(dtype, epi, A, lda, Bm, ldb, M, N, K, bias, R, ldr, C, ldc, s);
   }
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+}
+
+// C = epi(op(A) op(B)) on the tensor cores for the backward's operand layouts: a_mn = 1 takes A
+// stored [K, M] (lda its row stride), b_mn = 0 takes B stored [N, K].  epi 4 accumulates fp32
+// into Cf with k_splits work units per output tile.
+hstu_status_t gemm_tc_layout(int epi, int a_mn, int b_mn, const void* A, int64_t lda,
+                             const void* Bm, int64_t ldb, int M, int N, int K, int k_splits,
+                             const float* bias, const void* R, int64_t ldr, void* C, int64_t ldc, void* C2,
+                             int64_t ld_c2, float* Cf, int32_t* status, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  const bool ok_a = a_mn ? make_map_bf16(&ta, A, K, M, lda, 64, 64)
+                         : make_map_bf16(&ta, A, M, K, lda, 64, 128);
+  const bool ok_b = b_mn ? make_map_bf16(&tb, Bm, K, N, ldb, 64, 64)
+                         : make_map_bf16(&tb, Bm, N, K, ldb, 64, 256);
+  if (!ok_a || !ok_b) return HSTU_ERR_CUDA;
+  GemmArgs ga{};
+  ga.ta = &ta;
+  ga.tb = &tb;
+  ga.M = M;
+  ga.N = N;
+  ga.K = K;
+  ga.k_splits = k_splits;
+  ga.epi = epi;
+  ga.a_mn = a_mn;
+  ga.b_mn = b_mn;
+  ga.bias = bias;
+  ga.resid = static_cast<const __nv_bfloat16*>(R);
+  ga.ld_r = ldr;
+  ga.C = static_cast<__nv_bfloat16*>(C);
+  ga.ldc = ldc;
+  ga.C2 = static_cast<__nv_bfloat16*>(C2);
+  ga.ld_c2 = ld_c2;
+  ga.Cf = Cf;
+  ga.status = status;
+  const cudaError_t e = launch_gemm_tc(ga, s);
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+}
+
+// Split-K factor that gives about one work unit per SM for an M x N fp32 weight gradient.
+int weight_grad_splits(int M, int N, int K) {
+  const int tiles = gemm_tc_mn_tiles(M, N);
+  const int kblocks = (K + 63) / 64;
+  int ks = num_sms_current() / (tiles > 0 ? tiles : 1);
+  if (ks < 1) ks = 1;
+  if (ks > kblocks) ks = kblocks > 0 ? kblocks : 1;
+  return ks;
+}
+
+// Layout of the layer backward's workspace: the attention backward's (status word, work list,
+// fp32 dQ accumulator) first, then the saved and gradient activations.
+struct LayerBwdLayout {
+  size_t attn, z, a, av, g, dg, dav, da, total;
+};
+
+LayerBwdLayout layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_attn_desc_t& ad) {
+  const size_t T = static_cast<size_t>(d->total_tokens);
+  const size_t n1 = 2 * static_cast<size_t>(d->num_heads) * (d->d_qk + d->d_v);
+  const size_t hv = static_cast<size_t>(d->num_heads) * d->d_v;
+  LayerBwdLayout l;
+  l.attn = 0;
+  l.z = align_up(hstu_attention_backward_workspace_size(&ad));
+  l.a = l.z + align_up(T * n1 * 2);
+  l.av = l.a + align_up(T * n1 * 2);
+  l.g = l.av + align_up(T * hv * 2);
+  l.dg = l.g + align_up(T * hv * 2);
+  l.dav = l.dg + align_up(T * hv * 2);
+  l.da = l.dav + align_up(T * hv * 2);
+  l.total = l.da + align_up(T * n1 * 2);
+  return l;
+}
+
+// The attention problem of a layer: Q, K, V are column blocks of the f1 output [U | V | Q | K].
+hstu_attn_desc_t layer_attn_desc(const hstu_layer_desc_t* d) {
+  hstu_attn_desc_t a;
+  std::memset(&a, 0, sizeof(a));
+  const int64_t n1 = 2 * static_cast<int64_t>(d->num_heads) * (d->d_qk + d->d_v);
+  a.num_seqs = d->num_seqs;
+  a.total_tokens = d->total_tokens;
+  a.max_seq_len = d->max_seq_len;
+  a.seq_offsets = d->seq_offsets;
+  a.timestamps = d->timestamps;
+  a.num_heads = d->num_heads;
+  a.d_qk = d->d_qk;
+  a.d_v = d->d_v;
+  a.ld_q = a.ld_k = a.ld_v = n1;
+  a.ld_o = static_cast<int64_t>(d->num_heads) * d->d_v;
+  a.mask = d->mask;
+  a.num_candidates = d->num_candidates;
+  a.mfalcon_microbatch = d->mfalcon_microbatch;
+  a.rab_pos = d->rab_pos;
+  a.max_pos_dist = d->max_pos_dist;
+  a.rab_time = d->rab_time;
+  a.num_time_buckets = d->num_time_buckets;
+  a.alpha = d->alpha;
+  a.dtype = d->dtype;
+  return a;
 }
 
 }  // namespace
@@ -494,6 +614,116 @@ hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* d, const void* x, cons
         hstu_layer_forward_stage(d, stage, x, w1, b1, w2, b2, y, ws, ws_bytes, stream);
     if (st != HSTU_OK) return st;
   }
+  return HSTU_OK;
+}
+
+size_t hstu_layer_backward_workspace_size(const hstu_layer_desc_t* d) {
+  if (d == nullptr || d->total_tokens < 0 || d->num_seqs < 0 || d->max_seq_len < 0 ||
+      d->num_heads < 1 || d->d_qk < 1 || d->d_v < 1)
+    return 0;
+  const hstu_attn_desc_t ad = layer_attn_desc(d);
+  return layer_bwd_layout(d, ad).total;
+}
+
+hstu_status_t hstu_layer_backward(const hstu_layer_desc_t* d, const void* x, const void* w1,
+                                  const float* b1, const void* w2, const float* b2,
+                                  const void* d_y, void* d_x, float* d_w1, float* d_b1,
+                                  float* d_w2, float* d_b2, float* d_rab_pos, float* d_rab_time,
+                                  float* d_ln_gamma, float* d_ln_beta, void* ws,
+                                  size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
+                                  d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
+                                  d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
+                                  d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
+  if (st != HSTU_OK) return st;
+  if (d->d_model < 1 || !std::isfinite(d->ln_eps) || d->ln_eps < 0.f) return HSTU_ERR_INVALID_ARG;
+  const int H = d->num_heads, T = d->total_tokens, dm = d->d_model;
+  const int hv = H * d->d_v;
+  const int n1 = 2 * H * (d->d_qk + d->d_v);
+  // tensor-core GEMMs and 16-byte vectors throughout: bf16, widths multiples of 8, LayerNorm
+  // rows of 128 .. 1024 features held in one warp
+  if (d->dtype != HSTU_BF16 || dm % 8 != 0 || (hv != 128 && hv != 256 && hv != 512 && hv != 1024))
+    return HSTU_ERR_UNSUPPORTED;
+  const hstu_attn_desc_t ad = layer_attn_desc(d);
+  const LayerBwdLayout L = layer_bwd_layout(d, ad);
+  st = check_ws(ws, ws_bytes, L.total);
+  if (st != HSTU_OK) return st;
+  if ((d->ln_gamma != nullptr && d_ln_gamma == nullptr) ||
+      (d->ln_beta != nullptr && d_ln_beta == nullptr) || (b1 != nullptr && d_b1 == nullptr) ||
+      (b2 != nullptr && d_b2 == nullptr))
+    return HSTU_ERR_INVALID_ARG;
+  if (T == 0 || d->num_seqs == 0) return HSTU_OK;
+  const void* ptrs[] = {x, w1, w2, d_y, d_x, d_w1, d_w2};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  if (x == d_x || d_y == d_x) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(base);
+  auto* z = reinterpret_cast<__nv_bfloat16*>(base + L.z);
+  auto* a = reinterpret_cast<__nv_bfloat16*>(base + L.a);
+  auto* av = reinterpret_cast<__nv_bfloat16*>(base + L.av);
+  auto* g = reinterpret_cast<__nv_bfloat16*>(base + L.g);
+  auto* dg = reinterpret_cast<__nv_bfloat16*>(base + L.dg);
+  auto* dav = reinterpret_cast<__nv_bfloat16*>(base + L.dav);
+  auto* da = reinterpret_cast<__nv_bfloat16*>(base + L.da);
+  const size_t attn_ws = L.z;  // the attention calls' part of the workspace
+  // column blocks [U | V | Q | K] of the f1 output and of its gradient
+  const int64_t offU = 0, offV = hv, offQ = 2 * static_cast<int64_t>(hv),
+                offK = offQ + static_cast<int64_t>(H) * d->d_qk;
+  const int nsm = num_sms_current();
+
+  // ---- forward, keeping what the backward reads: Z (pre-activation), A = SiLU(Z), AV, G
+  st = gemm_tc_layout(3, 0, 1, x, dm, w1, n1, T, n1, dm, 1, b1, nullptr, 0, a, n1, z, n1, nullptr,
+                      status, s);
+  if (st != HSTU_OK) return st;
+  st = hstu_attention_forward(&ad, a + offQ, a + offK, a + offV, av, ws, attn_ws, stream);
+  if (st != HSTU_OK) return st;
+  if (launch_ln_gate(0, av, hv, a + offU, n1, d->ln_gamma, d->ln_beta, d->ln_eps, g, hv, T, hv,
+                     s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  // ---- f2 and the residual edge: dG = dY W2ᵀ, dW2 = Gᵀ dY, db2 = Σ dY
+  st = gemm_tc_layout(2, 0, 0, d_y, dm, w2, dm, T, hv, dm, 1, nullptr, nullptr, 0, dg, hv,
+                      nullptr, 0, nullptr, status, s);
+  if (st != HSTU_OK) return st;
+  cudaError_t e = cudaMemsetAsync(d_w2, 0, sizeof(float) * hv * dm, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = gemm_tc_layout(4, 1, 1, g, hv, d_y, dm, hv, dm, T, weight_grad_splits(hv, dm, T), nullptr,
+                      nullptr, 0, nullptr, dm, nullptr, 0, d_w2, status, s);
+  if (st != HSTU_OK) return st;
+  if (d_b2 != nullptr && (e = launch_colsum(static_cast<const __nv_bfloat16*>(d_y), dm, T, dm,
+                                            d_b2, s)) != cudaSuccess)
+    return cuda_fail(e);
+  // ---- gate and LayerNorm: dU into dA's U block, dAV
+  if (d_ln_gamma != nullptr && (e = cudaMemsetAsync(d_ln_gamma, 0, sizeof(float) * hv, s)) != cudaSuccess)
+    return cuda_fail(e);
+  if (d_ln_beta != nullptr && (e = cudaMemsetAsync(d_ln_beta, 0, sizeof(float) * hv, s)) != cudaSuccess)
+    return cuda_fail(e);
+  e = launch_ln_gate_bwd(av, hv, a + offU, n1, dg, hv, d->ln_gamma, d->ln_beta, d->ln_eps, dav,
+                         hv, da + offU, n1, d->ln_gamma ? d_ln_gamma : nullptr,
+                         d->ln_beta ? d_ln_beta : nullptr, T, hv, nsm, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // ---- attention: dQ, dK, dV into dA's Q, K, V blocks; the bias-table gradients
+  hstu_attn_desc_t bd = ad;
+  bd.ld_o = hv;  // dO = dAV
+  st = hstu_attention_backward(&bd, a + offQ, a + offK, a + offV, dav, da + offQ, da + offK,
+                               da + offV, d_rab_pos, d_rab_time, ws, attn_ws, stream);
+  if (st != HSTU_OK) return st;
+  // ---- SiLU and f1: dZ = dA ⊙ SiLU'(Z) (in place), dX = dY + dZ W1ᵀ, dW1 = Xᵀ dZ, db1 = Σ dZ
+  e = launch_silu_grad_mul(z, n1, da, n1, da, n1, T, n1, nsm, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = gemm_tc_layout(1, 0, 0, da, n1, w1, n1, T, dm, n1, 1, nullptr, d_y, dm, d_x, dm, nullptr,
+                      0, nullptr, status, s);
+  if (st != HSTU_OK) return st;
+  e = cudaMemsetAsync(d_w1, 0, sizeof(float) * dm * n1, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = gemm_tc_layout(4, 1, 1, x, dm, da, n1, dm, n1, T, weight_grad_splits(dm, n1, T), nullptr,
+                      nullptr, 0, nullptr, n1, nullptr, 0, d_w1, status, s);
+  if (st != HSTU_OK) return st;
+  if (d_b1 != nullptr && (e = launch_colsum(da, n1, T, n1, d_b1, s)) != cudaSuccess)
+    return cuda_fail(e);
+  (void)b2;  // b2 does not enter any gradient but its own (db2 = Σ dY)
   return HSTU_OK;
 }
 

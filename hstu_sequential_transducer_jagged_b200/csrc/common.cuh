@@ -37,6 +37,24 @@ struct AttnGeom {
   int32_t* status;
 };
 
+// One launch of the persistent tensor-core GEMM (gemm_tc.cu): C[M, N] = epi(A · B), A and B
+// through the tensor maps ta / tb in the layouts a_mn / b_mn select; see the kernel's comment.
+struct GemmArgs {
+  const CUtensorMap* ta;
+  const CUtensorMap* tb;
+  int M, N, K, k_splits;
+  int epi, a_mn, b_mn;
+  const float* bias;               // [N] or nullptr
+  const __nv_bfloat16* resid;      // epi 1
+  int64_t ld_r;
+  __nv_bfloat16* C;                // epi 0-3
+  int64_t ldc;                     // row stride of C (or of Cf for epi 4)
+  __nv_bfloat16* C2;               // epi 3: the pre-activation
+  int64_t ld_c2;
+  float* Cf;                       // epi 4: fp32 [M, N], accumulated into
+  int* status;
+};
+
 // History length n of a sequence: every token for the causal mask, L - m under M-FALCON.
 __host__ __device__ __forceinline__ int hist_len(int L, int mask, int m) {
   if (mask == 1) {

@@ -48,13 +48,29 @@ __device__ __forceinline__ float silu_fast(float x) {
 
 }  // namespace
 
-// EPI 0: C = SiLU(acc + bias);  EPI 1: C = acc + bias + R (residual, bf16 [M, N], ld_r).
-template <int EPI>
+// Operand layouts (template parameters):
+//   A_MN = 0: A is stored [M, K] row-major (K-major operand): one box {64 k, 128 m} per stage.
+//   A_MN = 1: A is stored [K, M] row-major (MN-major operand, e.g. Gᵀ of a [T, F] activation):
+//             two boxes {64 m, 64 k} per stage, 8 KB apart.
+//   B_MN = 1: B is stored [K, N] row-major (MN-major): four boxes {64 n, 64 k}, 8 KB apart.
+//   B_MN = 0: B is stored [N, K] row-major (K-major, e.g. Wᵀ of a stored weight): one box
+//             {64 k, 256 n}.
+// Epilogues:
+//   EPI 0: C = SiLU(acc + bias)                       (bf16)
+//   EPI 1: C = acc + bias + R                         (bf16, residual R [M, N] with ld_r)
+//   EPI 2: C = acc + bias                             (bf16)
+//   EPI 3: C = SiLU(acc + bias) and C2 = acc + bias   (bf16, C2 with ld_c2: the pre-activation)
+//   EPI 4: Cf += acc                                  (fp32, atomic: split-K partial sums)
+// With k_splits > 1 each output tile is computed by k_splits work units over consecutive K
+// ranges (EPI 4 only).
+template <int EPI, int A_MN, int B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b, int M, int N, int K,
-                        const float* __restrict__ bias, const __nv_bfloat16* __restrict__ resid,
-                        int64_t ld_r, __nv_bfloat16* __restrict__ C, int64_t ldc,
+                        int k_splits, const float* __restrict__ bias,
+                        const __nv_bfloat16* __restrict__ resid, int64_t ld_r,
+                        __nv_bfloat16* __restrict__ C, int64_t ldc,
+                        __nv_bfloat16* __restrict__ C2, int64_t ld_c2, float* __restrict__ Cf,
                         int* status) {
   if (*reinterpret_cast<volatile int*>(status) == kStatusTimeout) return;
   extern __shared__ uint8_t smem_raw[];
@@ -63,8 +79,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int kblocks = (K + kBK - 1) / kBK;
+  const int kb_per = (kblocks + k_splits - 1) / k_splits;
   const int n_tiles = (N + kBN - 1) / kBN;
-  const int tiles = ((M + kBM - 1) / kBM) * n_tiles;
+  const int mn_tiles = ((M + kBM - 1) / kBM) * n_tiles;
+  const int tiles = mn_tiles * k_splits;
   const int stride = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
@@ -98,9 +116,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int g = 0;  // K blocks issued so far (the ring runs on across tiles)
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += stride) {
-        const int m0 = (t / n_tiles) * kBM;
-        const int n0 = (t % n_tiles) * kBN;
-        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+        const int mn = t % mn_tiles, ks = t / mn_tiles;
+        const int m0 = (mn / n_tiles) * kBM;
+        const int n0 = (mn % n_tiles) * kBN;
+        const int kb1 = min(kblocks, (ks + 1) * kb_per);
+        for (int kb = ks * kb_per; kb < kb1; ++kb, ++g) {
           const int st = g % kGemmStages;
           if (g >= kGemmStages &&
               !mbar_wait(&sm.empty[st], ((g / kGemmStages) - 1) & 1, abort_flag, status)) {
@@ -108,10 +128,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&sm.full[st], kABytes + kBBytes);
-          tma_load_2d(sm.a[st], &tm_a, &sm.full[st], kb * kBK, m0);
+          if (A_MN) {
 #pragma unroll
-          for (int q = 0; q < kBN / 64; ++q)
-            tma_load_2d(sm.b[st] + q * (kBK * 128), &tm_b, &sm.full[st], n0 + 64 * q, kb * kBK);
+            for (int q = 0; q < kBM / 64; ++q)
+              tma_load_2d(sm.a[st] + q * (kBK * 128), &tm_a, &sm.full[st], m0 + 64 * q, kb * kBK);
+          } else {
+            tma_load_2d(sm.a[st], &tm_a, &sm.full[st], kb * kBK, m0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int q = 0; q < kBN / 64; ++q)
+              tma_load_2d(sm.b[st] + q * (kBK * 128), &tm_b, &sm.full[st], n0 + 64 * q, kb * kBK);
+          } else {
+            tma_load_2d(sm.b[st], &tm_b, &sm.full[st], kb * kBK, n0);
+          }
         }
       }
       if (!ok) {  // leave no TMA write in flight into shared memory about to be released
@@ -123,12 +153,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 1);
-      const uint64_t da0 = smem_desc_sw128(smem_u32(sm.a[0]), 16, 1024);
-      const uint64_t db0 = smem_desc_sw128(smem_u32(sm.b[0]), kBK * 128, 1024);
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, A_MN, B_MN);
+      // K-major: the next 16 k are 32 bytes further in the swizzled row; MN-major: 16 rows of
+      // 128 bytes further, with the 64-wide M (N) chunks kBK x 128 bytes apart
+      const uint64_t da0 = A_MN ? smem_desc_sw128(smem_u32(sm.a[0]), kBK * 128, 1024)
+                                : smem_desc_sw128(smem_u32(sm.a[0]), 16, 1024);
+      const uint64_t db0 = B_MN ? smem_desc_sw128(smem_u32(sm.b[0]), kBK * 128, 1024)
+                                : smem_desc_sw128(smem_u32(sm.b[0]), 16, 1024);
+      constexpr uint64_t a_step = A_MN ? 128 : 2;
+      constexpr uint64_t b_step = B_MN ? 128 : 2;
       int g = 0, j = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += stride, ++j) {
+        const int ks = t / mn_tiles;
+        const int kb0 = ks * kb_per, kb1 = min(kblocks, (ks + 1) * kb_per);
         const int ab = j & 1;
         // the epilogue has read this accumulator buffer's previous tile
         if (j >= 2 && !mbar_wait(&sm.acc_empty[ab], ((j - 2) >> 1) & 1, abort_flag, status)) {
@@ -137,7 +175,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem + 256u * ab;
-        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const int st = g % kGemmStages;
           if (!mbar_wait(&sm.full[st], (g / kGemmStages) & 1, abort_flag, status)) {
             ok = false;
@@ -148,7 +186,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t db = db0 + static_cast<uint64_t>(st) * (kBBytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ss(d, da + 2 * kk, db + 128 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ss(d, da + a_step * kk, db + b_step * kk, idesc,
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
           mma_commit(&sm.empty[st]);
         }
         if (ok) mma_commit(&sm.acc_full[ab]);
@@ -167,18 +206,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int j = 0;
     for (int t = blockIdx.x; t < tiles; t += stride, ++j) {
       const int ab = j & 1;
-      const int m0 = (t / n_tiles) * kBM;
-      const int n0 = (t % n_tiles) * kBN + 128 * half;
+      const int mn = t % mn_tiles, ks = t / mn_tiles;
+      const int m0 = (mn / n_tiles) * kBM;
+      const int n0 = (mn % n_tiles) * kBN + 128 * half;
       const int row = m0 + quad * 32 + lane;
       if (!warp_all(mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, abort_flag, status))) break;
       tc_fence_after();
+      // a K range past the end (k_splits not dividing the K blocks) contributed nothing
+      const bool empty_range = ks * kb_per >= kblocks;
 #pragma unroll 1
       for (int ch = 0; ch < 128 / 32; ++ch) {
         uint32_t acc[32];
         tmem_ld32(lane_addr + 256u * ab + ch * 32, acc);
         tmem_wait_ld();
         const int c0 = n0 + ch * 32;
-        if (row < M && c0 < N) {
+        if (row < M && c0 < N && !empty_range) {
+          if constexpr (EPI == 4) {
+            float* cp = Cf + static_cast<int64_t>(row) * ldc + c0;
+            if (c0 + 32 <= N) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                atomicAdd(reinterpret_cast<float4*>(cp + e),
+                          make_float4(__uint_as_float(acc[e]), __uint_as_float(acc[e + 1]),
+                                      __uint_as_float(acc[e + 2]), __uint_as_float(acc[e + 3])));
+            } else {
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < N) atomicAdd(cp + e, __uint_as_float(acc[e]));
+            }
+          } else {
           float vals[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -186,6 +241,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float x = __uint_as_float(acc[e]);
             if (bias != nullptr && c < N) x += __ldg(bias + c);
             vals[e] = x;
+          }
+          if (EPI == 3) {  // the pre-activation, before the SiLU overwrites vals
+            __nv_bfloat16* pp = C2 + static_cast<int64_t>(row) * ld_c2 + c0;
+            if (c0 + 32 <= N) {
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                uint4 ov;
+                ov.x = pack_bf16x2(vals[8 * w + 0], vals[8 * w + 1]);
+                ov.y = pack_bf16x2(vals[8 * w + 2], vals[8 * w + 3]);
+                ov.z = pack_bf16x2(vals[8 * w + 4], vals[8 * w + 5]);
+                ov.w = pack_bf16x2(vals[8 * w + 6], vals[8 * w + 7]);
+                reinterpret_cast<uint4*>(pp)[w] = ov;
+              }
+            } else {
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < N) pp[e] = __float2bfloat16_rn(vals[e]);
+            }
           }
           if (EPI == 1) {
             const __nv_bfloat16* rp = resid + static_cast<int64_t>(row) * ld_r + c0;
@@ -206,7 +278,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int e = 0; e < 32; ++e)
                 if (c0 + e < N) vals[e] += __bfloat162float(rp[e]);
             }
-          } else {
+          } else if (EPI == 0 || EPI == 3) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) vals[e] = silu_fast(vals[e]);
           }
@@ -226,6 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (c0 + e < N) cp[e] = __float2bfloat16_rn(vals[e]);
           }
+          }
         }
       }
       // this warp's part of the accumulator buffer is read: the MMA warp may reuse it
@@ -242,32 +315,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-cudaError_t launch_gemm_bf16_tc(int epi, const CUtensorMap& ta, const CUtensorMap& tb, int M,
-                                int N, int K, const float* bias, const __nv_bfloat16* resid,
-                                int64_t ld_r, __nv_bfloat16* C, int64_t ldc, int* status,
-                                cudaStream_t stream) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
+namespace {
+template <int EPI, int A_MN, int B_MN>
+cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  auto kern = gemm_bf16_tc_kernel<EPI, A_MN, B_MN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kGemmThreads, smem, stream>>>(*a.ta, *a.tb, a.M, a.N, a.K, a.k_splits, a.bias,
+                                             a.resid, a.ld_r, a.C, a.ldc, a.C2, a.ld_c2, a.Cf,
+                                             a.status);
+  return cudaGetLastError();
+}
+}  // namespace
+
+// Tiles of one launch for the given shape, before split-K.
+int gemm_tc_mn_tiles(int M, int N) { return ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN); }
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream) {
+  if (a.M <= 0 || a.N <= 0) return cudaSuccess;
+  if (a.k_splits < 1 || (a.k_splits > 1 && a.epi != 4)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(GemmSmem) + 1024;
-  const int tiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+  const int tiles = gemm_tc_mn_tiles(a.M, a.N) * a.k_splits;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = tiles < sms ? tiles : sms;
-  cudaError_t e;
-  if (epi == 0) {
-    e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    gemm_bf16_tc_kernel<0><<<grid, kGemmThreads, smem, stream>>>(ta, tb, M, N, K, bias, resid,
-                                                                  ld_r, C, ldc, status);
-  } else {
-    e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    gemm_bf16_tc_kernel<1><<<grid, kGemmThreads, smem, stream>>>(ta, tb, M, N, K, bias, resid,
-                                                                  ld_r, C, ldc, status);
+  const int key = a.epi * 4 + a.a_mn * 2 + a.b_mn;
+  switch (key) {
+    case 0 * 4 + 0 * 2 + 1: return launch_gemm_t<0, 0, 1>(a, grid, smem, stream);  // f1 + SiLU
+    case 1 * 4 + 0 * 2 + 1: return launch_gemm_t<1, 0, 1>(a, grid, smem, stream);  // f2 + residual
+    case 3 * 4 + 0 * 2 + 1: return launch_gemm_t<3, 0, 1>(a, grid, smem, stream);  // f1, pre kept
+    case 2 * 4 + 0 * 2 + 0: return launch_gemm_t<2, 0, 0>(a, grid, smem, stream);  // dY W2^T
+    case 1 * 4 + 0 * 2 + 0: return launch_gemm_t<1, 0, 0>(a, grid, smem, stream);  // dY + dZ W1^T
+    case 4 * 4 + 1 * 2 + 1: return launch_gemm_t<4, 1, 1>(a, grid, smem, stream);  // X^T dZ
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace hstu

@@ -176,6 +176,35 @@ hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* desc, const void* x, c
                                  const float* b1, const void* w2, const float* b2, void* y,
                                  void* ws, size_t ws_bytes, hstu_stream_t stream);
 
+/* Bytes of workspace hstu_layer_backward needs: the attention backward's workspace, then the
+ * saved forward activations (f1 pre-activation and output [T, 2H(d_qk+d_v)] each, the attention
+ * output and the gated norm [T, H d_v] each) and the gradient activations (dG and dAV
+ * [T, H d_v], the f1 output's gradient [T, 2H(d_qk+d_v)]). */
+size_t hstu_layer_backward_workspace_size(const hstu_layer_desc_t* desc);
+
+/* Gradients of L = Σ d_y ⊙ Y through one layer Y = X + f2(Norm(A(X)V(X)) ⊙ U(X)): the chain rule
+ * of [Review §2.1] backwards through f2 and the residual edge, the gate and LayerNorm, the
+ * attention ([GenRank 6.2] §6.2.3, the relative-bias gradient), the SiLU and f1 — the training
+ * pass over whole user sequences of [FunRec 7.1] §7.1.3.  The forward is recomputed inside the
+ * call (nothing is kept between calls), so it needs only the layer's inputs:
+ *   d_x = dY + dpre W1ᵀ            bf16 [T, d_model] (may not alias x or d_y)
+ *   d_w1 = Xᵀ dpre                 fp32 [d_model, 2H(d_qk+d_v)]
+ *   d_b1 = Σ_t dpre                fp32 [2H(d_qk+d_v)]  (required when b1 != NULL, else may be NULL)
+ *   d_w2 = Gᵀ dY                   fp32 [H d_v, d_model]
+ *   d_b2 = Σ_t dY                  fp32 [d_model]       (may be NULL)
+ *   d_rab_pos, d_rab_time          fp32 tables, as hstu_attention_backward (overwritten)
+ *   d_ln_gamma, d_ln_beta          fp32 [H d_v], required when ln_gamma / ln_beta are set
+ * with dpre = [dU | dV | dQ | dK] ⊙ SiLU'(X W1 + b1).  Every output is overwritten.  bf16 only,
+ * d_model a multiple of 8 and H d_v in {128, 256, 512, 1024} (else HSTU_ERR_UNSUPPORTED);
+ * 16-byte aligned pointers.  Weight gradients are fp32 sums in no fixed order (atomic split-K
+ * reduction), so they are reproducible only to rounding. */
+hstu_status_t hstu_layer_backward(const hstu_layer_desc_t* desc, const void* x, const void* w1,
+                                  const float* b1, const void* w2, const float* b2,
+                                  const void* d_y, void* d_x, float* d_w1, float* d_b1,
+                                  float* d_w2, float* d_b2, float* d_rab_pos, float* d_rab_time,
+                                  float* d_ln_gamma, float* d_ln_beta, void* ws,
+                                  size_t ws_bytes, hstu_stream_t stream);
+
 /* Stages of hstu_layer_forward, callable one at a time (e.g. to time each kernel).  The
  * intermediates live in ws at fixed offsets, so the stages must run in order on one workspace:
  *   HSTU_STAGE_F1           uvqk = SiLU(x W1 + b1)                       (tensor-core GEMM)
