@@ -31,6 +31,7 @@ EXPORTED = [
     "hstu_status_string", "hstu_version", "hstu_last_error_string",
     "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout", "hstu_alibi_tables",
     "hstu_debug_bias_index", "hstu_layer_backward_workspace_size", "hstu_layer_backward",
+    "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
 ]
 
 # Rules of hstu_debug_bias_index (hstu_bias_rule_t)
@@ -94,6 +95,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_layer_forward": (i32, [ldp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_layer_forward_stage": (i32, [ldp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_layer_backward_workspace_size": (sz, [ldp]),
+        "hstu_stochastic_length_workspace_size": (sz, [i32, i32]),
+        "hstu_stochastic_length": (i32, [vp, i32, i32, i32, i32, ctypes.c_double, vp, vp, vp, vp,
+                                         vp, sz, vp]),
+        "hstu_gather_rows": (i32, [vp, i64, vp, vp, i32, vp, i64, i64, vp]),
         "hstu_layer_backward": (i32, [ldp] + [vp] * 15 + [vp, sz, vp]),
         "hstu_jagged_padded_copy": (i32, [vp, i32, i32, vp, i64, vp, i64, i64, i32, vp]),
         "hstu_debug_time_buckets": (i32, [vp, i32, vp, i32, vp]),
@@ -350,6 +355,38 @@ def layer_backward(x, w1, w2, d_y, seq_offsets, max_seq_len, timestamps=None, ra
         _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["db1"]), _ptr(out["dw2"]), _ptr(out["db2"]),
         _ptr(out["d_rab_pos"]), _ptr(out["d_rab_time"]), _ptr(out["d_ln_gamma"]),
         _ptr(out["d_ln_beta"]), ws.ptr, ws.nbytes, _stream_ptr(stream)), "hstu_layer_backward")
+    return out
+
+
+def stochastic_length(seq_offsets, max_seq_len, u, token_keys, *, sub_len, n_alpha,
+                      ws: Optional[Workspace] = None, stream=None):
+    """(new_offsets, kept_index) of hstu_stochastic_length: int32 device tensors [B+1] and [T]
+    (only the first new_offsets[B] entries of kept_index are meaningful)."""
+    B = seq_offsets.numel() - 1
+    T = token_keys.numel()
+    new_off = torch.empty(B + 1, dtype=torch.int32, device=seq_offsets.device)
+    kept = torch.empty(max(T, 1), dtype=torch.int32, device=seq_offsets.device)
+    need = lib().hstu_stochastic_length_workspace_size(B, T)
+    ws = workspace(need, seq_offsets.device) if ws is None else ws.ensure(need)
+    _check(lib().hstu_stochastic_length(_ptr(seq_offsets), B, T, int(max_seq_len), int(sub_len),
+                                        float(n_alpha), _ptr(u), _ptr(token_keys), _ptr(new_off),
+                                        _ptr(kept), ws.ptr, ws.nbytes, _stream_ptr(stream)),
+           "hstu_stochastic_length")
+    return new_off, kept
+
+
+def gather_rows(src: torch.Tensor, index: torch.Tensor, count: Optional[torch.Tensor] = None,
+                max_rows: Optional[int] = None, out: Optional[torch.Tensor] = None, stream=None):
+    """out[r] = src[index[r]] for r < min(count, max_rows) (hstu_gather_rows); src 1-D or 2-D."""
+    n = int(index.numel() if max_rows is None else max_rows)
+    row = src.view(src.shape[0], -1)
+    if out is None:
+        out = torch.zeros((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    o2 = out.view(out.shape[0], -1)
+    rb = row.shape[1] * row.element_size()
+    _check(lib().hstu_gather_rows(_ptr(row), row.stride(0) * row.element_size(), _ptr(index),
+                                  _ptr(count), n, _ptr(o2), o2.stride(0) * o2.element_size(), rb,
+                                  _stream_ptr(stream)), "hstu_gather_rows")
     return out
 
 

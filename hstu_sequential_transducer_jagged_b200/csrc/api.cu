@@ -67,6 +67,13 @@ cudaError_t launch_ln_gate_bwd(const __nv_bfloat16* av, int64_t ld_av, const __n
 cudaError_t launch_silu_grad_mul(const __nv_bfloat16* z, int64_t ld_z, const __nv_bfloat16* da,
                                  int64_t ld_da, __nv_bfloat16* dz, int64_t ld_dz, int rows,
                                  int cols, int num_sms, cudaStream_t stream);
+cudaError_t launch_stochastic_length(const int32_t* off, int B, int T, int max_len, int sub_len,
+                                     double n_alpha, const float* u, const uint32_t* keys,
+                                     int32_t* local_idx, int32_t* lens, int32_t* new_off,
+                                     int32_t* kept, int32_t* status, cudaStream_t stream);
+cudaError_t launch_gather_rows(const void* src, int64_t src_stride, const int32_t* index,
+                               const int32_t* count, int n, void* dst, int64_t dst_stride,
+                               int64_t row_bytes, int num_sms, cudaStream_t stream);
 cudaError_t launch_colsum(const __nv_bfloat16* m, int64_t ld, int rows, int cols, float* out,
                           cudaStream_t stream);
 int attn_bwd_tc_ts_box();
@@ -725,6 +732,57 @@ hstu_status_t hstu_layer_backward(const hstu_layer_desc_t* d, const void* x, con
     return cuda_fail(e);
   (void)b2;  // b2 does not enter any gradient but its own (db2 = Σ dY)
   return HSTU_OK;
+}
+
+size_t hstu_stochastic_length_workspace_size(int32_t num_seqs, int32_t total_tokens) {
+  if (num_seqs < 0 || total_tokens < 0) return 0;
+  return kStatusBytes + align_up(sizeof(int32_t) * static_cast<size_t>(total_tokens)) +
+         align_up(sizeof(int32_t) * static_cast<size_t>(num_seqs));
+}
+
+hstu_status_t hstu_stochastic_length(const int32_t* seq_offsets, int32_t num_seqs,
+                                     int32_t total_tokens, int32_t max_seq_len, int32_t sub_len,
+                                     double n_alpha, const float* u, const uint32_t* token_keys,
+                                     int32_t* new_offsets, int32_t* kept_index, void* ws,
+                                     size_t ws_bytes, hstu_stream_t stream) {
+  if (num_seqs < 0 || total_tokens < 0 || max_seq_len < 0 || max_seq_len > kMaxSeqLen ||
+      sub_len < 1 || !std::isfinite(n_alpha) || n_alpha < 0.0)
+    return HSTU_ERR_INVALID_ARG;
+  if (total_tokens > 0 && static_cast<int64_t>(num_seqs) * max_seq_len < total_tokens)
+    return HSTU_ERR_INVALID_ARG;
+  const hstu_status_t st =
+      check_ws(ws, ws_bytes, hstu_stochastic_length_workspace_size(num_seqs, total_tokens));
+  if (st != HSTU_OK) return st;
+  if (new_offsets == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (num_seqs > 0 && (seq_offsets == nullptr || u == nullptr)) return HSTU_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (token_keys == nullptr || kept_index == nullptr))
+    return HSTU_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* local_idx = reinterpret_cast<int32_t*>(base + kStatusBytes);
+  int32_t* lens = reinterpret_cast<int32_t*>(
+      base + kStatusBytes + align_up(sizeof(int32_t) * static_cast<size_t>(total_tokens)));
+  const cudaError_t e = launch_stochastic_length(
+      seq_offsets, num_seqs, total_tokens, max_seq_len, sub_len, n_alpha, u, token_keys,
+      local_idx, lens, new_offsets, kept_index, reinterpret_cast<int32_t*>(base),
+      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+}
+
+hstu_status_t hstu_gather_rows(const void* src, int64_t src_row_stride_bytes,
+                               const int32_t* index, const int32_t* count, int32_t max_rows,
+                               void* dst, int64_t dst_row_stride_bytes, int64_t row_bytes,
+                               hstu_stream_t stream) {
+  if (max_rows < 0 || row_bytes < 0) return HSTU_ERR_INVALID_ARG;
+  if (max_rows == 0 || row_bytes == 0) return HSTU_OK;
+  if (src == nullptr || dst == nullptr || index == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (row_bytes % 4 != 0 || src_row_stride_bytes % 4 != 0 || dst_row_stride_bytes % 4 != 0 ||
+      (reinterpret_cast<uintptr_t>(src) & 3) != 0 || (reinterpret_cast<uintptr_t>(dst) & 3) != 0 ||
+      src_row_stride_bytes < row_bytes || dst_row_stride_bytes < row_bytes)
+    return HSTU_ERR_INVALID_ARG;
+  const cudaError_t e = launch_gather_rows(src, src_row_stride_bytes, index, count, max_rows, dst,
+                                           dst_row_stride_bytes, row_bytes, num_sms_current(),
+                                           reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
 hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_seqs,

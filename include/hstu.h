@@ -232,6 +232,41 @@ hstu_status_t hstu_jagged_padded_copy(const int32_t* seq_offsets, int32_t num_se
                                       int64_t padded_row_stride_bytes, int64_t row_bytes,
                                       int32_t to_padded, hstu_stream_t stream);
 
+/* Stochastic Length of "HSTU：Scaling Law 的首次探索" §7.1.5: long sequences are, at random,
+ * replaced by a shorter subsequence while training, which cuts the attention's O(n²) work.  The
+ * page's formula is garbled; this library reads it as: a sequence of n tokens stays whole when
+ * n <= N^{α/2}; otherwise, with probability 1 - N^α / n², it is replaced by sub_len =
+ * floor(N^{α/2}) of its tokens in their original order, else it stays whole (N the longest length
+ * the data allows, α in (1, 2]; α = 2 never truncates).  The page picks the subsequence "by
+ * feature weighting" without saying how; here it is uniformly random: the sub_len tokens with
+ * the smallest token_keys (ties to the lower index).
+ *   sub_len = floor(N^{α/2}) >= 1 and n_alpha = N^α are computed by the caller, so that the
+ *   decision u[b] < 1 - n_alpha / n² is the same fp64 expression everywhere.
+ *   u: device fp32 [B], uniform draws on [0, 1), one per sequence; token_keys: device uint32 [T],
+ *   random keys (the random numbers are inputs: the result is a pure function of them).
+ *   new_offsets: device int32 [B+1] out, the offsets of the kept tokens; kept_index: device
+ *   int32 [T] out, the global indices of the kept tokens in the new order (its first
+ *   new_offsets[B] entries are written).  ws: hstu_stochastic_length_workspace_size bytes
+ *   (status word first; zero it once with hstu_workspace_init).  Malformed seq_offsets set the
+ *   status word (HSTU_ERR_DEVICE_CHECK) and those sequences keep no token.
+ * New total and lengths live on the device; read new_offsets back when the host needs them.
+ * hstu_gather_rows then moves any per-token array (embeddings, timestamps) to the new layout. */
+size_t hstu_stochastic_length_workspace_size(int32_t num_seqs, int32_t total_tokens);
+hstu_status_t hstu_stochastic_length(const int32_t* seq_offsets, int32_t num_seqs,
+                                     int32_t total_tokens, int32_t max_seq_len, int32_t sub_len,
+                                     double n_alpha, const float* u, const uint32_t* token_keys,
+                                     int32_t* new_offsets, int32_t* kept_index, void* ws,
+                                     size_t ws_bytes, hstu_stream_t stream);
+
+/* dst row r = src row index[r] for r < min(*count, max_rows) (count: device int32, e.g.
+ * &new_offsets[B] of hstu_stochastic_length; NULL gathers max_rows rows).  index: device int32.
+ * Rows of row_bytes bytes; pointers, strides and row_bytes multiples of 4 (16-byte vectors when
+ * all are multiples of 16).  Asynchronous on stream. */
+hstu_status_t hstu_gather_rows(const void* src, int64_t src_row_stride_bytes,
+                               const int32_t* index, const int32_t* count, int32_t max_rows,
+                               void* dst, int64_t dst_row_stride_bytes, int64_t row_bytes,
+                               hstu_stream_t stream);
+
 /* Tables for the parameter-free relative bias of "6.2 HSTU的工程突破" §6.2.3, Eq. (6.2.6):
  * bias(i, j) = -m_p (p_i - p_j) - m_t bucket(t_i - t_j).  The bias is linear in the integer
  * position difference and in the bucket index, so it is the learned-table bias with

@@ -465,3 +465,48 @@ def attention_forward_alibi(q, k, v, seq_offsets, timestamps, m_p, m_t, *, num_h
             scores = alpha * (Q[s:e, h, :] @ K[s:e, h, :].T) + bias
             out[s:e, h, :] = np.where(ok, silu(scores), 0.0) @ V[s:e, h, :]
     return out.reshape(T, H * d_v)
+
+
+# --------------------------------------------------------------------------------------------
+# Stochastic Length ([FunRec 7.1] §7.1.5): long sequences are, at random, replaced by a shorter
+# subsequence during training.  The page's formula is garbled; the reading used here:
+#   a sequence of length n is left whole when n <= N^{α/2}; otherwise, with probability
+#   p = 1 - N^α / n², it is replaced by a subsequence of N^{α/2} of its tokens (keeping their
+#   order), and with probability 1 - p it is left whole.  N is the longest sequence length the
+#   data allows, α in (1, 2] (α = 2: never truncated).  The page selects the subsequence "by
+#   feature weighting" without saying how; the plainest reading, a uniformly random subset, is
+#   taken: the N^{α/2} tokens with the smallest random keys (ties broken by the lower index).
+# The random draws are inputs: u[b] (uniform on [0, 1)) decides per sequence, key[t] (uint32)
+# orders the tokens.  sub_len = floor(N^{α/2}) and n_alpha = N^α are passed as numbers, so that
+# the decision u < 1 - n_alpha / n² is taken in fp64 from the same operands on every side.
+# --------------------------------------------------------------------------------------------
+
+def stochastic_length_params(max_len_N: int, alpha: float):
+    """(sub_len, n_alpha) = (floor(N^{α/2}), N^α) for the longest length N and exponent α."""
+    return int(np.floor(float(max_len_N) ** (alpha / 2.0))), float(max_len_N) ** alpha
+
+
+def stochastic_length(seq_offsets, u, keys, sub_len: int, n_alpha: float):
+    """Per sequence: whole, or the sub_len tokens with the smallest (key, index), in index order.
+
+    Returns (new_offsets int64 [B+1], kept int64 [T']): kept lists the global index of every
+    token that stays, sequence by sequence, in increasing order; new_offsets delimits them.
+    """
+    seq_offsets = np.asarray(seq_offsets, dtype=np.int64)
+    keys = np.asarray(keys, dtype=np.uint32)
+    u = np.asarray(u, dtype=np.float32)
+    new_off = [0]
+    kept = []
+    for b in range(len(seq_offsets) - 1):
+        s, e = int(seq_offsets[b]), int(seq_offsets[b + 1])
+        n = e - s
+        idx = np.arange(s, e, dtype=np.int64)
+        p = 1.0 - float(n_alpha) / (float(n) * float(n)) if n > 0 else 0.0
+        if n > sub_len and float(u[b]) < p:
+            # sort by (key, index) and keep the first sub_len, then restore the index order
+            order = np.lexsort((idx, keys[s:e].astype(np.int64)))
+            idx = np.sort(idx[order[:sub_len]])
+        kept.append(idx)
+        new_off.append(new_off[-1] + len(idx))
+    kept = np.concatenate(kept) if kept else np.zeros(0, np.int64)
+    return np.array(new_off, dtype=np.int64), kept

@@ -517,3 +517,58 @@ def test_layer_backward_zero_w2_passes_dy_through():
     for name in ("dw1", "db1", "d_rab_pos", "d_rab_time", "d_ln_gamma", "d_ln_beta"):
         assert not np.any(g[name]), name
     assert np.abs(g["dw2"]).max() > 0
+
+
+# ----------------------------------------------------------------- Stochastic Length (§7.1.5)
+def test_stochastic_length_alpha_two_keeps_everything():
+    """α = 2: N^{α/2} = N, so no sequence of at most N tokens is truncated."""
+    rng = np.random.default_rng(0)
+    lengths = rng.integers(0, 512, size=20)
+    off = W.offsets_from_lengths(lengths)
+    sub_len, n_alpha = O.stochastic_length_params(512, 2.0)
+    assert sub_len == 512 and n_alpha == 512.0 ** 2
+    new_off, kept = O.stochastic_length(off, rng.random(20).astype(np.float32),
+                                        rng.integers(0, 2 ** 32, int(off[-1]), dtype=np.uint64)
+                                        .astype(np.uint32), sub_len, n_alpha)
+    assert np.array_equal(new_off, off) and np.array_equal(kept, np.arange(off[-1]))
+
+
+def test_stochastic_length_selection_brute_force():
+    """A truncated sequence keeps exactly the sub_len tokens of smallest (key, index), counted
+    pair by pair, in index order; ties in the keys go to the lower index."""
+    rng = np.random.default_rng(1)
+    for trial in range(30):
+        n = int(rng.integers(2, 60))
+        sub_len = int(rng.integers(1, n))
+        keys = rng.integers(0, 8 if trial % 2 else 2 ** 32, size=n, dtype=np.uint64).astype(np.uint32)
+        off = np.array([0, n])
+        _, kept = O.stochastic_length(off, np.array([0.0], np.float32), keys, sub_len, 0.0)
+        rank = np.array([sum((int(keys[s]), s) < (int(keys[t]), t) for s in range(n))
+                         for t in range(n)])
+        assert np.array_equal(kept, np.nonzero(rank < sub_len)[0])
+
+
+def test_stochastic_length_probability():
+    """A sequence longer than N^{α/2} is truncated with probability 1 - N^α / n² (binomial
+    check over 20 000 sequences, 5 standard deviations)."""
+    N, alpha, n = 4096, 1.7, 3000
+    sub_len, n_alpha = O.stochastic_length_params(N, alpha)
+    rng = np.random.default_rng(2)
+    B = 20000
+    off = np.arange(B + 1, dtype=np.int64) * n
+    keys = np.zeros(B * n, dtype=np.uint32)
+    new_off, _ = O.stochastic_length(off, rng.random(B).astype(np.float32), keys, sub_len, n_alpha)
+    frac = np.mean(np.diff(new_off) == sub_len)
+    p = 1.0 - n_alpha / n ** 2
+    assert abs(frac - p) <= 5 * np.sqrt(p * (1 - p) / B)
+
+
+def test_stochastic_length_sparsity_claim():
+    """The page reports 80%+ sequence sparsity at α about 1.6-1.7: for sequences of the longest
+    length N = 8192 the expected fraction of causal attention pairs kept is below 20 %."""
+    N = 8192
+    for alpha in (1.6, 1.7):
+        k, n_alpha = O.stochastic_length_params(N, alpha)
+        p = 1.0 - n_alpha / N ** 2
+        kept_pairs = p * k * (k + 1) / 2 + (1 - p) * N * (N + 1) / 2
+        assert kept_pairs / (N * (N + 1) / 2) < 0.2, alpha
