@@ -32,6 +32,8 @@ EXPORTED = [
     "hstu_attention_forward_static_ws", "hstu_debug_wait_timeout", "hstu_alibi_tables",
     "hstu_debug_bias_index", "hstu_layer_backward_workspace_size", "hstu_layer_backward",
     "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
+    "hstu_layer_cache_bytes", "hstu_layer_forward_cached", "hstu_layer_candidates_workspace_size",
+    "hstu_layer_forward_candidates",
 ]
 
 # Rules of hstu_debug_bias_index (hstu_bias_rule_t)
@@ -95,6 +97,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_layer_forward": (i32, [ldp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_layer_forward_stage": (i32, [ldp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_layer_backward_workspace_size": (sz, [ldp]),
+        "hstu_layer_cache_bytes": (sz, [ldp]),
+        "hstu_layer_forward_cached": (i32, [ldp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "hstu_layer_candidates_workspace_size": (sz, [ldp]),
+        "hstu_layer_forward_candidates": (i32, [ldp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_stochastic_length_workspace_size": (sz, [i32, i32]),
         "hstu_stochastic_length": (i32, [vp, i32, i32, i32, i32, ctypes.c_double, vp, vp, vp, vp,
                                          vp, sz, vp]),
@@ -320,6 +326,59 @@ def layer_forward(x, w1, w2, seq_offsets, max_seq_len, timestamps=None, rab_pos=
     _check(lib().hstu_layer_forward(ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2),
                                     _ptr(b2), _ptr(out), ws.ptr, ws.nbytes, _stream_ptr(stream)),
            "hstu_layer_forward")
+    return out
+
+
+def _layer_call_desc(x_rows_T, seq_offsets, max_seq_len, timestamps, d_model, dtype, **kw):
+    return layer_desc(seq_offsets=seq_offsets, total_tokens=x_rows_T, max_seq_len=max_seq_len,
+                      timestamps=timestamps, d_model=d_model, dtype=dtype, **kw)
+
+
+def layer_forward_cached(x, w1, w2, cache, seq_offsets, max_seq_len, timestamps=None,
+                         rab_pos=None, rab_time=None, *, num_heads, d_qk, d_v, max_pos_dist=0,
+                         num_time_buckets=1, alpha=1.0, num_candidates, microbatch=128, b1=None,
+                         b2=None, ln_eps=1e-5, out=None, ws: Optional[Workspace] = None,
+                         stream=None):
+    """M-FALCON prefill (hstu_layer_forward_cached): the layer forward, keeping its f1 output in
+    cache (a [T, 2H(d_qk+d_v)] tensor of x's dtype)."""
+    T, d_model = x.shape
+    out = torch.empty_like(x) if out is None else out
+    desc = _layer_call_desc(T, seq_offsets, max_seq_len, timestamps, d_model, _dtype_code(x),
+                            num_heads=num_heads, d_qk=d_qk, d_v=d_v, mask=MASK_MFALCON,
+                            num_candidates=num_candidates, microbatch=microbatch,
+                            rab_pos=rab_pos, max_pos_dist=max_pos_dist, rab_time=rab_time,
+                            num_time_buckets=num_time_buckets, alpha=alpha, ln_eps=ln_eps)
+    need = lib().hstu_layer_workspace_size(ctypes.byref(desc))
+    ws = workspace(need, x.device) if ws is None else ws.ensure(need)
+    _check(lib().hstu_layer_forward_cached(ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1),
+                                           _ptr(w2), _ptr(b2), _ptr(out), _ptr(cache), ws.ptr,
+                                           ws.nbytes, _stream_ptr(stream)),
+           "hstu_layer_forward_cached")
+    return out
+
+
+def layer_forward_candidates(x_cand, w1, w2, cache, seq_offsets, total_tokens, max_seq_len,
+                             timestamps=None, rab_pos=None, rab_time=None, *, num_heads, d_qk,
+                             d_v, max_pos_dist=0, num_time_buckets=1, alpha=1.0, num_candidates,
+                             microbatch=128, b1=None, b2=None, ln_eps=1e-5, out=None,
+                             ws: Optional[Workspace] = None, stream=None):
+    """M-FALCON candidates only (hstu_layer_forward_candidates): x_cand [B m, d_model] ->
+    y_cand, reading the history's f1 output from cache."""
+    d_model = x_cand.shape[1]
+    out = torch.empty_like(x_cand) if out is None else out
+    desc = _layer_call_desc(int(total_tokens), seq_offsets, max_seq_len, timestamps, d_model,
+                            _dtype_code(x_cand), num_heads=num_heads, d_qk=d_qk, d_v=d_v,
+                            mask=MASK_MFALCON, num_candidates=num_candidates,
+                            microbatch=microbatch, rab_pos=rab_pos, max_pos_dist=max_pos_dist,
+                            rab_time=rab_time, num_time_buckets=num_time_buckets, alpha=alpha,
+                            ln_eps=ln_eps)
+    need = lib().hstu_layer_candidates_workspace_size(ctypes.byref(desc))
+    ws = workspace(need, x_cand.device) if ws is None else ws.ensure(need)
+    _check(lib().hstu_layer_forward_candidates(ctypes.byref(desc), _ptr(x_cand), _ptr(w1),
+                                               _ptr(b1), _ptr(w2), _ptr(b2), _ptr(out),
+                                               _ptr(cache), ws.ptr, ws.nbytes,
+                                               _stream_ptr(stream)),
+           "hstu_layer_forward_candidates")
     return out
 
 

@@ -19,8 +19,8 @@ cudaError_t launch_attn_fwd_tc(int D, const CUtensorMap& tq, const CUtensorMap& 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);
 int gemm_tc_mn_tiles(int M, int N);
 cudaError_t launch_build_worklist(const int32_t* offsets, int B, int T, int max_len, int mask,
-                                  int m, int group, WorkItem* items, int32_t* count,
-                                  int32_t* hist, int max_cost, int32_t* status,
+                                  int m, int group, int cand_only, WorkItem* items,
+                                  int32_t* count, int32_t* hist, int max_cost, int32_t* status,
                                   cudaStream_t stream);
 cudaError_t launch_attn_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& tts,
@@ -74,6 +74,11 @@ cudaError_t launch_stochastic_length(const int32_t* off, int B, int T, int max_l
 cudaError_t launch_gather_rows(const void* src, int64_t src_stride, const int32_t* index,
                                const int32_t* count, int n, void* dst, int64_t dst_stride,
                                int64_t row_bytes, int num_sms, cudaStream_t stream);
+cudaError_t launch_candidate_rows(const int32_t* off, int B, int m, int32_t* idx, int32_t* status,
+                                  cudaStream_t stream);
+cudaError_t launch_scatter_rows(const void* src, int64_t src_stride, const int32_t* index, int n,
+                                void* dst, int64_t dst_stride, int64_t row_bytes, int num_sms,
+                                cudaStream_t stream);
 cudaError_t launch_colsum(const __nv_bfloat16* m, int64_t ld, int rows, int cols, float* out,
                           cudaStream_t stream);
 int attn_bwd_tc_ts_box();
@@ -226,10 +231,11 @@ AttnGeom make_geom(const void* ws, const WsLayout& w, const int64_t* ts, const f
 }
 
 cudaError_t build_list(const void* ws, const WsLayout& w, const int32_t* offsets, int B, int T,
-                       int max_len, int mask, int m, int group, cudaStream_t s) {
+                       int max_len, int mask, int m, int group, cudaStream_t s,
+                       int cand_only = 0) {
   uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(ws));
   return launch_build_worklist(offsets, B, T, max_len, mask, mask == HSTU_MASK_MFALCON ? m : 0,
-                               group,
+                               group, cand_only,
                                reinterpret_cast<WorkItem*>(base + w.items),
                                reinterpret_cast<int32_t*>(base + 4),
                                reinterpret_cast<int32_t*>(base + w.hist), max_cost(max_len),
@@ -250,7 +256,7 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
                                 int max_len, const AttnGeom& g, int B, int T, int D, int dtype,
                                 const void* q, int64_t ld_q, const void* k, int64_t ld_k,
                                 const void* v, int64_t ld_v, void* o, int64_t ld_o,
-                                cudaStream_t s) {
+                                cudaStream_t s, int cand_only = 0) {
   const bool tc = attn_uses_tc(D, dtype, q, ld_q, k, ld_k, v, ld_v, o, ld_o);
   // the paired kernel keeps the position table in shared memory (it fits for P up to about
   // 1100 next to its tiles: the shared-memory check below decides) and loads the timestamps
@@ -260,7 +266,7 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
                     (!use_time || aligned16(g.ts)) &&
                     attn_fwd_pair_smem(g.P, g.rab_pos != nullptr) <= 227 * 1024;
   const int group = pair ? 2 : 1;
-  if (build_list(ws, w, offsets, B, T, max_len, g.mask, g.num_candidates, group, s) !=
+  if (build_list(ws, w, offsets, B, T, max_len, g.mask, g.num_candidates, group, s, cand_only) !=
       cudaSuccess)
     return HSTU_ERR_CUDA;
   const int grid = max_items(T, B, group) * g.H;
@@ -552,10 +558,16 @@ size_t hstu_layer_workspace_size(const hstu_layer_desc_t* d) {
   return w.total_attn + align_up(T * n1 * es) + 2 * align_up(T * hv * es);
 }
 
-hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* d, int32_t stage,
-                                       const void* x, const void* w1, const float* b1,
-                                       const void* w2, const float* b2, void* y, void* ws,
-                                       size_t ws_bytes, hstu_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// One stage of the layer forward (see hstu_layer_forward_stage).  uvqk_ext, when set, takes the
+// place of the workspace's f1 output [T, 2H(d_qk+d_v)] (the M-FALCON cache of
+// hstu_layer_forward_cached).
+hstu_status_t layer_stage(const hstu_layer_desc_t* d, int32_t stage, const void* x,
+                          const void* w1, const float* b1, const void* w2, const float* b2,
+                          void* y, void* ws, size_t ws_bytes, hstu_stream_t stream,
+                          void* uvqk_ext) {
   if (d == nullptr) return HSTU_ERR_INVALID_ARG;
   if (stage < HSTU_STAGE_F1 || stage > HSTU_STAGE_NORM_GATE_F2) return HSTU_ERR_INVALID_ARG;
   hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
@@ -582,8 +594,8 @@ hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* d, int32_t stage
   const WsLayout w = attn_layout(T, d->num_seqs, d->max_seq_len);
   const size_t es = elem_size(d->dtype);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  uint8_t* uvqk = base + w.total_attn;
-  uint8_t* av = uvqk + align_up(static_cast<size_t>(T) * n1 * es);
+  uint8_t* uvqk = uvqk_ext != nullptr ? static_cast<uint8_t*>(uvqk_ext) : base + w.total_attn;
+  uint8_t* av = base + w.total_attn + align_up(static_cast<size_t>(T) * n1 * es);
   uint8_t* gbuf = av + align_up(static_cast<size_t>(T) * hv * es);
   int32_t* status = reinterpret_cast<int32_t*>(base);
   const uint8_t* u_ptr = uvqk;
@@ -609,6 +621,16 @@ hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* d, int32_t stage
   return gemm(d->dtype, 1, gbuf, hv, w2, d->d_model, T, d->d_model, hv, b2, x, d->d_model, y,
               d->d_model, status, s);
 }
+}  // namespace
+
+extern "C" {
+
+hstu_status_t hstu_layer_forward_stage(const hstu_layer_desc_t* d, int32_t stage,
+                                       const void* x, const void* w1, const float* b1,
+                                       const void* w2, const float* b2, void* y, void* ws,
+                                       size_t ws_bytes, hstu_stream_t stream) {
+  return layer_stage(d, stage, x, w1, b1, w2, b2, y, ws, ws_bytes, stream, nullptr);
+}
 
 hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* d, const void* x, const void* w1,
                                  const float* b1, const void* w2, const float* b2, void* y,
@@ -622,6 +644,116 @@ hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* d, const void* x, cons
     if (st != HSTU_OK) return st;
   }
   return HSTU_OK;
+}
+
+size_t hstu_layer_cache_bytes(const hstu_layer_desc_t* d) {
+  if (d == nullptr || d->total_tokens < 0 || d->num_heads < 1 || d->d_qk < 1 || d->d_v < 1)
+    return 0;
+  return static_cast<size_t>(d->total_tokens) * 2 * d->num_heads * (d->d_qk + d->d_v) *
+         elem_size(d->dtype);
+}
+
+hstu_status_t hstu_layer_forward_cached(const hstu_layer_desc_t* d, const void* x,
+                                        const void* w1, const float* b1, const void* w2,
+                                        const float* b2, void* y, void* cache, void* ws,
+                                        size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (d->num_seqs > 0 && d->total_tokens > 0 && (cache == nullptr || !aligned16(cache)))
+    return HSTU_ERR_INVALID_ARG;
+  if (x == nullptr || w1 == nullptr || w2 == nullptr || y == nullptr || x == y)
+    return d->num_seqs == 0 || d->total_tokens == 0 ? HSTU_OK : HSTU_ERR_INVALID_ARG;
+  for (int32_t stage = HSTU_STAGE_F1; stage <= HSTU_STAGE_NORM_GATE_F2; ++stage) {
+    const hstu_status_t st =
+        layer_stage(d, stage, x, w1, b1, w2, b2, y, ws, ws_bytes, stream, cache);
+    if (st != HSTU_OK) return st;
+  }
+  return HSTU_OK;
+}
+
+size_t hstu_layer_candidates_workspace_size(const hstu_layer_desc_t* d) {
+  if (d == nullptr || d->total_tokens < 0 || d->num_seqs < 0 || d->max_seq_len < 0 ||
+      d->num_heads < 1 || d->d_qk < 1 || d->d_v < 1 || d->num_candidates < 0)
+    return 0;
+  const WsLayout w = attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len);
+  const size_t es = elem_size(d->dtype);
+  const size_t bm = static_cast<size_t>(d->num_seqs) * d->num_candidates;
+  const size_t n1 = 2 * static_cast<size_t>(d->num_heads) * (d->d_qk + d->d_v);
+  const size_t hv = static_cast<size_t>(d->num_heads) * d->d_v;
+  // f1 output of the candidates, their row indices, the attention output [T, hv] (the candidate
+  // tiles' rows), and the candidates' AV, U and gated norm
+  return w.total_attn + align_up(bm * n1 * es) + align_up(bm * 4) +
+         align_up(static_cast<size_t>(d->total_tokens) * hv * es) + 3 * align_up(bm * hv * es);
+}
+
+hstu_status_t hstu_layer_forward_candidates(const hstu_layer_desc_t* d, const void* x_cand,
+                                            const void* w1, const float* b1, const void* w2,
+                                            const float* b2, void* y_cand, void* cache,
+                                            void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
+                                  d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
+                                  d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
+                                  d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
+  if (st != HSTU_OK) return st;
+  if (d->mask != HSTU_MASK_MFALCON || d->num_candidates < 1) return HSTU_ERR_INVALID_ARG;
+  if (d->d_model < 1 || !std::isfinite(d->ln_eps) || d->ln_eps < 0.f) return HSTU_ERR_INVALID_ARG;
+  const int H = d->num_heads, T = d->total_tokens, m = d->num_candidates, B = d->num_seqs;
+  const int hv = H * d->d_v, n1 = 2 * H * (d->d_qk + d->d_v), D = d->d_qk;
+  if (hv > 1024) return HSTU_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * m > T) return HSTU_ERR_INVALID_ARG;  // every sequence holds m
+  st = check_ws(ws, ws_bytes, hstu_layer_candidates_workspace_size(d));
+  if (st != HSTU_OK) return st;
+  if (B == 0 || T == 0) return HSTU_OK;
+  const void* ptrs[] = {x_cand, w1, w2, y_cand, cache};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  if (x_cand == y_cand) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout w = attn_layout(T, B, d->max_seq_len);
+  const size_t es = elem_size(d->dtype);
+  const int bm = B * m;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(base);
+  uint8_t* zc = base + w.total_attn;
+  int32_t* idx = reinterpret_cast<int32_t*>(zc + align_up(static_cast<size_t>(bm) * n1 * es));
+  uint8_t* av = reinterpret_cast<uint8_t*>(idx) + align_up(static_cast<size_t>(bm) * 4);
+  uint8_t* avc = av + align_up(static_cast<size_t>(T) * hv * es);
+  uint8_t* uc = avc + align_up(static_cast<size_t>(bm) * hv * es);
+  uint8_t* gc = uc + align_up(static_cast<size_t>(bm) * hv * es);
+  uint8_t* ca = static_cast<uint8_t*>(cache);
+  const int nsm = num_sms_current();
+  // candidate rows of the jagged layout, then the candidates' f1 output into their cache rows
+  cudaError_t e = launch_candidate_rows(d->seq_offsets, B, m, idx, status, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = gemm(d->dtype, 0, x_cand, d->d_model, w1, n1, bm, n1, d->d_model, b1, nullptr, 0, zc, n1,
+            status, s);
+  if (st != HSTU_OK) return st;
+  e = launch_scatter_rows(zc, static_cast<int64_t>(n1) * es, idx, bm, ca,
+                          static_cast<int64_t>(n1) * es, static_cast<int64_t>(n1) * es, nsm, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // attention of the query tiles that hold candidates: the history's K / V come from the cache
+  const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                               d->num_time_buckets, H, T, d->mask, m, d->alpha);
+  const uint8_t* u_ptr = ca;
+  const uint8_t* v_ptr = ca + static_cast<size_t>(hv) * es;
+  const uint8_t* q_ptr = ca + static_cast<size_t>(2 * hv) * es;
+  const uint8_t* k_ptr = q_ptr + static_cast<size_t>(H) * d->d_qk * es;
+  st = attn_forward_core(ws, w, d->seq_offsets, d->max_seq_len, g, B, T, D, d->dtype, q_ptr, n1,
+                         k_ptr, n1, v_ptr, n1, av, hv, s, 1);
+  if (st != HSTU_OK) return st;
+  // the candidates' AV and U rows, Norm(AV) ⊙ U, f2 + residual
+  if ((e = launch_gather_rows(av, static_cast<int64_t>(hv) * es, idx, nullptr, bm, avc,
+                              static_cast<int64_t>(hv) * es, static_cast<int64_t>(hv) * es, nsm,
+                              s)) != cudaSuccess ||
+      (e = launch_gather_rows(u_ptr, static_cast<int64_t>(n1) * es, idx, nullptr, bm, uc,
+                              static_cast<int64_t>(hv) * es, static_cast<int64_t>(hv) * es, nsm,
+                              s)) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = launch_ln_gate(d->dtype == HSTU_BF16 ? 0 : 1, avc, hv, uc, hv, d->ln_gamma,
+                          d->ln_beta, d->ln_eps, gc, hv, bm, hv, s)) != cudaSuccess)
+    return cuda_fail(e);
+  return gemm(d->dtype, 1, gc, hv, w2, d->d_model, bm, d->d_model, hv, b2, x_cand, d->d_model,
+              y_cand, d->d_model, status, s);
 }
 
 size_t hstu_layer_backward_workspace_size(const hstu_layer_desc_t* d) {

@@ -17,6 +17,8 @@ namespace hstu {
 // `group` consecutive 128-row query tiles of one sequence (1 or 2); items are placed in
 // decreasing order of cost (KV tiles visited, summed over the group) by a counting sort, so the
 // longest items start first.  hist holds max_cost + 1 counters (global workspace).
+// cand_only (M-FALCON candidates-only calls): items whose tiles hold no candidate row are left
+// out, and every sequence must have at least m tokens.
 __device__ __forceinline__ int item_cost(int qt0, int group, int L, int n) {
   int cost = 0;
   for (int a = 0; a < group; ++a) {
@@ -31,7 +33,7 @@ __device__ __forceinline__ int item_cost(int qt0, int group, int L, int n) {
 constexpr int kWorklistSmemBins = 4096;
 
 __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B, int T,
-                                      int max_len, int mask, int m, int group,
+                                      int max_len, int mask, int m, int group, int cand_only,
                                       WorkItem* __restrict__ items, int32_t* __restrict__ count,
                                       int32_t* __restrict__ hist_global, int max_cost,
                                       int32_t* status) {
@@ -46,7 +48,7 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
   if (threadIdx.x == 0 && (offsets[0] != 0 || offsets[B] != T)) bad = 1;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int L = offsets[b + 1] - offsets[b];
-    if (L < 0 || L > max_len) bad = 1;
+    if (L < 0 || L > max_len || (cand_only && L < m)) bad = 1;
   }
   __syncthreads();
   if (bad) {
@@ -61,7 +63,7 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
     const int n = hist_len(L, mask, m);
     const int nt = (L + kTileRows - 1) / kTileRows;
     for (int qt = lane * group; qt < nt; qt += 32 * group)
-      atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
+      if (!cand_only || (qt + group) * kTileRows > n) atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {  // exclusive scan in decreasing cost
@@ -79,6 +81,7 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
     const int n = hist_len(L, mask, m);
     const int nt = (L + kTileRows - 1) / kTileRows;
     for (int qt = lane * group; qt < nt; qt += 32 * group) {
+      if (cand_only && (qt + group) * kTileRows <= n) continue;
       const int pos = atomicAdd(&hist[item_cost(qt, group, L, n)], 1);
       WorkItem it;
       it.seq = b;
@@ -91,10 +94,10 @@ __global__ void build_worklist_kernel(const int32_t* __restrict__ offsets, int B
 }
 
 cudaError_t launch_build_worklist(const int32_t* offsets, int B, int T, int max_len, int mask,
-                                  int m, int group, WorkItem* items, int32_t* count,
-                                  int32_t* hist, int max_cost, int32_t* status,
+                                  int m, int group, int cand_only, WorkItem* items,
+                                  int32_t* count, int32_t* hist, int max_cost, int32_t* status,
                                   cudaStream_t stream) {
-  build_worklist_kernel<<<1, 1024, 0, stream>>>(offsets, B, T, max_len, mask, m, group, items,
+  build_worklist_kernel<<<1, 1024, 0, stream>>>(offsets, B, T, max_len, mask, m, group, cand_only, items,
                                                 count, hist, max_cost, status);
   return cudaGetLastError();
 }

@@ -175,7 +175,77 @@ __global__ void gather_rows_kernel(const uint8_t* __restrict__ src, int64_t src_
   }
 }
 
+// dst row index[r] = src row r for r < n; V-byte vectors.
+template <typename Vec>
+__global__ void scatter_rows_kernel(const uint8_t* __restrict__ src, int64_t src_stride,
+                                    const int32_t* __restrict__ index, int n,
+                                    uint8_t* __restrict__ dst, int64_t dst_stride,
+                                    int64_t vecs_per_row) {
+  const int64_t total = static_cast<int64_t>(n) * vecs_per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vecs_per_row, v = i % vecs_per_row;
+    const int64_t to = index[r];
+    reinterpret_cast<Vec*>(dst + to * dst_stride)[v] =
+        reinterpret_cast<const Vec*>(src + r * src_stride)[v];
+  }
+}
+
+// M-FALCON candidate rows: idx[b m + c] = offsets[b + 1] - m + c, the c-th of the last m tokens of
+// sequence b.  A sequence shorter than m sets the device-check status (its rows point at row 0).
+__global__ void candidate_rows_kernel(const int32_t* __restrict__ off, int B, int m,
+                                      int32_t* __restrict__ idx, int32_t* status) {
+  const int64_t total = static_cast<int64_t>(B) * m;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int b = static_cast<int>(i / m), c = static_cast<int>(i % m);
+    const int s = off[b], e = off[b + 1];
+    if (e - s < m) {
+      atomicExch(status, kStatusDeviceCheck);
+      idx[i] = 0;
+    } else {
+      idx[i] = e - m + c;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_candidate_rows(const int32_t* off, int B, int m, int32_t* idx, int32_t* status,
+                                  cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(B) * m;
+  if (total <= 0) return cudaSuccess;
+  const int64_t blocks = (total + 255) / 256;
+  candidate_rows_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(
+      off, B, m, idx, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const void* src, int64_t src_stride, const int32_t* index, int n,
+                                void* dst, int64_t dst_stride, int64_t row_bytes, int num_sms,
+                                cudaStream_t stream) {
+  if (n <= 0 || row_bytes <= 0) return cudaSuccess;
+  const uintptr_t align = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) |
+                          static_cast<uintptr_t>(src_stride) |
+                          static_cast<uintptr_t>(dst_stride) | static_cast<uintptr_t>(row_bytes);
+  const int vb = (align % 16 == 0) ? 16 : (align % 8 == 0) ? 8 : 4;
+  const int64_t vecs = row_bytes / vb;
+  const int64_t total = static_cast<int64_t>(n) * vecs;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > static_cast<int64_t>(num_sms) * 16) blocks = static_cast<int64_t>(num_sms) * 16;
+  const auto* s = static_cast<const uint8_t*>(src);
+  auto* d = static_cast<uint8_t*>(dst);
+  if (vb == 16)
+    scatter_rows_kernel<uint4><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        s, src_stride, index, n, d, dst_stride, vecs);
+  else if (vb == 8)
+    scatter_rows_kernel<uint2><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        s, src_stride, index, n, d, dst_stride, vecs);
+  else
+    scatter_rows_kernel<uint32_t><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        s, src_stride, index, n, d, dst_stride, vecs);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_stochastic_length(const int32_t* off, int B, int T, int max_len, int sub_len,
                                      double n_alpha, const float* u, const uint32_t* keys,

@@ -176,6 +176,34 @@ hstu_status_t hstu_layer_forward(const hstu_layer_desc_t* desc, const void* x, c
                                  const float* b1, const void* w2, const float* b2, void* y,
                                  void* ws, size_t ws_bytes, hstu_stream_t stream);
 
+/* ---- M-FALCON cross-request cache ("HSTU：Scaling Law 的首次探索" §7.1.5: the history's K/V are
+ * computed once and reused for every later microbatch and request; only candidate rows are new).
+ * The cache of one layer is that layer's f1 output [U | V | Q | K] of every token of the jagged
+ * batch, [T, 2H(d_qk+d_v)] in desc->dtype, caller-owned (hstu_layer_cache_bytes).
+ *   hstu_layer_forward_cached: hstu_layer_forward that keeps its f1 output in cache (prefill).
+ *   hstu_layer_forward_candidates: the same layer for the candidates only.  desc describes the
+ *     same batch and history as the prefill (same seq_offsets, the M-FALCON mask, m =
+ *     num_candidates >= 1 candidates at the end of every sequence, each sequence at least m
+ *     long, else the status word reports HSTU_ERR_DEVICE_CHECK); timestamps covers all T tokens
+ *     (the candidates' included).  x_cand / y_cand: [B m, d_model], the candidates of sequence 0,
+ *     then of sequence 1, ...  The history rows of cache are read, its candidate rows
+ *     overwritten; every candidate row of y_cand equals that row of a full
+ *     hstu_layer_forward over the history followed by these candidates (history rows never
+ *     depend on candidates, so a prefill with other candidates serves as well).  Work: f1 and
+ *     f2 on B m rows and the attention of the query tiles that hold candidates.
+ * For a stack, each layer has its own cache, and layer l's candidates call takes layer l-1's
+ * y_cand as x_cand. */
+size_t hstu_layer_cache_bytes(const hstu_layer_desc_t* desc);
+hstu_status_t hstu_layer_forward_cached(const hstu_layer_desc_t* desc, const void* x,
+                                        const void* w1, const float* b1, const void* w2,
+                                        const float* b2, void* y, void* cache, void* ws,
+                                        size_t ws_bytes, hstu_stream_t stream);
+size_t hstu_layer_candidates_workspace_size(const hstu_layer_desc_t* desc);
+hstu_status_t hstu_layer_forward_candidates(const hstu_layer_desc_t* desc, const void* x_cand,
+                                            const void* w1, const float* b1, const void* w2,
+                                            const float* b2, void* y_cand, void* cache,
+                                            void* ws, size_t ws_bytes, hstu_stream_t stream);
+
 /* Bytes of workspace hstu_layer_backward needs: the attention backward's workspace, then the
  * saved forward activations (f1 pre-activation and output [T, 2H(d_qk+d_v)] each, the attention
  * output and the gated norm [T, H d_v] each) and the gradient activations (dG and dAV
