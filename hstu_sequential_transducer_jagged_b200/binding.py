@@ -33,7 +33,7 @@ EXPORTED = [
     "hstu_debug_bias_index", "hstu_layer_backward_workspace_size", "hstu_layer_backward",
     "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
     "hstu_layer_cache_bytes", "hstu_layer_forward_cached", "hstu_layer_candidates_workspace_size",
-    "hstu_layer_forward_candidates",
+    "hstu_layer_forward_candidates", "hstu_attention_backward_typed",
 ]
 
 # Rules of hstu_debug_bias_index (hstu_bias_rule_t)
@@ -62,7 +62,8 @@ class AttnDesc(ctypes.Structure):
         ("mfalcon_microbatch", ctypes.c_int32), ("rab_pos", ctypes.c_void_p),
         ("max_pos_dist", ctypes.c_int32), ("rab_time", ctypes.c_void_p),
         ("num_time_buckets", ctypes.c_int32), ("alpha", ctypes.c_float),
-        ("dtype", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("token_types", ctypes.c_void_p),
+        ("rab_type", ctypes.c_void_p), ("num_types", ctypes.c_int32),
     ]
 
 
@@ -77,7 +78,8 @@ class LayerDesc(ctypes.Structure):
         ("max_pos_dist", ctypes.c_int32), ("rab_time", ctypes.c_void_p),
         ("num_time_buckets", ctypes.c_int32), ("alpha", ctypes.c_float),
         ("ln_eps", ctypes.c_float), ("ln_gamma", ctypes.c_void_p), ("ln_beta", ctypes.c_void_p),
-        ("dtype", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("token_types", ctypes.c_void_p),
+        ("rab_type", ctypes.c_void_p), ("num_types", ctypes.c_int32),
     ]
 
 
@@ -93,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hstu_attention_forward": (i32, [adp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_attention_backward_workspace_size": (sz, [adp]),
         "hstu_attention_backward": (i32, [adp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "hstu_attention_backward_typed": (i32, [adp] + [vp] * 11 + [sz, vp]),
         "hstu_layer_workspace_size": (sz, [ldp]),
         "hstu_layer_forward": (i32, [ldp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "hstu_layer_forward_stage": (i32, [ldp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -199,7 +202,7 @@ def threading_id() -> int:
 def attn_desc(*, seq_offsets, total_tokens, max_seq_len, timestamps, num_heads, d_qk, d_v,
               ld_q, ld_k, ld_v, ld_o, mask=MASK_CAUSAL, num_candidates=0, microbatch=1,
               rab_pos=None, max_pos_dist=0, rab_time=None, num_time_buckets=1, alpha=1.0,
-              dtype=DTYPE_BF16) -> AttnDesc:
+              dtype=DTYPE_BF16, token_types=None, rab_type=None, num_types=0) -> AttnDesc:
     return AttnDesc(
         num_seqs=seq_offsets.numel() - 1, total_tokens=int(total_tokens),
         max_seq_len=int(max_seq_len), seq_offsets=seq_offsets.data_ptr(),
@@ -208,13 +211,17 @@ def attn_desc(*, seq_offsets, total_tokens, max_seq_len, timestamps, num_heads, 
         num_candidates=num_candidates, mfalcon_microbatch=max(1, int(microbatch)),
         rab_pos=None if rab_pos is None else rab_pos.data_ptr(), max_pos_dist=max_pos_dist,
         rab_time=None if rab_time is None else rab_time.data_ptr(),
-        num_time_buckets=num_time_buckets, alpha=alpha, dtype=dtype)
+        num_time_buckets=num_time_buckets, alpha=alpha, dtype=dtype,
+        token_types=None if token_types is None else token_types.data_ptr(),
+        rab_type=None if rab_type is None else rab_type.data_ptr(),
+        num_types=int(num_types) if rab_type is not None else 0)
 
 
 def attention_forward(q, k, v, seq_offsets, max_seq_len, timestamps=None, rab_pos=None,
                       rab_time=None, *, num_heads, max_pos_dist=0, num_time_buckets=1,
                       alpha=1.0, mask=MASK_CAUSAL, num_candidates=0, microbatch=128, out=None,
-                      ws: Optional[Workspace] = None, stream=None):
+                      ws: Optional[Workspace] = None, stream=None, token_types=None,
+                      rab_type=None, num_types=0):
     """O = hstu_attention_forward(...) for [T, H*d] views q, k, v (row strides taken from them)."""
     T = q.shape[0]
     d = q.shape[1] // num_heads if q.dim() == 2 else q.shape[-1]
@@ -226,7 +233,8 @@ def attention_forward(q, k, v, seq_offsets, max_seq_len, timestamps=None, rab_po
                      ld_q=q.stride(0), ld_k=k.stride(0), ld_v=v.stride(0), ld_o=out.stride(0),
                      mask=mask, num_candidates=num_candidates, microbatch=microbatch,
                      rab_pos=rab_pos, max_pos_dist=max_pos_dist, rab_time=rab_time,
-                     num_time_buckets=num_time_buckets, alpha=alpha, dtype=_dtype_code(q))
+                     num_time_buckets=num_time_buckets, alpha=alpha, dtype=_dtype_code(q),
+                     token_types=token_types, rab_type=rab_type, num_types=num_types)
     need = lib().hstu_attention_workspace_size(ctypes.byref(desc))
     ws = workspace(need, q.device) if ws is None else ws.ensure(need)
     _check(lib().hstu_attention_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
@@ -265,7 +273,10 @@ def attention_forward_static_ws(q, k, v, seq_offsets, max_seq_len, timestamps=No
 def attention_backward(q, k, v, d_o, seq_offsets, max_seq_len, timestamps=None, rab_pos=None,
                        rab_time=None, *, num_heads, max_pos_dist=0, num_time_buckets=1,
                        alpha=1.0, mask=MASK_CAUSAL, num_candidates=0, microbatch=128,
-                       ws: Optional[Workspace] = None, stream=None):
+                       ws: Optional[Workspace] = None, stream=None, token_types=None,
+                       rab_type=None, num_types=0):
+    """(dq, dk, dv, d_rab_pos, d_rab_time) of hstu_attention_backward; with the token-type term
+    (rab_type given) hstu_attention_backward_typed, and d_rab_type appended."""
     T = q.shape[0]
     d = q.shape[1] // num_heads
     dq = torch.empty_like(q)
@@ -280,9 +291,17 @@ def attention_backward(q, k, v, d_o, seq_offsets, max_seq_len, timestamps=None, 
                      ld_q=q.stride(0), ld_k=k.stride(0), ld_v=v.stride(0), ld_o=d_o.stride(0),
                      mask=mask, num_candidates=num_candidates, microbatch=microbatch,
                      rab_pos=rab_pos, max_pos_dist=max_pos_dist, rab_time=rab_time,
-                     num_time_buckets=num_time_buckets, alpha=alpha, dtype=_dtype_code(q))
+                     num_time_buckets=num_time_buckets, alpha=alpha, dtype=_dtype_code(q),
+                     token_types=token_types, rab_type=rab_type, num_types=num_types)
     need = lib().hstu_attention_backward_workspace_size(ctypes.byref(desc))
     ws = workspace(need, q.device) if ws is None else ws.ensure(need)
+    if rab_type is not None:
+        d_type = torch.empty(num_types * num_types, dtype=torch.float32, device=q.device)
+        _check(lib().hstu_attention_backward_typed(
+            ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(d_o), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(d_pos), _ptr(d_time), _ptr(d_type), ws.ptr, ws.nbytes,
+            _stream_ptr(stream)), "hstu_attention_backward_typed")
+        return dq, dk, dv, d_pos, d_time, d_type
     _check(lib().hstu_attention_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(d_o),
                                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(d_pos), _ptr(d_time),
                                          ws.ptr, ws.nbytes, _stream_ptr(stream)),
@@ -293,7 +312,8 @@ def attention_backward(q, k, v, d_o, seq_offsets, max_seq_len, timestamps=None, 
 def layer_desc(*, seq_offsets, total_tokens, max_seq_len, timestamps, d_model, num_heads, d_qk,
                d_v, mask=MASK_CAUSAL, num_candidates=0, microbatch=1, rab_pos=None,
                max_pos_dist=0, rab_time=None, num_time_buckets=1, alpha=1.0, ln_eps=1e-5,
-               ln_gamma=None, ln_beta=None, dtype=DTYPE_BF16) -> LayerDesc:
+               ln_gamma=None, ln_beta=None, dtype=DTYPE_BF16, token_types=None, rab_type=None,
+               num_types=0) -> LayerDesc:
     return LayerDesc(
         num_seqs=seq_offsets.numel() - 1, total_tokens=int(total_tokens),
         max_seq_len=int(max_seq_len), seq_offsets=seq_offsets.data_ptr(),
@@ -304,14 +324,18 @@ def layer_desc(*, seq_offsets, total_tokens, max_seq_len, timestamps, d_model, n
         rab_time=None if rab_time is None else rab_time.data_ptr(),
         num_time_buckets=num_time_buckets, alpha=alpha, ln_eps=ln_eps,
         ln_gamma=None if ln_gamma is None else ln_gamma.data_ptr(),
-        ln_beta=None if ln_beta is None else ln_beta.data_ptr(), dtype=dtype)
+        ln_beta=None if ln_beta is None else ln_beta.data_ptr(), dtype=dtype,
+        token_types=None if token_types is None else token_types.data_ptr(),
+        rab_type=None if rab_type is None else rab_type.data_ptr(),
+        num_types=int(num_types) if rab_type is not None else 0)
 
 
 def layer_forward(x, w1, w2, seq_offsets, max_seq_len, timestamps=None, rab_pos=None,
                   rab_time=None, *, num_heads, d_qk, d_v, max_pos_dist=0, num_time_buckets=1,
                   alpha=1.0, mask=MASK_CAUSAL, num_candidates=0, microbatch=128, b1=None,
                   b2=None, ln_eps=1e-5, ln_gamma=None, ln_beta=None, out=None,
-                  ws: Optional[Workspace] = None, stream=None):
+                  ws: Optional[Workspace] = None, stream=None, token_types=None, rab_type=None,
+                  num_types=0):
     T, d_model = x.shape
     if out is None:
         out = torch.empty_like(x)
@@ -320,7 +344,8 @@ def layer_forward(x, w1, w2, seq_offsets, max_seq_len, timestamps=None, rab_pos=
                       d_v=d_v, mask=mask, num_candidates=num_candidates, microbatch=microbatch,
                       rab_pos=rab_pos, max_pos_dist=max_pos_dist, rab_time=rab_time,
                       num_time_buckets=num_time_buckets, alpha=alpha, ln_eps=ln_eps,
-                      ln_gamma=ln_gamma, ln_beta=ln_beta, dtype=_dtype_code(x))
+                      ln_gamma=ln_gamma, ln_beta=ln_beta, dtype=_dtype_code(x),
+                      token_types=token_types, rab_type=rab_type, num_types=num_types)
     need = lib().hstu_layer_workspace_size(ctypes.byref(desc))
     ws = workspace(need, x.device) if ws is None else ws.ensure(need)
     _check(lib().hstu_layer_forward(ctypes.byref(desc), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2),

@@ -227,7 +227,25 @@ AttnGeom make_geom(const void* ws, const WsLayout& w, const int64_t* ts, const f
   g.num_candidates = (mask == HSTU_MASK_MFALCON) ? m : 0;
   g.alpha = alpha;
   g.status = reinterpret_cast<int32_t*>(base);
+  g.types = nullptr;
+  g.rab_type = nullptr;
+  g.NT = 0;
+  g.d_type = nullptr;
   return g;
+}
+
+// The token-type term's arguments (rab_type NULL: off).
+hstu_status_t check_types(const int32_t* types, const float* rab_type, int NT, int T) {
+  if (rab_type == nullptr) return HSTU_OK;
+  if (NT < 1 || NT > 64 || (T > 0 && types == nullptr)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+void set_types(AttnGeom* g, const int32_t* types, const float* rab_type, int NT) {
+  if (rab_type == nullptr) return;
+  g->types = types;
+  g->rab_type = rab_type;
+  g->NT = NT;
 }
 
 cudaError_t build_list(const void* ws, const WsLayout& w, const int32_t* offsets, int B, int T,
@@ -262,7 +280,8 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
   // 1100 next to its tiles: the shared-memory check below decides) and loads the timestamps
   // with TMA (16-byte aligned base)
   const bool use_time = g.ts != nullptr && g.rab_time != nullptr;
-  const bool pair = tc && D == 64 && (g.rab_pos == nullptr || g.P <= 2048) &&
+  const bool pair = tc && D == 64 && g.rab_type == nullptr &&
+                    (g.rab_pos == nullptr || g.P <= 2048) &&
                     (!use_time || aligned16(g.ts)) &&
                     attn_fwd_pair_smem(g.P, g.rab_pos != nullptr) <= 227 * 1024;
   const int group = pair ? 2 : 1;
@@ -426,6 +445,9 @@ hstu_attn_desc_t layer_attn_desc(const hstu_layer_desc_t* d) {
   a.num_time_buckets = d->num_time_buckets;
   a.alpha = d->alpha;
   a.dtype = d->dtype;
+  a.token_types = d->token_types;
+  a.rab_type = d->rab_type;
+  a.num_types = d->num_types;
   return a;
 }
 
@@ -456,6 +478,8 @@ hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* d, const void* q, c
                                   d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
                                   d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
   if (st != HSTU_OK) return st;
+  st = check_types(d->token_types, d->rab_type, d->num_types, d->total_tokens);
+  if (st != HSTU_OK) return st;
   const int D = d->d_qk;
   const int64_t cols = static_cast<int64_t>(d->num_heads) * D;
   if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
@@ -466,9 +490,10 @@ hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* d, const void* q, c
   if (d->num_seqs == 0 || d->total_tokens == 0) return HSTU_OK;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return HSTU_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
-                               d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
-                               d->num_candidates, d->alpha);
+  AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                         d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
+                         d->num_candidates, d->alpha);
+  set_types(&g, d->token_types, d->rab_type, d->num_types);
   return attn_forward_core(ws, w, d->seq_offsets, d->max_seq_len, g, d->num_seqs,
                            d->total_tokens, D, d->dtype, q, d->ld_q, k, d->ld_k, v, d->ld_v, o,
                            d->ld_o, s);
@@ -478,7 +503,23 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
                                       const void* v, const void* d_o, void* dq, void* dk,
                                       void* dv, float* d_rab_pos, float* d_rab_time, void* ws,
                                       size_t ws_bytes, hstu_stream_t stream) {
+  if (d == nullptr || d->rab_type != nullptr) return HSTU_ERR_INVALID_ARG;
+  return hstu_attention_backward_typed(d, q, k, v, d_o, dq, dk, dv, d_rab_pos, d_rab_time,
+                                       nullptr, ws, ws_bytes, stream);
+}
+
+hstu_status_t hstu_attention_backward_typed(const hstu_attn_desc_t* d, const void* q,
+                                            const void* k, const void* v, const void* d_o,
+                                            void* dq, void* dk, void* dv, float* d_rab_pos,
+                                            float* d_rab_time, float* d_rab_type, void* ws,
+                                            size_t ws_bytes, hstu_stream_t stream) {
   if (d == nullptr) return HSTU_ERR_INVALID_ARG;
+  {
+    const hstu_status_t tst = check_types(d->token_types, d->rab_type, d->num_types,
+                                          d->total_tokens);
+    if (tst != HSTU_OK) return tst;
+    if (d->rab_type != nullptr && d_rab_type == nullptr) return HSTU_ERR_INVALID_ARG;
+  }
   hstu_status_t st = check_common(d->num_seqs, d->total_tokens, d->max_seq_len, d->seq_offsets,
                                   d->num_heads, d->d_qk, d->d_v, d->mask, d->num_candidates,
                                   d->mfalcon_microbatch, d->rab_pos, d->max_pos_dist,
@@ -503,6 +544,10 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
   if (d_rab_time != nullptr && d->rab_time != nullptr &&
       cudaMemsetAsync(d_rab_time, 0, sizeof(float) * d->num_time_buckets, s) != cudaSuccess)
     return HSTU_ERR_CUDA;
+  if (d->rab_type != nullptr &&
+      cudaMemsetAsync(d_rab_type, 0, sizeof(float) * d->num_types * d->num_types, s) !=
+          cudaSuccess)
+    return HSTU_ERR_CUDA;
   if (d->num_seqs == 0 || d->total_tokens == 0) return HSTU_OK;
   if (q == nullptr || k == nullptr || v == nullptr || d_o == nullptr || dq == nullptr ||
       dk == nullptr || dv == nullptr)
@@ -510,15 +555,17 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* d, const void* q, 
   if (build_list(ws, w, d->seq_offsets, d->num_seqs, d->total_tokens, d->max_seq_len, d->mask,
                  d->num_candidates, 1, s) != cudaSuccess)
     return HSTU_ERR_CUDA;
-  const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
-                               d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
-                               d->num_candidates, d->alpha);
+  AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                         d->num_time_buckets, d->num_heads, d->total_tokens, d->mask,
+                         d->num_candidates, d->alpha);
+  set_types(&g, d->token_types, d->rab_type, d->num_types);
+  if (d->rab_type != nullptr) g.d_type = d_rab_type;
   const int grid = max_items(d->total_tokens, d->num_seqs) * d->num_heads;
   // Head width 64 in bf16 with 16-byte aligned rows runs on the tensor cores (bias-gradient bins
   // and table copies in shared memory); every other shape on CUDA cores.
   const bool use_time = d->timestamps != nullptr && d->rab_time != nullptr;
-  const bool tc = D == 64 && attn_uses_tc(D, d->dtype, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o,
-                                          d->ld_o) &&
+  const bool tc = D == 64 && d->rab_type == nullptr &&
+                  attn_uses_tc(D, d->dtype, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o, d->ld_o) &&
                   aligned16(dq) && aligned16(dk) && aligned16(dv) && (!use_time || aligned16(d->timestamps)) &&
                   attn_bwd_tc_smem(d->rab_pos ? d->max_pos_dist : 0,
                                    d->rab_time ? d->num_time_buckets : 0) <= 227 * 1024;
@@ -576,6 +623,8 @@ hstu_status_t layer_stage(const hstu_layer_desc_t* d, int32_t stage, const void*
                                   d->rab_time, d->num_time_buckets, d->alpha, d->dtype);
   if (st != HSTU_OK) return st;
   if (d->d_model < 1 || !std::isfinite(d->ln_eps) || d->ln_eps < 0.f) return HSTU_ERR_INVALID_ARG;
+  st = check_types(d->token_types, d->rab_type, d->num_types, d->total_tokens);
+  if (st != HSTU_OK) return st;
   const int H = d->num_heads, D = d->d_qk, T = d->total_tokens;
   const int hv = H * d->d_v;
   const int n1 = 2 * H * (d->d_qk + d->d_v);
@@ -609,8 +658,9 @@ hstu_status_t layer_stage(const hstu_layer_desc_t* d, int32_t stage, const void*
                 status, s);
   }
   if (stage == HSTU_STAGE_ATTENTION) {
-    const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
-                                 d->num_time_buckets, H, T, d->mask, d->num_candidates, d->alpha);
+    AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                           d->num_time_buckets, H, T, d->mask, d->num_candidates, d->alpha);
+    set_types(&g, d->token_types, d->rab_type, d->num_types);
     return attn_forward_core(ws, w, d->seq_offsets, d->max_seq_len, g, d->num_seqs, T, D,
                              d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av, hv, s);
   }
@@ -732,8 +782,11 @@ hstu_status_t hstu_layer_forward_candidates(const hstu_layer_desc_t* d, const vo
                           static_cast<int64_t>(n1) * es, static_cast<int64_t>(n1) * es, nsm, s);
   if (e != cudaSuccess) return cuda_fail(e);
   // attention of the query tiles that hold candidates: the history's K / V come from the cache
-  const AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
-                               d->num_time_buckets, H, T, d->mask, m, d->alpha);
+  AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                         d->num_time_buckets, H, T, d->mask, m, d->alpha);
+  st = check_types(d->token_types, d->rab_type, d->num_types, T);
+  if (st != HSTU_OK) return st;
+  set_types(&g, d->token_types, d->rab_type, d->num_types);
   const uint8_t* u_ptr = ca;
   const uint8_t* v_ptr = ca + static_cast<size_t>(hv) * es;
   const uint8_t* q_ptr = ca + static_cast<size_t>(2 * hv) * es;
@@ -782,7 +835,8 @@ hstu_status_t hstu_layer_backward(const hstu_layer_desc_t* d, const void* x, con
   const int n1 = 2 * H * (d->d_qk + d->d_v);
   // tensor-core GEMMs and 16-byte vectors throughout: bf16, widths multiples of 8, LayerNorm
   // rows of 128 .. 1024 features held in one warp
-  if (d->dtype != HSTU_BF16 || dm % 8 != 0 || (hv != 128 && hv != 256 && hv != 512 && hv != 1024))
+  if (d->dtype != HSTU_BF16 || dm % 8 != 0 || (hv != 128 && hv != 256 && hv != 512 && hv != 1024) ||
+      d->rab_type != nullptr)
     return HSTU_ERR_UNSUPPORTED;
   const hstu_attn_desc_t ad = layer_attn_desc(d);
   const LayerBwdLayout L = layer_bwd_layout(d, ad);

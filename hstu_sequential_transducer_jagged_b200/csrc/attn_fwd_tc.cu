@@ -72,7 +72,8 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p
                                            int i, int pi, int n, int P, const float* pos_tab,
                                            const float* time_tab, bool use_time,
                                            const long long* ts_tile, long long ti, int NB,
-                                           bool row_valid) {
+                                           bool row_valid, const int32_t* types_seq,
+                                           const float* type_row, int L) {
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float pv[2];
@@ -91,6 +92,8 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[32], uint32_t (&p
           bias += pos_tab[pos_index_direct(pi, pj, P)];
         }
         if (use_time) bias += time_tab[time_bucket64(ti - ts_tile[c - (c_base & ~127)], NB)];
+        // token-type term: type_row = rab_type + type_i * NT (keys past the sequence are masked)
+        if (type_row != nullptr && j < L) bias += type_row[__ldg(types_seq + j)];
         h = fmaf(half_alpha, acc, 0.5f * bias);
       }
       float p = fmaf(h, tanh_fast(h), h);
@@ -287,6 +290,9 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float half_alpha = 0.5f * g.alpha;
     const float* time_tab = sm.rab_time;
+    const int32_t* types_seq = g.rab_type != nullptr ? g.types + it.row0 : nullptr;
+    const float* type_row =
+        g.rab_type != nullptr ? g.rab_type + (row_valid ? types_seq[i] : 0) * g.NT : nullptr;
     bool ok = true;
     for (int t = 0; t < nkv; ++t) {
       const int st = t % kStages;
@@ -304,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
       int mode = 2;
       float half_bias = 0.f;
       if (full_vis) {
-        bool uni = true;
+        bool uni = type_row == nullptr;  // the token-type term varies along the row
         float bias = 0.f;
         if (pos_tab != nullptr) {
           const int dmin = pi - last;  // smallest position difference in the segment
@@ -330,13 +336,13 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
         const int cb = c0l + ch * 32;
         if (mode == 0)
           silu_chunk<D, 0>(s, pk, half_alpha, half_bias, cb, i, pi, n, g.P, pos_tab, time_tab,
-                           use_time, ts_tile, ti, g.NB, row_valid);
+                           use_time, ts_tile, ti, g.NB, row_valid, types_seq, type_row, L);
         else if (mode == 1)
           silu_chunk<D, 1>(s, pk, half_alpha, half_bias, cb, i, pi, n, g.P, pos_tab, time_tab,
-                           use_time, ts_tile, ti, g.NB, row_valid);
+                           use_time, ts_tile, ti, g.NB, row_valid, types_seq, type_row, L);
         else
           silu_chunk<D, 2>(s, pk, half_alpha, half_bias, cb, i, pi, n, g.P, pos_tab, time_tab,
-                           use_time, ts_tile, ti, g.NB, row_valid);
+                           use_time, ts_tile, ti, g.NB, row_valid, types_seq, type_row, L);
         tmem_st16(lane_addr + kColP + ch * 16, pk);
       }
       tmem_wait_st();

@@ -35,6 +35,11 @@ struct AttnGeom {
   int32_t num_candidates;
   float alpha;
   int32_t* status;
+  // token-type term rab_type[type_i * NT + type_j] (types [T] in [0, NT)), or nullptr
+  const int32_t* types;
+  const float* rab_type;
+  int32_t NT;
+  float* d_type;            // backward: gradient of rab_type [NT*NT] (accumulated), or nullptr
 };
 
 // One launch of the persistent tensor-core GEMM (gemm_tc.cu): C[M, N] = epi(A · B), A and B

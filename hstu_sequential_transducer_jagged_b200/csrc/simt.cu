@@ -42,11 +42,17 @@ struct PairBias {
   float value;
   int pidx;
   int tidx;
+  int yidx;  // token-type pair index, -1 without the type term
 };
 
+// row0: the sequence's first token (for the token types).
 __device__ __forceinline__ PairBias pair_bias(const AttnGeom& g, int i, int j, int n, long long ti,
-                                              long long tj) {
-  PairBias b{0.f, -1, -1};
+                                              long long tj, int row0) {
+  PairBias b{0.f, -1, -1, -1};
+  if (g.rab_type != nullptr) {
+    b.yidx = g.types[row0 + i] * g.NT + g.types[row0 + j];
+    b.value += g.rab_type[b.yidx];
+  }
   if (g.rab_pos != nullptr) {
     const int pi = i < n ? i : n;
     const int pj = j < n ? j : n;
@@ -113,7 +119,7 @@ __global__ void __launch_bounds__(128)
         float s = 0.f;
 #pragma unroll
         for (int d = 0; d < D; ++d) s = fmaf(qr[d], ks[r][d], s);
-        const PairBias pb = pair_bias(g, i, j, n, ti, tss[r]);
+        const PairBias pb = pair_bias(g, i, j, n, ti, tss[r], it.row0);
         const float p = silu_f(g.alpha * s + pb.value);
 #pragma unroll
         for (int d = 0; d < D; ++d) acc[d] = fmaf(p, vs[r][d], acc[d]);
@@ -197,11 +203,12 @@ __global__ void __launch_bounds__(128)
   __shared__ float xs[kKvChunk][D];   // partner rows: K (KIND 0) or Q (KIND 1, 2)
   __shared__ float ys[kKvChunk][D];   // partner rows: V (KIND 0) or dO (KIND 1, 2)
   __shared__ long long tss[kKvChunk];
-  extern __shared__ float bias_grad[];  // KIND 0: [2P+1] position then [NB] time
+  extern __shared__ float bias_grad[];  // KIND 0: [2P+1] position, [NB] time, [NT^2] type
   const int npos = (g.rab_pos != nullptr) ? 2 * g.P + 1 : 0;
   const int ntime = (g.ts != nullptr && g.rab_time != nullptr) ? g.NB : 0;
+  const int ntype = (g.rab_type != nullptr) ? g.NT * g.NT : 0;
   if (KIND == 0) {
-    for (int e = threadIdx.x; e < npos + ntime; e += blockDim.x) bias_grad[e] = 0.f;
+    for (int e = threadIdx.x; e < npos + ntime + ntype; e += blockDim.x) bias_grad[e] = 0.f;
   }
   float a[D], b[D], acc[D];
 #pragma unroll
@@ -254,7 +261,7 @@ __global__ void __launch_bounds__(128)
       }
       const long long t_q = (KIND == 0) ? tr : tss[rr];
       const long long t_k = (KIND == 0) ? tss[rr] : tr;
-      const PairBias pb = pair_bias(g, qi, kj, n, t_q, t_k);
+      const PairBias pb = pair_bias(g, qi, kj, n, t_q, t_k, it.row0);
       const float s = g.alpha * qk + pb.value;
       if (KIND == 2) {
         const float pa = silu_f(s);
@@ -267,6 +274,7 @@ __global__ void __launch_bounds__(128)
         if (KIND == 0) {
           if (pb.pidx >= 0) atomicAdd(&bias_grad[pb.pidx], ds);
           if (pb.tidx >= 0 && ntime > 0) atomicAdd(&bias_grad[npos + pb.tidx], ds);
+          if (pb.yidx >= 0) atomicAdd(&bias_grad[npos + ntime + pb.yidx], ds);
         }
       }
     }
@@ -283,6 +291,9 @@ __global__ void __launch_bounds__(128)
       if (bias_grad[e] != 0.f) atomicAdd(&d_pos[e], bias_grad[e]);
     for (int e = threadIdx.x; e < ntime; e += blockDim.x)
       if (bias_grad[npos + e] != 0.f) atomicAdd(&d_time[e], bias_grad[npos + e]);
+    for (int e = threadIdx.x; e < ntype; e += blockDim.x)
+      if (bias_grad[npos + ntime + e] != 0.f && g.d_type != nullptr)
+        atomicAdd(&g.d_type[e], bias_grad[npos + ntime + e]);
   }
 }
 
@@ -346,7 +357,8 @@ static cudaError_t bwd_simt_d(const AttnGeom& g, const void* q, int64_t ld_q, co
                               float* d_time, int grid, cudaStream_t stream) {
   const size_t bias_smem =
       sizeof(float) * (((g.rab_pos != nullptr) ? 2 * g.P + 1 : 0) +
-                       ((g.ts != nullptr && g.rab_time != nullptr) ? g.NB : 0));
+                       ((g.ts != nullptr && g.rab_time != nullptr) ? g.NB : 0) +
+                       ((g.rab_type != nullptr) ? g.NT * g.NT : 0));
   if (bias_smem > 200 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_simt_kernel<T, D, 0>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -88,6 +88,14 @@ typedef struct {
   int32_t num_time_buckets;   /* NB >= 1 */
   float alpha;                /* scale of <q, k>; 1.0 is the literal formula */
   int32_t dtype;              /* hstu_dtype_t of Q/K/V/O (fp32 accumulation either way) */
+  /* Token-type term of bias_{i,j} = f(p_i - p_j, t_i - t_j, type_i, type_j) ("HSTU：Scaling Law
+   * 的首次探索" §7.1.4 innovation 2: content and action tokens relate differently), read as a
+   * learned table added to the two above: + rab_type[type_i * NT + type_j].  rab_type NULL
+   * (the default of a zeroed descriptor) disables it.  Calls with it run the single-tile
+   * tensor-core forward (or the CUDA-core kernels) and the CUDA-core backward. */
+  const int32_t* token_types; /* device int32 [T], values in [0, NT) */
+  const float* rab_type;      /* device fp32 [NT * NT] or NULL */
+  int32_t num_types;          /* NT in [1, 64] when rab_type is set */
 } hstu_attn_desc_t;
 
 /* Bytes of workspace hstu_attention_forward needs (status word + tile work list). */
@@ -146,6 +154,16 @@ hstu_status_t hstu_attention_backward(const hstu_attn_desc_t* desc, const void* 
                                       void* dk, void* dv, float* d_rab_pos, float* d_rab_time,
                                       void* ws, size_t ws_bytes, hstu_stream_t stream);
 
+/* hstu_attention_backward with the token-type term: also d_rab_type (fp32 [NT * NT],
+ * overwritten) = Σ dS over visible pairs with (type_i, type_j) = (a, b) at a NT + b.  Runs on
+ * the CUDA cores.  hstu_attention_backward itself returns HSTU_ERR_INVALID_ARG when
+ * desc->rab_type is set (it has no place for that gradient). */
+hstu_status_t hstu_attention_backward_typed(const hstu_attn_desc_t* desc, const void* q,
+                                            const void* k, const void* v, const void* d_o,
+                                            void* dq, void* dk, void* dv, float* d_rab_pos,
+                                            float* d_rab_time, float* d_rab_type, void* ws,
+                                            size_t ws_bytes, hstu_stream_t stream);
+
 /* One HSTU layer over a jagged batch ([Review §2.1], all three formulas + residual edge). */
 typedef struct {
   int32_t num_seqs, total_tokens, max_seq_len;
@@ -161,6 +179,9 @@ typedef struct {
   const float* ln_gamma;       /* fp32 [H*d_v] or NULL (= 1) */
   const float* ln_beta;        /* fp32 [H*d_v] or NULL (= 0) */
   int32_t dtype;               /* hstu_dtype_t of x, w1, w2, y */
+  const int32_t* token_types;  /* token-type term, as in hstu_attn_desc_t (NULL rab_type: off) */
+  const float* rab_type;
+  int32_t num_types;
 } hstu_layer_desc_t;
 
 /* Bytes of workspace hstu_layer_forward needs: status + work list + the f1 output
@@ -223,6 +244,7 @@ size_t hstu_layer_backward_workspace_size(const hstu_layer_desc_t* desc);
  *   d_rab_pos, d_rab_time          fp32 tables, as hstu_attention_backward (overwritten)
  *   d_ln_gamma, d_ln_beta          fp32 [H d_v], required when ln_gamma / ln_beta are set
  * with dpre = [dU | dV | dQ | dK] ⊙ SiLU'(X W1 + b1).  Every output is overwritten.  bf16 only,
+ * no token-type term (HSTU_ERR_UNSUPPORTED when desc->rab_type is set),
  * d_model a multiple of 8 and H d_v in {128, 256, 512, 1024} (else HSTU_ERR_UNSUPPORTED);
  * 16-byte aligned pointers.  Weight gradients are fp32 sums in no fixed order (atomic split-K
  * reduction), so they are reproducible only to rounding. */

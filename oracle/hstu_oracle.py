@@ -112,6 +112,16 @@ def allowed_pairs(L: int, mask: int, num_candidates: int):
     return causal & ((j < n) | (j == i))
 
 
+def type_bias_matrix(rows, types, rab_type, num_types):
+    """The token-type term of bias_{i,j} = f(p_i - p_j, t_i - t_j, type_i, type_j) ([FunRec 7.1]
+    §7.1.4 innovation 2: content and action tokens relate differently).  Reading: a learned
+    table over (type_i, type_j) pairs, rab_type[type_i * NT + type_j], added to the position and
+    time terms.  types: int [L] of one sequence, values in [0, NT)."""
+    types = np.asarray(types, dtype=np.int64)
+    idx = types[np.asarray(rows, dtype=np.int64)][:, None] * num_types + types[None, :]
+    return np.asarray(rab_type, dtype=np.float64)[idx]
+
+
 def bias_matrix(rows, L, ts, rab_pos, rab_time, max_pos_dist, num_buckets, mask, num_candidates):
     """rab_{p,t}(i, j) for the given query rows i and all keys j of one sequence (fp64)."""
     p = positions(L, mask, num_candidates)
@@ -137,10 +147,13 @@ def _heads(a, H, d):
 
 def attention_forward(q, k, v, seq_offsets, timestamps, rab_pos, rab_time, *, num_heads,
                       d_qk, d_v, max_pos_dist, num_time_buckets, alpha=1.0,
-                      mask=MASK_CAUSAL, num_candidates=0, rows=None):
+                      mask=MASK_CAUSAL, num_candidates=0, rows=None, token_types=None,
+                      rab_type=None, num_types=0):
     """Jagged pointwise attention.  q,k: [T, H*d_qk], v: [T, H*d_v] -> out [T, H*d_v] (fp64).
 
     If ``rows`` is given (global token indices), only those output rows are computed (others 0).
+    With token_types [T] and rab_type [NT*NT] the bias also carries the type term
+    (type_bias_matrix).
     """
     H = num_heads
     T = int(seq_offsets[-1])
@@ -164,6 +177,8 @@ def attention_forward(q, k, v, seq_offsets, timestamps, rab_pos, rab_time, *, nu
             okb = ok[blk:blk + 512]
             bias = bias_matrix(r, L, ts, rab_pos, rab_time, max_pos_dist, num_time_buckets,
                                mask, num_candidates)
+            if rab_type is not None:
+                bias = bias + type_bias_matrix(r, token_types[s:e], rab_type, num_types)
             for h in range(H):
                 scores = alpha * (Q[s + r, h, :] @ K[s:e, h, :].T) + bias
                 a = np.where(okb, silu(scores), 0.0)
@@ -211,7 +226,7 @@ def attention_forward_mfalcon_microbatched(q, k, v, seq_offsets, timestamps, rab
 
 def attention_backward(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time, *, num_heads,
                        d_qk, d_v, max_pos_dist, num_time_buckets, alpha=1.0, mask=MASK_CAUSAL,
-                       num_candidates=0):
+                       num_candidates=0, token_types=None, rab_type=None, num_types=0):
     """Gradients of L = Σ dO ⊙ out through the pointwise attention (chain rule, fp64).
 
     With S = α QKᵀ + rab, A = φ2(S) on allowed pairs (0 elsewhere), out = A V:
@@ -220,6 +235,8 @@ def attention_backward(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time,
       d rab_pos[k]  = Σ over allowed pairs with position index k of dS (all heads, all sequences);
       d rab_time[b] = Σ over allowed pairs with time bucket b of dS.
     The bias backward is the N×N rab gradient that [GenRank §6.2.3] names as RAB's cost.
+    With the type term (rab_type given) a sixth result d rab_type[a NT + b] = Σ over allowed
+    pairs with type_i = a, type_j = b of dS is returned.
     """
     H = num_heads
     T = int(seq_offsets[-1])
@@ -230,6 +247,7 @@ def attention_backward(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time,
     dV = np.zeros_like(V)
     d_pos = np.zeros(2 * max_pos_dist + 1, dtype=np.float64)
     d_time = np.zeros(num_time_buckets, dtype=np.float64)
+    d_type = None if rab_type is None else np.zeros(num_types * num_types, dtype=np.float64)
     for b in range(len(seq_offsets) - 1):
         s, e = int(seq_offsets[b]), int(seq_offsets[b + 1])
         L = e - s
@@ -240,6 +258,11 @@ def attention_backward(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time,
         ok = allowed_pairs(L, mask, num_candidates)
         bias = bias_matrix(rows, L, ts, rab_pos, rab_time, max_pos_dist, num_time_buckets,
                            mask, num_candidates)
+        yidx = None
+        if rab_type is not None:
+            bias = bias + type_bias_matrix(rows, token_types[s:e], rab_type, num_types)
+            ty = np.asarray(token_types[s:e], dtype=np.int64)
+            yidx = ty[:, None] * num_types + ty[None, :]
         p = positions(L, mask, num_candidates)
         pidx = position_index(p[:, None] - p[None, :], max_pos_dist)
         tidx = None
@@ -257,8 +280,11 @@ def attention_backward(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time,
                 d_pos += np.bincount(pidx[ok], weights=dS[ok], minlength=d_pos.size)
             if tidx is not None and rab_time is not None:
                 d_time += np.bincount(tidx[ok], weights=dS[ok], minlength=d_time.size)
-    return (dQ.reshape(T, H * d_qk), dK.reshape(T, H * d_qk), dV.reshape(T, H * d_v),
-            d_pos, d_time)
+            if yidx is not None:
+                d_type += np.bincount(yidx[ok], weights=dS[ok], minlength=d_type.size)
+    out = (dQ.reshape(T, H * d_qk), dK.reshape(T, H * d_qk), dV.reshape(T, H * d_v), d_pos,
+           d_time)
+    return out if d_type is None else out + (d_type,)
 
 
 # --------------------------------------------------------------------------------------------
@@ -297,13 +323,15 @@ def layer_norm(a, eps=1e-5, gamma=None, beta=None):
 def layer_forward(x, w1, w2, seq_offsets, timestamps, rab_pos, rab_time, *, num_heads, d_qk,
                   d_v, max_pos_dist, num_time_buckets, alpha=1.0, mask=MASK_CAUSAL,
                   num_candidates=0, b1=None, b2=None, ln_eps=1e-5, ln_gamma=None,
-                  ln_beta=None, return_intermediates=False):
+                  ln_beta=None, return_intermediates=False, token_types=None, rab_type=None,
+                  num_types=0):
     z = silu(linear(x, w1, b1))                                        # φ1(f1(X))
     u, v, q, k = split_uvqk(z, num_heads, d_qk, d_v)                   # Split
     av = attention_forward(q, k, v, seq_offsets, timestamps, rab_pos, rab_time,
                            num_heads=num_heads, d_qk=d_qk, d_v=d_v, max_pos_dist=max_pos_dist,
                            num_time_buckets=num_time_buckets, alpha=alpha, mask=mask,
-                           num_candidates=num_candidates)              # A(X)V(X)
+                           num_candidates=num_candidates, token_types=token_types,
+                           rab_type=rab_type, num_types=num_types)     # A(X)V(X)
     g = layer_norm(av, ln_eps, ln_gamma, ln_beta) * u                  # Norm(AV) ⊙ U
     y = np.asarray(x, dtype=np.float64) + linear(g, w2, b2)            # X + f2(·)
     if return_intermediates:

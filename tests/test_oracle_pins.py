@@ -572,3 +572,90 @@ def test_stochastic_length_sparsity_claim():
         p = 1.0 - n_alpha / N ** 2
         kept_pairs = p * k * (k + 1) / 2 + (1 - p) * N * (N + 1) / 2
         assert kept_pairs / (N * (N + 1) / 2) < 0.2, alpha
+
+
+# ------------------------------------------------------- token-type bias ([FunRec 7.1] §7.1.4)
+def _typed_case(seed, lengths, NT, mask=O.MASK_CAUSAL, m=0):
+    case = W.random_attention_case(seed, lengths, H=2, d=8, P=6, NB=8, mask=mask,
+                                   num_candidates=m, gap_mean=30.0)
+    rng = np.random.default_rng(seed + 1)
+    types = rng.integers(0, NT, size=case.total_tokens)
+    rab_type = rng.normal(0.0, 0.5, size=NT * NT)
+    return case, types, rab_type
+
+
+def _akw(case):
+    return dict(num_heads=case.num_heads, d_qk=case.d_qk, d_v=case.d_v,
+                max_pos_dist=case.max_pos_dist, num_time_buckets=case.num_time_buckets,
+                alpha=case.alpha, mask=case.mask, num_candidates=case.num_candidates)
+
+
+def test_type_bias_explicit_pairwise_loop():
+    """The type term inside the SiLU, against a pair-by-pair loop of the whole bias
+    rab_pos + rab_time + rab_type[type_i NT + type_j]."""
+    for mask, m in ((O.MASK_CAUSAL, 0), (O.MASK_MFALCON, 3)):
+        case, types, rt = _typed_case(31, [9, 1, 12], 3, mask, m)
+        got = O.attention_forward(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
+                                  case.rab_pos, case.rab_time, token_types=types, rab_type=rt,
+                                  num_types=3, **_akw(case))
+        H, d, P, NB = 2, 8, 6, 8
+        want = np.zeros_like(got)
+        off = case.seq_offsets
+        for b in range(len(off) - 1):
+            s, e = int(off[b]), int(off[b + 1])
+            L = e - s
+            n = L - m if mask == O.MASK_MFALCON else L
+            for i in range(L):
+                for j in range(L):
+                    vis = j <= i and (mask == O.MASK_CAUSAL or j < n or j == i)
+                    if not vis:
+                        continue
+                    pi, pj = min(i, n), min(j, n)
+                    dt = int(case.timestamps[s + i]) - int(case.timestamps[s + j])
+                    bkt = min(max(max(dt, 1).bit_length() - 1, 0), NB - 1)
+                    bias = (float(case.rab_pos[min(max(pi - pj, -P), P) + P])
+                            + float(case.rab_time[bkt]) + float(rt[types[s + i] * 3 + types[s + j]]))
+                    for h in range(H):
+                        sc = float(np.dot(case.q[s + i, h * d:(h + 1) * d].astype(np.float64),
+                                          case.k[s + j, h * d:(h + 1) * d].astype(np.float64)))
+                        x = sc + bias
+                        want[s + i, h * d:(h + 1) * d] += x / (1 + math.exp(-x)) * \
+                            case.v[s + j, h * d:(h + 1) * d].astype(np.float64)
+        assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_type_bias_single_type_is_a_constant_shift():
+    """One token type: the type term is the constant rab_type[0] on every pair, the same as
+    adding it to every position-table entry."""
+    case, types, rt = _typed_case(32, [10, 7], 1)
+    got = O.attention_forward(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
+                              case.rab_pos, case.rab_time, token_types=np.zeros_like(types),
+                              rab_type=rt, num_types=1, **_akw(case))
+    want = O.attention_forward(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
+                               case.rab_pos + rt[0], case.rab_time, **_akw(case))
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_type_bias_gradient_finite_differences():
+    """d rab_type against central differences of Σ dO ⊙ out, and its total equal to the other
+    two tables' totals (every visible pair has one index in each table)."""
+    case, types, rt = _typed_case(33, [8, 5], 2)
+    d_o = np.random.default_rng(4).standard_normal(case.q.shape)
+    res = O.attention_backward(case.q, case.k, case.v, d_o, case.seq_offsets, case.timestamps,
+                               case.rab_pos, case.rab_time, token_types=types, rab_type=rt,
+                               num_types=2, **_akw(case))
+    d_type = res[5]
+
+    def loss(tab):
+        o = O.attention_forward(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
+                                case.rab_pos, case.rab_time, token_types=types, rab_type=tab,
+                                num_types=2, **_akw(case))
+        return float(np.sum(o * d_o))
+
+    for c in range(4):
+        e = np.zeros(4)
+        e[c] = 1e-6
+        fd = (loss(rt + e) - loss(rt - e)) / 2e-6
+        assert abs(fd - d_type[c]) <= 1e-6 * max(1.0, abs(fd))
+    assert abs(d_type.sum() - res[3].sum()) <= 1e-9 * max(1.0, abs(res[3].sum()))
+    assert abs(d_type.sum() - res[4].sum()) <= 1e-9 * max(1.0, abs(res[4].sum()))
