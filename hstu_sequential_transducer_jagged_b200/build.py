@@ -14,7 +14,7 @@ LIB_NAME = "libhstu_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["api.cu", "attn_fwd_tc.cu", "attn_fwd_pair.cu", "attn_bwd_tc.cu", "gemm_tc.cu", "pointwise.cu",
            "simt.cu", "layer_bwd.cu",
-           "sampling.cu"]
+           "sampling.cu", "f2_fused.cu"]
 HEADERS = ["ptx.cuh", "common.cuh", "bias_index.cuh"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

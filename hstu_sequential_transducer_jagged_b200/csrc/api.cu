@@ -79,6 +79,12 @@ cudaError_t launch_candidate_rows(const int32_t* off, int B, int m, int32_t* idx
 cudaError_t launch_scatter_rows(const void* src, int64_t src_stride, const int32_t* index, int n,
                                 void* dst, int64_t dst_stride, int64_t row_bytes, int num_sms,
                                 cudaStream_t stream);
+bool f2_fused_supported(int F, int N);
+cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_w2, int M, int N,
+                            int F, const __nv_bfloat16* u, int64_t ld_u, const float* gamma,
+                            const float* beta, float eps, const float* bias,
+                            const __nv_bfloat16* x, int64_t ld_x, __nv_bfloat16* y, int64_t ld_y,
+                            int* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_colsum(const __nv_bfloat16* m, int64_t ld, int rows, int cols, float* out,
                           cudaStream_t stream);
 int attn_bwd_tc_ts_box();
@@ -350,6 +356,33 @@ hstu_status_t gemm(int dtype, int epi, const void* A, int64_t lda, const void* B
     e = launch_gemm_simt(dtype, epi, A, lda, Bm, ldb, M, N, K, bias, R, ldr, C, ldc, s);
   }
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+}
+
+// Y = X + (Norm(AV) ⊙ U) W2 + b2 over `rows` tokens: one fused tensor-core kernel for bf16 with
+// H d_v <= 512 (G formed in shared memory), else LayerNorm ⊙ U into g_buf and the GEMM.
+hstu_status_t norm_gate_f2(int dtype, const void* av, int64_t ld_av, const void* u, int64_t ld_u,
+                           const float* gamma, const float* beta, float eps, const void* w2,
+                           const float* b2, const void* x, void* y, int rows, int F, int d_model,
+                           void* g_buf, int32_t* status, cudaStream_t s) {
+  const bool fused = dtype == HSTU_BF16 && f2_fused_supported(F, d_model) && ld_av % 8 == 0 &&
+                     ld_u % 8 == 0 && d_model % 8 == 0 && aligned16(av) && aligned16(u) &&
+                     aligned16(w2) && aligned16(x) && aligned16(y);
+  if (fused) {
+    CUtensorMap tav, tw2;
+    if (!make_map_bf16(&tav, av, rows, F, ld_av, 64, 128) ||
+        !make_map_bf16(&tw2, w2, F, d_model, d_model, 64, 64))
+      return HSTU_ERR_CUDA;
+    const cudaError_t e = launch_f2_fused(
+        tav, tw2, rows, d_model, F, static_cast<const __nv_bfloat16*>(u), ld_u, gamma, beta, eps,
+        b2, static_cast<const __nv_bfloat16*>(x), d_model, static_cast<__nv_bfloat16*>(y),
+        d_model, status, num_sms_current(), s);
+    return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
+  }
+  if (launch_ln_gate(dtype == HSTU_BF16 ? 0 : 1, av, ld_av, u, ld_u, gamma, beta, eps, g_buf, F,
+                     rows, F, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  return gemm(dtype, 1, g_buf, F, w2, d_model, rows, d_model, F, b2, x, d_model, y, d_model,
+              status, s);
 }
 
 // C = epi(op(A) op(B)) on the tensor cores for the backward's operand layouts: a_mn = 1 takes A
@@ -665,11 +698,8 @@ hstu_status_t layer_stage(const hstu_layer_desc_t* d, int32_t stage, const void*
                              d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av, hv, s);
   }
   // Norm(AV) ⊙ U, then f2 + residual: Y = X + G W2 + b2
-  if (launch_ln_gate(d->dtype == HSTU_BF16 ? 0 : 1, av, hv, u_ptr, n1, d->ln_gamma, d->ln_beta,
-                     d->ln_eps, gbuf, hv, T, hv, s) != cudaSuccess)
-    return HSTU_ERR_CUDA;
-  return gemm(d->dtype, 1, gbuf, hv, w2, d->d_model, T, d->d_model, hv, b2, x, d->d_model, y,
-              d->d_model, status, s);
+  return norm_gate_f2(d->dtype, av, hv, u_ptr, n1, d->ln_gamma, d->ln_beta, d->ln_eps, w2, b2, x,
+                      y, T, hv, d->d_model, gbuf, status, s);
 }
 }  // namespace
 
@@ -802,11 +832,8 @@ hstu_status_t hstu_layer_forward_candidates(const hstu_layer_desc_t* d, const vo
                               static_cast<int64_t>(hv) * es, static_cast<int64_t>(hv) * es, nsm,
                               s)) != cudaSuccess)
     return cuda_fail(e);
-  if ((e = launch_ln_gate(d->dtype == HSTU_BF16 ? 0 : 1, avc, hv, uc, hv, d->ln_gamma,
-                          d->ln_beta, d->ln_eps, gc, hv, bm, hv, s)) != cudaSuccess)
-    return cuda_fail(e);
-  return gemm(d->dtype, 1, gc, hv, w2, d->d_model, bm, d->d_model, hv, b2, x_cand, d->d_model,
-              y_cand, d->d_model, status, s);
+  return norm_gate_f2(d->dtype, avc, hv, uc, hv, d->ln_gamma, d->ln_beta, d->ln_eps, w2, b2,
+                      x_cand, y_cand, bm, hv, d->d_model, gc, status, s);
 }
 
 size_t hstu_layer_backward_workspace_size(const hstu_layer_desc_t* d) {
