@@ -179,3 +179,95 @@ def test_wait_timeout_probe_rejects_bad_workspace(lib):
     assert lib.hstu_debug_wait_timeout(None, 256, None) == 3
     assert lib.hstu_debug_wait_timeout(ctypes.c_void_p((1 << 20) + 8), 256, None) == 3
     assert lib.hstu_debug_wait_timeout(FAKE, 100, None) == 3
+
+
+def test_static_scratch_rejects_bad_strides_before_touching_the_array(lib):
+    # a stride below the row width is rejected on the host (the shared array is not touched)
+    assert lib.hstu_attention_forward_static_ws(ctypes.byref(_desc(ld_q=64)), FAKE, FAKE, FAKE,
+                                                FAKE, None, None) == 1
+    assert lib.hstu_attention_forward_static_ws(ctypes.byref(_desc()), None, FAKE, FAKE, FAKE,
+                                                None, None) == 1
+
+
+def test_layer_backward_validates_on_the_host(lib):
+    bf = dict(dtype=0, d_model=128, num_heads=2, d_qk=64, d_v=64)
+    d = _ldesc(**bf)
+    need = lib.hstu_layer_backward_workspace_size(ctypes.byref(d))
+    assert need > lib.hstu_layer_workspace_size(ctypes.byref(d))
+    ws = ctypes.c_void_p(1 << 20)
+    args = [FAKE, FAKE, None, FAKE, None, FAKE, ctypes.c_void_p(3 << 20), FAKE, None, FAKE,
+            None, None, None, None, None]
+    # fp32 layers and rows of H*d_v outside {128, 256, 512, 1024} are not supported
+    assert lib.hstu_layer_backward(ctypes.byref(_ldesc()), *args, ws, 1 << 40, None) == 2
+    assert lib.hstu_layer_backward(ctypes.byref(_ldesc(**dict(bf, d_v=48, d_qk=48))), *args, ws,
+                                   1 << 40, None) == 2
+    # too small a workspace
+    assert lib.hstu_layer_backward(ctypes.byref(d), *args, ws, need - 1, None) == 3
+    # d_x aliasing x
+    bad = list(args)
+    bad[6] = FAKE
+    assert lib.hstu_layer_backward(ctypes.byref(d), *bad, ws, need, None) == 1
+    # a LayerNorm affine without its gradient buffer
+    d2 = _ldesc(ln_gamma=1 << 20, **bf)
+    assert lib.hstu_layer_backward(ctypes.byref(d2), *args, ws, 1 << 40, None) == 1
+
+
+def test_stochastic_length_and_gather_validate(lib):
+    ws = ctypes.c_void_p(1 << 20)
+    need = lib.hstu_stochastic_length_workspace_size(4, 100)
+    assert need >= 256 + 400 + 16
+    ok = [FAKE, 4, 100, 64, 10, 1000.0, FAKE, FAKE, FAKE, FAKE, ws, need, None]
+    for i, bad in ((4, 0), (5, float("nan")), (5, -1.0), (3, -1), (2, -1)):
+        a = list(ok)
+        a[i] = bad
+        assert lib.hstu_stochastic_length(*a) == 1, (i, bad)
+    a = list(ok)
+    a[3] = 10  # 4 sequences of <= 10 tokens cannot hold 100
+    assert lib.hstu_stochastic_length(*a) == 1
+    a = list(ok)
+    a[11] = need - 1
+    assert lib.hstu_stochastic_length(*a) == 3
+    # gather: misaligned rows, negative sizes, nothing to do
+    assert lib.hstu_gather_rows(FAKE, 16, FAKE, None, 4, FAKE, 16, 6, None) == 1
+    assert lib.hstu_gather_rows(FAKE, 16, FAKE, None, -1, FAKE, 16, 16, None) == 1
+    assert lib.hstu_gather_rows(FAKE, 16, FAKE, None, 0, FAKE, 16, 16, None) == 0
+    assert lib.hstu_gather_rows(None, 16, FAKE, None, 4, FAKE, 16, 16, None) == 1
+
+
+def test_mfalcon_cache_calls_validate(lib):
+    d = _ldesc(dtype=0, d_model=128, num_heads=2, d_qk=64, d_v=64, mask=1, num_candidates=16)
+    assert lib.hstu_layer_cache_bytes(ctypes.byref(d)) == 100 * 2 * 2 * 128 * 2
+    need = lib.hstu_layer_candidates_workspace_size(ctypes.byref(d))
+    ws = ctypes.c_void_p(1 << 20)
+    # the candidates pass needs the M-FALCON mask and at least one candidate
+    causal = _ldesc(dtype=0, d_model=128, num_heads=2, d_qk=64, d_v=64)
+    assert lib.hstu_layer_forward_candidates(ctypes.byref(causal), FAKE, FAKE, None, FAKE, None,
+                                             ctypes.c_void_p(2 << 20), FAKE, ws, 1 << 40,
+                                             None) == 1
+    # B * m above T
+    many = _ldesc(dtype=0, d_model=128, num_heads=2, d_qk=64, d_v=64, mask=1, num_candidates=60)
+    assert lib.hstu_layer_forward_candidates(ctypes.byref(many), FAKE, FAKE, None, FAKE, None,
+                                             ctypes.c_void_p(2 << 20), FAKE, ws, 1 << 40,
+                                             None) == 1
+    assert lib.hstu_layer_forward_candidates(ctypes.byref(d), FAKE, FAKE, None, FAKE, None,
+                                             ctypes.c_void_p(2 << 20), FAKE, ws, need - 1,
+                                             None) == 3
+    # the cached forward needs a cache
+    assert lib.hstu_layer_forward_cached(ctypes.byref(d), FAKE, FAKE, None, FAKE, None,
+                                         ctypes.c_void_p(2 << 20), None, ws, 1 << 40, None) == 1
+
+
+def test_type_bias_arguments(lib):
+    # rab_type without token types, or NT outside [1, 64]
+    for kw in (dict(rab_type=1 << 20, num_types=2, token_types=None),
+               dict(rab_type=1 << 20, num_types=0, token_types=1 << 20),
+               dict(rab_type=1 << 20, num_types=65, token_types=1 << 20)):
+        d = _desc(**kw)
+        assert lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                          None) == 1
+    d = _desc(rab_type=1 << 20, num_types=2, token_types=1 << 20)
+    # the plain backward has no place for the type gradient; the typed one needs its buffer
+    assert lib.hstu_attention_backward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       None, None, FAKE, 1 << 30, None) == 1
+    assert lib.hstu_attention_backward_typed(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                             FAKE, None, None, None, FAKE, 1 << 30, None) == 1
