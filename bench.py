@@ -107,7 +107,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", str(gpu_index)], stdout=subprocess.PIPE,
+                 "-lms", "20", "-i", str(gpu_index)], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -426,6 +426,66 @@ def time_layer_stack(lib, Bd, dev, name, steps, warmup, seed=0):
             "l2": "256 MB buffer written between steps (outside the step events)"}
 
 
+def time_layer_backward(lib, Bd, dev, steps, warmup, seed=0, batch=0):
+    """One layer's backward (hstu_layer_backward, forward recomputed inside) on layer 0 of the
+    4-layer workload, next to that layer's forward; L2 flushed between timed calls.  FLOPs:
+    forward f1 + attention + f2, backward 2x the GEMMs and 8 d per attention pair (plus the
+    recomputed forward, reported apart)."""
+    import torch
+    wl = W.make(WORKLOAD, seed=seed)
+    if batch > 0:
+        wl = truncate_batch(wl, batch)
+    bf = torch.bfloat16
+    lp = wl.layers[0]
+    x = torch.from_numpy(wl.x).to(bf).to(dev)
+    w1 = torch.from_numpy(lp.w1).to(bf).to(dev)
+    w2 = torch.from_numpy(lp.w2).to(bf).to(dev)
+    off = torch.from_numpy(wl.seq_offsets).to(dev)
+    ts = torch.from_numpy(wl.timestamps).to(dev)
+    rp, rt = torch.from_numpy(lp.rab_pos).to(dev), torch.from_numpy(lp.rab_time).to(dev)
+    d_y = torch.randn(x.shape, generator=torch.Generator().manual_seed(seed)).to(bf).to(dev)
+    kw = dict(num_heads=wl.num_heads, d_qk=wl.d_qk, d_v=wl.d_v, max_pos_dist=wl.max_pos_dist,
+              num_time_buckets=wl.num_time_buckets, alpha=wl.alpha)
+    desc = Bd.layer_desc(seq_offsets=off, total_tokens=wl.total_tokens, max_seq_len=wl.max_seq_len,
+                         timestamps=ts, d_model=wl.d_model, rab_pos=rp, rab_time=rt,
+                         ln_eps=wl.ln_eps, **kw)
+    ws = Bd.Workspace(lib.hstu_layer_backward_workspace_size(ctypes.byref(desc)), dev)
+    y = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        Bd.layer_forward(x, w1, w2, off, wl.max_seq_len, ts, rp, rt, out=y, ws=ws, **kw)
+
+    def bwd():
+        Bd.layer_backward(x, w1, w2, d_y, off, wl.max_seq_len, ts, rp, rt, ws=ws, **kw)
+
+    res = {}
+    for name, fn in (("fwd", fwd), ("bwd", bwd)):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        res[name] = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    if ws.sync_status() != 0:
+        raise RuntimeError("device status word set")
+    aflops, gflops = attention_flops(wl), gemm_flops(wl)
+    bwd_alg = 2 * gflops + 2 * aflops  # dX, dW per GEMM; 8 d per pair for the attention
+    return {"workload": wl.name + " layer 0", "tokens": wl.total_tokens, "steps": steps,
+            "fwd_ms": res["fwd"], "bwd_ms": res["bwd"],
+            "fwd_bwd_tokens_per_s": wl.total_tokens / ((res["fwd"] + res["bwd"]) / 1e3),
+            "bwd_tflops_algorithmic": bwd_alg / (res["bwd"] / 1e3) / 1e12,
+            "bwd_recompute_gflop": (aflops + gflops) / 1e9,
+            "l2": "256 MB buffer written before each timed call (outside its events)"}
+
+
 def measure_other_configs(lib, Bd, dev, peaks):
     """The other four workloads, each timed on its own (they are parity cases of the same
     kernels; the headline line is the 4-layer stack)."""
@@ -441,6 +501,9 @@ def measure_other_configs(lib, Bd, dev, peaks):
     r["fwd_frac_of_bf16_peak"] = r["fwd_tflops"] / pk
     r["bwd_frac_of_bf16_peak"] = r["bwd_tflops"] / pk
     out[r["workload"]] = r
+    r = time_layer_backward(lib, Bd, dev, 10, 3)
+    r["bwd_frac_of_bf16_peak"] = r["bwd_tflops_algorithmic"] / pk
+    out["layer_backward"] = r
     return out
 
 
@@ -532,7 +595,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other four workloads (timed after the headline line)")
-    ap.add_argument("--mode", default="stack", choices=["stack", "attn", "attn_bwd"],
+    ap.add_argument("--mode", default="stack", choices=["stack", "attn", "attn_bwd", "layer_bwd"],
                     help="attn: time only the attention stage of layer 0 (profiling aid); "
                          "attn_bwd: attention forward and backward on the B=64 workload")
     ap.add_argument("--batch", type=int, default=0,
@@ -560,6 +623,11 @@ def main():
     lib = Bd.lib()
     if args.mode == "attn_bwd":
         run_attention_bwd(args, lib, Bd, dev)
+        return
+    if args.mode == "layer_bwd":
+        r = time_layer_backward(lib, Bd, dev, args.steps, args.warmup, args.seed, args.batch)
+        r["mode"] = "layer_bwd"
+        print(json.dumps(r), flush=True)
         return
 
     # CPU oracle baseline first (rank 0, one GPU), before any other GPU work

@@ -225,10 +225,13 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[W], uint32_t (&pk
     } else if (MODE == kModeElem || MODE == kModeCausal) {
       // exact for every row: beyond the band the clamped table repeats its last entry
       const float4 pv = pos4[pos4_row(rc.pbase, c, rc.P2)];
-      bb[0] = rc.half_bias + pv.x;
-      bb[1] = rc.half_bias + pv.y;
-      bb[2] = rc.half_bias + pv.z;
-      bb[3] = rc.half_bias + pv.w;
+      const float2 hb = make_float2(rc.half_bias, rc.half_bias);
+      const float2 b01 = add2(hb, make_float2(pv.x, pv.y));
+      const float2 b23 = add2(hb, make_float2(pv.z, pv.w));
+      bb[0] = b01.x;
+      bb[1] = b01.y;
+      bb[2] = b23.x;
+      bb[3] = b23.y;
     } else {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -247,10 +250,19 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&s)[W], uint32_t (&pk
 #pragma unroll
       for (int u = 0; u < 4; ++u) bb[u] += time_h[time_bucket64(rc.ti - ts[c + u], rc.nbm1 + 1)];
     }
+    // SiLU(x) = h (1 + tanh h), h = x / 2, on pairs of scores with packed f32x2 FMAs
     float p[4];
+    const float2 ha = make_float2(rc.half_alpha, rc.half_alpha);
+#pragma unroll
+    for (int u = 0; u < 4; u += 2) {
+      const float2 h = fma2(ha, make_float2(__uint_as_float(s[q + u]), __uint_as_float(s[q + u + 1])),
+                            make_float2(bb[u], bb[u + 1]));
+      const float2 pp = fma2(h, make_float2(tanh_fast(h.x), tanh_fast(h.y)), h);
+      p[u] = pp.x;
+      p[u + 1] = pp.y;
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      p[u] = silu_half(fmaf(rc.half_alpha, __uint_as_float(s[q + u]), bb[u]));
       const int j = rc.c0t + c + u;
       if (MODE == kModeCausal) p[u] = j <= rc.i ? p[u] : 0.f;
       if (MODE == kModeGeneral) {
