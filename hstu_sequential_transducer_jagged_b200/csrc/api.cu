@@ -56,15 +56,17 @@ cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tts, const AttnGeom& g, __nv_bfloat16* dq,
                                int64_t ld_dq, __nv_bfloat16* dk, int64_t ld_dk,
                                __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc, float* d_pos,
-                               float* d_time, int grid, bool fast, cudaStream_t stream);
+                               float* d_time, int grid, bool fast, const SiluGradZ& zg,
+                               cudaStream_t stream);
 size_t attn_bwd_tc_smem(int P, int NB);
 cudaError_t launch_ln_gate_bwd(const __nv_bfloat16* av, int64_t ld_av, const __nv_bfloat16* u,
                                int64_t ld_u, const __nv_bfloat16* dg, int64_t ld_dg,
                                const float* gamma, const float* beta, float eps,
                                __nv_bfloat16* d_av, int64_t ld_dav, __nv_bfloat16* d_u,
-                               int64_t ld_du, float* d_gamma, float* d_beta, int rows, int F,
-                               int num_sms, cudaStream_t stream);
-cudaError_t launch_silu_grad_mul(const __nv_bfloat16* z, int64_t ld_z, const __nv_bfloat16* da,
+                               int64_t ld_du, const float* z_u, int64_t ld_z, float* d_gamma,
+                               float* d_beta, int rows, int F, int num_sms,
+                               cudaStream_t stream);
+cudaError_t launch_silu_grad_mul(const float* z, int64_t ld_z, const __nv_bfloat16* da,
                                  int64_t ld_da, __nv_bfloat16* dz, int64_t ld_dz, int rows,
                                  int cols, int num_sms, cudaStream_t stream);
 cudaError_t launch_stochastic_length(const int32_t* off, int B, int T, int max_len, int sub_len,
@@ -386,8 +388,8 @@ hstu_status_t norm_gate_f2(int dtype, const void* av, int64_t ld_av, const void*
 }
 
 // C = epi(op(A) op(B)) on the tensor cores for the backward's operand layouts: a_mn = 1 takes A
-// stored [K, M] (lda its row stride), b_mn = 0 takes B stored [N, K].  epi 4 accumulates fp32
-// into Cf with k_splits work units per output tile.
+// stored [K, M] (lda its row stride), b_mn = 0 takes B stored [N, K].  epi 3 also writes the
+// fp32 pre-activation to C2; epi 4 accumulates fp32 into Cf with k_splits work units per tile.
 hstu_status_t gemm_tc_layout(int epi, int a_mn, int b_mn, const void* A, int64_t lda,
                              const void* Bm, int64_t ldb, int M, int N, int K, int k_splits,
                              const float* bias, const void* R, int64_t ldr, void* C, int64_t ldc, void* C2,
@@ -413,7 +415,7 @@ hstu_status_t gemm_tc_layout(int epi, int a_mn, int b_mn, const void* A, int64_t
   ga.ld_r = ldr;
   ga.C = static_cast<__nv_bfloat16*>(C);
   ga.ldc = ldc;
-  ga.C2 = static_cast<__nv_bfloat16*>(C2);
+  ga.C2 = static_cast<float*>(C2);
   ga.ld_c2 = ld_c2;
   ga.Cf = Cf;
   ga.status = status;
@@ -444,7 +446,7 @@ LayerBwdLayout layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_attn_desc
   LayerBwdLayout l;
   l.attn = 0;
   l.z = align_up(hstu_attention_backward_workspace_size(&ad));
-  l.a = l.z + align_up(T * n1 * 2);
+  l.a = l.z + align_up(T * n1 * 4);  // the pre-activation in fp32
   l.av = l.a + align_up(T * n1 * 2);
   l.g = l.av + align_up(T * hv * 2);
   l.dg = l.g + align_up(T * hv * 2);
@@ -484,6 +486,14 @@ hstu_attn_desc_t layer_attn_desc(const hstu_layer_desc_t* d) {
   return a;
 }
 
+}  // namespace
+
+namespace {
+hstu_status_t attn_backward_impl(const hstu_attn_desc_t* d, const void* q, const void* k,
+                                 const void* v, const void* d_o, void* dq, void* dk, void* dv,
+                                 float* d_rab_pos, float* d_rab_time, float* d_rab_type,
+                                 void* ws, size_t ws_bytes, hstu_stream_t stream,
+                                 const SiluGradZ& zg, bool* zg_applied);
 }  // namespace
 
 extern "C" {
@@ -546,6 +556,22 @@ hstu_status_t hstu_attention_backward_typed(const hstu_attn_desc_t* d, const voi
                                             void* dq, void* dk, void* dv, float* d_rab_pos,
                                             float* d_rab_time, float* d_rab_type, void* ws,
                                             size_t ws_bytes, hstu_stream_t stream) {
+  return attn_backward_impl(d, q, k, v, d_o, dq, dk, dv, d_rab_pos, d_rab_time, d_rab_type, ws,
+                            ws_bytes, stream, SiluGradZ{nullptr, nullptr, nullptr, 0}, nullptr);
+}
+
+}  // extern "C"
+
+namespace {
+// The attention backward.  zg (a layer's backward) multiplies dQ, dK, dV by SiLU'(Z) before
+// their rounding when the tensor-core kernel runs; *zg_applied reports whether it did (the
+// CUDA-core kernels leave dQ, dK, dV unscaled).
+hstu_status_t attn_backward_impl(const hstu_attn_desc_t* d, const void* q, const void* k,
+                                 const void* v, const void* d_o, void* dq, void* dk, void* dv,
+                                 float* d_rab_pos, float* d_rab_time, float* d_rab_type,
+                                 void* ws, size_t ws_bytes, hstu_stream_t stream,
+                                 const SiluGradZ& zg, bool* zg_applied) {
+  if (zg_applied != nullptr) *zg_applied = false;
   if (d == nullptr) return HSTU_ERR_INVALID_ARG;
   {
     const hstu_status_t tst = check_types(d->token_types, d->rab_type, d->num_types,
@@ -618,13 +644,17 @@ hstu_status_t hstu_attention_backward_typed(const hstu_attn_desc_t* d, const voi
     e = launch_attn_bwd_tc(tq, tk, tv, tdo, tts, g, static_cast<__nv_bfloat16*>(dq), d->ld_q,
                            static_cast<__nv_bfloat16*>(dk), d->ld_k,
                            static_cast<__nv_bfloat16*>(dv), d->ld_v, dq_acc, d_rab_pos,
-                           d_rab_time, pgrid, true, s);
+                           d_rab_time, pgrid, true, zg, s);
+    if (zg_applied != nullptr) *zg_applied = zg.q != nullptr;
   } else {
     e = launch_attn_bwd_simt(d->dtype, D, g, q, d->ld_q, k, d->ld_k, v, d->ld_v, d_o, d->ld_o,
                              dq, dk, dv, d_rab_pos, d_rab_time, grid, s);
   }
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
+}  // namespace
+
+extern "C" {
 
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* d) {
   if (d == nullptr || d->total_tokens < 0 || d->num_seqs < 0 || d->max_seq_len < 0 ||
@@ -881,7 +911,7 @@ hstu_status_t hstu_layer_backward(const hstu_layer_desc_t* d, const void* x, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* status = reinterpret_cast<int32_t*>(base);
-  auto* z = reinterpret_cast<__nv_bfloat16*>(base + L.z);
+  auto* z = reinterpret_cast<float*>(base + L.z);
   auto* a = reinterpret_cast<__nv_bfloat16*>(base + L.a);
   auto* av = reinterpret_cast<__nv_bfloat16*>(base + L.av);
   auto* g = reinterpret_cast<__nv_bfloat16*>(base + L.g);
@@ -921,18 +951,23 @@ hstu_status_t hstu_layer_backward(const hstu_layer_desc_t* d, const void* x, con
   if (d_ln_beta != nullptr && (e = cudaMemsetAsync(d_ln_beta, 0, sizeof(float) * hv, s)) != cudaSuccess)
     return cuda_fail(e);
   e = launch_ln_gate_bwd(av, hv, a + offU, n1, dg, hv, d->ln_gamma, d->ln_beta, d->ln_eps, dav,
-                         hv, da + offU, n1, d->ln_gamma ? d_ln_gamma : nullptr,
+                         hv, da + offU, n1, z + offU, n1, d->ln_gamma ? d_ln_gamma : nullptr,
                          d->ln_beta ? d_ln_beta : nullptr, T, hv, nsm, s);
   if (e != cudaSuccess) return cuda_fail(e);
   // ---- attention: dQ, dK, dV into dA's Q, K, V blocks; the bias-table gradients
   hstu_attn_desc_t bd = ad;
   bd.ld_o = hv;  // dO = dAV
-  st = hstu_attention_backward(&bd, a + offQ, a + offK, a + offV, dav, da + offQ, da + offK,
-                               da + offV, d_rab_pos, d_rab_time, ws, attn_ws, stream);
+  bool zg_applied = false;
+  st = attn_backward_impl(&bd, a + offQ, a + offK, a + offV, dav, da + offQ, da + offK,
+                          da + offV, d_rab_pos, d_rab_time, nullptr, ws, attn_ws, stream,
+                          SiluGradZ{z + offQ, z + offK, z + offV, n1}, &zg_applied);
   if (st != HSTU_OK) return st;
-  // ---- SiLU and f1: dZ = dA ⊙ SiLU'(Z) (in place), dX = dY + dZ W1ᵀ, dW1 = Xᵀ dZ, db1 = Σ dZ
-  e = launch_silu_grad_mul(z, n1, da, n1, da, n1, T, n1, nsm, s);
-  if (e != cudaSuccess) return cuda_fail(e);
+  // ---- SiLU and f1: dpre = dA ⊙ SiLU'(Z) (already applied to U, and to V, Q, K when the
+  // tensor-core backward produced them), dX = dY + dpre W1ᵀ, dW1 = Xᵀ dpre, db1 = Σ dpre
+  if (!zg_applied) {
+    e = launch_silu_grad_mul(z + offV, n1, da + offV, n1, da + offV, n1, T, n1 - hv, nsm, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   st = gemm_tc_layout(1, 0, 0, da, n1, w1, n1, T, dm, n1, 1, nullptr, d_y, dm, d_x, dm, nullptr,
                       0, nullptr, status, s);
   if (st != HSTU_OK) return st;

@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        __nv_bfloat16* __restrict__ dk_out, int64_t ld_dk,
                        __nv_bfloat16* __restrict__ dv_out, int64_t ld_dv,
                        float* __restrict__ dq_acc, int64_t ld_acc,
-                       float* __restrict__ d_pos, float* __restrict__ d_time) {
+                       float* __restrict__ d_pos, float* __restrict__ d_time, SiluGradZ zg) {
   const int nitems = *g.item_count;
   const int total = nitems * g.H;
   if (static_cast<int>(blockIdx.x) >= total) return;
@@ -516,6 +516,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_addr + (which ? kColDK : kColDV) + 32 * hq, a);
         tmem_wait_ld32(a);
         if (jvalid) {
+          // a layer's backward: dpre = dK (dV) ⊙ SiLU'(Z) before the one rounding to bf16
+          const float* zrow = which ? zg.k : zg.v;
+          if (zrow != nullptr) {
+            zrow += static_cast<int64_t>(it.row0 + jrow) * zg.ld + head * kD + 32 * hq;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 z4 = *reinterpret_cast<const float4*>(zrow + e);
+              a[e] = __float_as_uint(__uint_as_float(a[e]) * silu_grad_z(z4.x));
+              a[e + 1] = __float_as_uint(__uint_as_float(a[e + 1]) * silu_grad_z(z4.y));
+              a[e + 2] = __float_as_uint(__uint_as_float(a[e + 2]) * silu_grad_z(z4.z));
+              a[e + 3] = __float_as_uint(__uint_as_float(a[e + 3]) * silu_grad_z(z4.w));
+            }
+          }
           __nv_bfloat16* dst = (which ? dk_out : dv_out) +
                                static_cast<int64_t>(it.row0 + jrow) * (which ? ld_dk : ld_dv) +
                                head * kD + 32 * hq;
@@ -591,16 +604,25 @@ namespace hstu {
 namespace {
 // dQ accumulator (fp32, row stride ld_src) -> bf16 rows; 8 columns per thread (cols and ld_dst
 // multiples of 8, dst 16-byte aligned: checked by the caller).
+// With z (a layer's backward), the rows are first multiplied by SiLU'(z): dpre of the Q block.
 __global__ void f32_to_bf16_rows(const float* __restrict__ src, int64_t ld_src,
                                  __nv_bfloat16* __restrict__ dst, int64_t ld_dst, int rows,
-                                 int cols) {
+                                 int cols, const float* __restrict__ z, int64_t ld_z) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int per_row = cols / 8;
   if (idx >= static_cast<int64_t>(rows) * per_row) return;
   const int64_t r = idx / per_row;
   const int c = static_cast<int>(idx % per_row) * 8;
-  const float4 a = *reinterpret_cast<const float4*>(src + r * ld_src + c);
-  const float4 b = *reinterpret_cast<const float4*>(src + r * ld_src + c + 4);
+  float4 a = *reinterpret_cast<const float4*>(src + r * ld_src + c);
+  float4 b = *reinterpret_cast<const float4*>(src + r * ld_src + c + 4);
+  if (z != nullptr) {
+    const float4 za = *reinterpret_cast<const float4*>(z + r * ld_z + c);
+    const float4 zb = *reinterpret_cast<const float4*>(z + r * ld_z + c + 4);
+    a = make_float4(a.x * silu_grad_z(za.x), a.y * silu_grad_z(za.y), a.z * silu_grad_z(za.z),
+                    a.w * silu_grad_z(za.w));
+    b = make_float4(b.x * silu_grad_z(zb.x), b.y * silu_grad_z(zb.y), b.z * silu_grad_z(zb.z),
+                    b.w * silu_grad_z(zb.w));
+  }
   uint4 o;
   o.x = pack_bf16x2(a.x, a.y);
   o.y = pack_bf16x2(a.z, a.w);
@@ -630,7 +652,7 @@ cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                __nv_bfloat16* dq, int64_t ld_dq, __nv_bfloat16* dk,
                                int64_t ld_dk, __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc,
                                float* d_pos, float* d_time, int grid, bool fast,
-                               cudaStream_t stream) {
+                               const SiluGradZ& zg, cudaStream_t stream) {
   const size_t smem = attn_bwd_tc_smem(g.rab_pos ? g.P : 0, g.rab_time ? g.NB : 0);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   // d_pos / d_time are accumulated into: the caller zeroes them
@@ -641,12 +663,12 @@ cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, ld_dk, dv, ld_dv, dq_acc,
-                                           static_cast<int64_t>(g.H) * 64, d_pos, d_time);
+                                           static_cast<int64_t>(g.H) * 64, d_pos, d_time, zg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(g.T) * g.H * 8;  // 8 columns per thread
   f32_to_bf16_rows<<<static_cast<int>((n + 255) / 256), 256, 0, stream>>>(
-      dq_acc, static_cast<int64_t>(g.H) * 64, dq, ld_dq, g.T, g.H * 64);
+      dq_acc, static_cast<int64_t>(g.H) * 64, dq, ld_dq, g.T, g.H * 64, zg.q, zg.ld);
   return cudaGetLastError();
 }
 }  // namespace hstu

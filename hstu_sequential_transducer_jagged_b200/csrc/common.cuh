@@ -54,11 +54,28 @@ struct GemmArgs {
   int64_t ld_r;
   __nv_bfloat16* C;                // epi 0-3
   int64_t ldc;                     // row stride of C (or of Cf for epi 4)
-  __nv_bfloat16* C2;               // epi 3: the pre-activation
+  float* C2;                       // epi 3: the pre-activation (fp32)
   int64_t ld_c2;
   float* Cf;                       // epi 4: fp32 [M, N], accumulated into
   int* status;
 };
+
+// SiLU' factors for a backward that produces dpre = dA ⊙ SiLU'(Z) directly: fp32 pre-activation
+// columns of the Q, K, V (and U) blocks, row stride ld (elements); q == nullptr: none.
+struct SiluGradZ {
+  const float* q;
+  const float* k;
+  const float* v;
+  int64_t ld;
+};
+
+// SiLU'(z) = σ(z) (1 + z (1 - σ(z))), σ(z) = (1 + tanh(z / 2)) / 2.
+__device__ __forceinline__ float silu_grad_z(float z) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+  const float sg = fmaf(0.5f, t, 0.5f);
+  return sg * fmaf(z, 1.f - sg, 1.f);
+}
 
 // History length n of a sequence: every token for the causal mask, L - m under M-FALCON.
 __host__ __device__ __forceinline__ int hist_len(int L, int mask, int m) {

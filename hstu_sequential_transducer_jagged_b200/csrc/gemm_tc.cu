@@ -59,7 +59,8 @@ __device__ __forceinline__ float silu_fast(float x) {
 //   EPI 0: C = SiLU(acc + bias)                       (bf16)
 //   EPI 1: C = acc + bias + R                         (bf16, residual R [M, N] with ld_r)
 //   EPI 2: C = acc + bias                             (bf16)
-//   EPI 3: C = SiLU(acc + bias) and C2 = acc + bias   (bf16, C2 with ld_c2: the pre-activation)
+//   EPI 3: C = SiLU(acc + bias) and C2 = acc + bias   (bf16 C; fp32 C2 with ld_c2: the
+//          pre-activation the backward's SiLU' reads)
 //   EPI 4: Cf += acc                                  (fp32, atomic: split-K partial sums)
 // With k_splits > 1 each output tile is computed by k_splits work units over consecutive K
 // ranges (EPI 4 only).
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         int k_splits, const float* __restrict__ bias,
                         const __nv_bfloat16* __restrict__ resid, int64_t ld_r,
                         __nv_bfloat16* __restrict__ C, int64_t ldc,
-                        __nv_bfloat16* __restrict__ C2, int64_t ld_c2, float* __restrict__ Cf,
+                        float* __restrict__ C2, int64_t ld_c2, float* __restrict__ Cf,
                         int* status) {
   if (*reinterpret_cast<volatile int*>(status) == kStatusTimeout) return;
   extern __shared__ uint8_t smem_raw[];
@@ -242,21 +243,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (bias != nullptr && c < N) x += __ldg(bias + c);
             vals[e] = x;
           }
-          if (EPI == 3) {  // the pre-activation, before the SiLU overwrites vals
-            __nv_bfloat16* pp = C2 + static_cast<int64_t>(row) * ld_c2 + c0;
+          if (EPI == 3) {  // the fp32 pre-activation, before the SiLU overwrites vals
+            float* pp = C2 + static_cast<int64_t>(row) * ld_c2 + c0;
             if (c0 + 32 <= N) {
 #pragma unroll
-              for (int w = 0; w < 4; ++w) {
-                uint4 ov;
-                ov.x = pack_bf16x2(vals[8 * w + 0], vals[8 * w + 1]);
-                ov.y = pack_bf16x2(vals[8 * w + 2], vals[8 * w + 3]);
-                ov.z = pack_bf16x2(vals[8 * w + 4], vals[8 * w + 5]);
-                ov.w = pack_bf16x2(vals[8 * w + 6], vals[8 * w + 7]);
-                reinterpret_cast<uint4*>(pp)[w] = ov;
-              }
+              for (int w = 0; w < 8; ++w)
+                reinterpret_cast<float4*>(pp)[w] = make_float4(vals[4 * w], vals[4 * w + 1],
+                                                               vals[4 * w + 2], vals[4 * w + 3]);
             } else {
               for (int e = 0; e < 32; ++e)
-                if (c0 + e < N) pp[e] = __float2bfloat16_rn(vals[e]);
+                if (c0 + e < N) pp[e] = vals[e];
             }
           }
           if (EPI == 1) {

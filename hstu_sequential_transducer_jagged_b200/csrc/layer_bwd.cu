@@ -80,6 +80,7 @@ __global__ void ln_gate_bwd_kernel(const __nv_bfloat16* __restrict__ av, int64_t
                                    const float* __restrict__ gamma, const float* __restrict__ beta,
                                    float eps, __nv_bfloat16* __restrict__ d_av, int64_t ld_dav,
                                    __nv_bfloat16* __restrict__ d_u, int64_t ld_du,
+                                   const float* __restrict__ z_u, int64_t ld_z,
                                    float* __restrict__ d_gamma, float* __restrict__ d_beta,
                                    int rows) {
   constexpr int F = 32 * PER;
@@ -124,6 +125,17 @@ __global__ void ln_gate_bwd_kernel(const __nv_bfloat16* __restrict__ av, int64_t
       s1 += fg[e];
       s2 += fg[e] * n;
     }
+    if (z_u != nullptr) {  // dpre of the U block: dU ⊙ SiLU'(Z_U), rounded once
+      const float* zr = z_u + static_cast<int64_t>(r) * ld_z + c0;
+#pragma unroll
+      for (int e = 0; e < PER; e += 4) {
+        const float4 z4 = *reinterpret_cast<const float4*>(zr + e);
+        du[e] *= silu_grad_z(z4.x);
+        du[e + 1] *= silu_grad_z(z4.y);
+        du[e + 2] *= silu_grad_z(z4.z);
+        du[e + 3] *= silu_grad_z(z4.w);
+      }
+    }
     store_row<PER>(d_u + static_cast<int64_t>(r) * ld_du + c0, du);
     const float m1 = warp_sum(s1) / F, m2 = warp_sum(s2) / F;
 #pragma unroll
@@ -139,9 +151,9 @@ __global__ void ln_gate_bwd_kernel(const __nv_bfloat16* __restrict__ av, int64_t
   }
 }
 
-// dz = da ⊙ SiLU'(z), SiLU'(z) = σ(z) (1 + z (1 - σ(z))), σ(z) = (1 + tanh(z/2)) / 2; rows x
-// cols bf16 (cols a multiple of 8, 16-byte aligned rows); dz may alias da.
-__global__ void silu_grad_mul_kernel(const __nv_bfloat16* __restrict__ z, int64_t ld_z,
+// dz = da ⊙ SiLU'(z), SiLU'(z) = σ(z) (1 + z (1 - σ(z))), σ(z) = (1 + tanh(z/2)) / 2; z fp32,
+// da / dz bf16, rows x cols (cols a multiple of 8, 16-byte aligned rows); dz may alias da.
+__global__ void silu_grad_mul_kernel(const float* __restrict__ z, int64_t ld_z,
                                      const __nv_bfloat16* da, int64_t ld_da, __nv_bfloat16* dz,
                                      int64_t ld_dz, int rows, int cols) {
   const int per_row = cols / kVec;
@@ -150,14 +162,13 @@ __global__ void silu_grad_mul_kernel(const __nv_bfloat16* __restrict__ z, int64_
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = idx / per_row;
     const int c = static_cast<int>(idx % per_row) * kVec;
-    float fz[8], fa[8], o[8];
-    load8(z + r * ld_z + c, fz);
+    float fa[8], o[8];
     load8(da + r * ld_da + c, fa);
+    const float4 z0 = *reinterpret_cast<const float4*>(z + r * ld_z + c);
+    const float4 z1 = *reinterpret_cast<const float4*>(z + r * ld_z + c + 4);
+    const float fz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float sg = fmaf(0.5f, tanh_fast(0.5f * fz[e]), 0.5f);
-      o[e] = fa[e] * sg * fmaf(fz[e], 1.f - sg, 1.f);
-    }
+    for (int e = 0; e < 8; ++e) o[e] = fa[e] * silu_grad_z(fz[e]);
     store8(dz + r * ld_dz + c, o);
   }
 }
@@ -181,8 +192,9 @@ cudaError_t launch_ln_gate_bwd(const __nv_bfloat16* av, int64_t ld_av, const __n
                                int64_t ld_u, const __nv_bfloat16* dg, int64_t ld_dg,
                                const float* gamma, const float* beta, float eps,
                                __nv_bfloat16* d_av, int64_t ld_dav, __nv_bfloat16* d_u,
-                               int64_t ld_du, float* d_gamma, float* d_beta, int rows, int F,
-                               int num_sms, cudaStream_t stream) {
+                               int64_t ld_du, const float* z_u, int64_t ld_z, float* d_gamma,
+                               float* d_beta, int rows, int F, int num_sms,
+                               cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
   const int threads = 256;
   int blocks = (rows * 32 + threads - 1) / threads;
@@ -191,7 +203,7 @@ cudaError_t launch_ln_gate_bwd(const __nv_bfloat16* av, int64_t ld_av, const __n
 #define HSTU_LN_BWD(PER)                                                                    \
   ln_gate_bwd_kernel<PER><<<blocks, threads, 0, stream>>>(av, ld_av, u, ld_u, dg, ld_dg, gamma, \
                                                           beta, eps, d_av, ld_dav, d_u, ld_du, \
-                                                          d_gamma, d_beta, rows)
+                                                          z_u, ld_z, d_gamma, d_beta, rows)
   switch (F) {
     case 128: HSTU_LN_BWD(4); break;
     case 256: HSTU_LN_BWD(8); break;
@@ -203,7 +215,7 @@ cudaError_t launch_ln_gate_bwd(const __nv_bfloat16* av, int64_t ld_av, const __n
   return cudaGetLastError();
 }
 
-cudaError_t launch_silu_grad_mul(const __nv_bfloat16* z, int64_t ld_z, const __nv_bfloat16* da,
+cudaError_t launch_silu_grad_mul(const float* z, int64_t ld_z, const __nv_bfloat16* da,
                                  int64_t ld_da, __nv_bfloat16* dz, int64_t ld_dz, int rows,
                                  int cols, int num_sms, cudaStream_t stream) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
