@@ -82,8 +82,8 @@ cudaError_t launch_scatter_rows(const void* src, int64_t src_stride, const int32
                                 void* dst, int64_t dst_stride, int64_t row_bytes, int num_sms,
                                 cudaStream_t stream);
 bool f2_fused_supported(int F, int N);
-cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_w2, int M, int N,
-                            int F, const __nv_bfloat16* u, int64_t ld_u, const float* gamma,
+cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_u,
+                            const CUtensorMap& tm_w2, int M, int N, int F, const float* gamma,
                             const float* beta, float eps, const float* bias,
                             const __nv_bfloat16* x, int64_t ld_x, __nv_bfloat16* y, int64_t ld_y,
                             int* status, int num_sms, cudaStream_t stream);
@@ -370,14 +370,15 @@ hstu_status_t norm_gate_f2(int dtype, const void* av, int64_t ld_av, const void*
                      ld_u % 8 == 0 && d_model % 8 == 0 && aligned16(av) && aligned16(u) &&
                      aligned16(w2) && aligned16(x) && aligned16(y);
   if (fused) {
-    CUtensorMap tav, tw2;
+    CUtensorMap tav, tu, tw2;
     if (!make_map_bf16(&tav, av, rows, F, ld_av, 64, 128) ||
+        !make_map_bf16(&tu, u, rows, F, ld_u, 64, 128) ||
         !make_map_bf16(&tw2, w2, F, d_model, d_model, 64, 64))
       return HSTU_ERR_CUDA;
     const cudaError_t e = launch_f2_fused(
-        tav, tw2, rows, d_model, F, static_cast<const __nv_bfloat16*>(u), ld_u, gamma, beta, eps,
-        b2, static_cast<const __nv_bfloat16*>(x), d_model, static_cast<__nv_bfloat16*>(y),
-        d_model, status, num_sms_current(), s);
+        tav, tu, tw2, rows, d_model, F, gamma, beta, eps, b2,
+        static_cast<const __nv_bfloat16*>(x), d_model, static_cast<__nv_bfloat16*>(y), d_model,
+        status, num_sms_current(), s);
     return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
   }
   if (launch_ln_gate(dtype == HSTU_BF16 ? 0 : 1, av, ld_av, u, ld_u, gamma, beta, eps, g_buf, F,

@@ -6,10 +6,11 @@
 // Persistent CTAs walk 128-row blocks of tokens.  Per block:
 //   warp 0      TMA: the block's AV rows [128, F] (F = H d_v <= 512) into shared memory, as
 //               F / 64 K-major 128-byte-swizzled slots of [128 rows][64 features] — already the
-//               A operand's layout; then W2 tiles [64 k][256 n] through a 3-stage ring;
+//               A operand's layout; the matching U slots (same swizzle) through a 2-slot ring;
+//               then W2 tiles [64 k][256 n] through a 2-stage ring;
 //   warps 2-5   one token row per thread: mean and biased variance of the row from shared memory
-//               (two passes), then G = ((AV - mean) rstd γ + β) ⊙ U written in place as bf16
-//               (U read from the f1 output), fenced for the tensor core's async proxy;
+//               (two passes), then, slot by slot as U arrives, G = ((AV - mean) rstd γ + β) ⊙ U
+//               written in place as bf16, fenced for the tensor core's async proxy;
 //   warp 1      tcgen05.mma: for each 256-wide output tile, F / 64 K blocks of four 128x256x16
 //               MMAs into one of two TMEM accumulators (2 x 256 columns);
 //   warps 6-13  epilogue: TMEM -> + b2 + X -> bf16 Y, one row per thread, 128 columns per warp.
@@ -27,14 +28,17 @@ constexpr int kTileN = 256;
 constexpr int kKB = 64;
 constexpr int kSlotBytes = kRows * kKB * 2;   // 16 KB: one K block of G
 constexpr int kBStageBytes = kKB * kTileN * 2; // 32 KB: four [64 k][64 n] boxes of W2
-constexpr int kBStages = 3;
+constexpr int kBStages = 2;
+constexpr int kUSlots = 2;
 constexpr int kMaxF = 512;                     // 8 slots: 128 KB
 constexpr int kThreads = 448;                  // 14 warps
 
 struct F2Smem {
   alignas(1024) uint8_t g[kMaxF / kKB][kSlotBytes];
+  alignas(1024) uint8_t u[kUSlots][kSlotBytes];
   alignas(1024) uint8_t b[kBStages][kBStageBytes];
   uint64_t g_loaded, g_ready, g_free;
+  uint64_t u_full[kUSlots], u_empty[kUSlots];
   uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
@@ -58,8 +62,8 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& raw, float (&f)[8]) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     f2_fused_kernel(const __grid_constant__ CUtensorMap tm_av,
+                    const __grid_constant__ CUtensorMap tm_u,
                     const __grid_constant__ CUtensorMap tm_w2, int M, int N, int F,
-                    const __nv_bfloat16* __restrict__ u, int64_t ld_u,
                     const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ x,
                     int64_t ld_x, __nv_bfloat16* __restrict__ y, int64_t ld_y, int* status) {
@@ -80,6 +84,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&sm.b_full[s], 1);
       mbar_init(&sm.b_empty[s], 1);
+    }
+    for (int s = 0; s < kUSlots; ++s) {
+      mbar_init(&sm.u_full[s], 1);
+      mbar_init(&sm.u_empty[s], 4);  // one elected lane per transform warp
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.acc_full[a], 1);
@@ -103,8 +111,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_av);
+      tma_prefetch_desc(&tm_u);
       tma_prefetch_desc(&tm_w2);
-      int it = 0, g = 0;  // blocks, W2 stages issued
+      int it = 0, g = 0, gu = 0;  // blocks, W2 stages and U slots issued
+      int av_issued = 0;          // blocks whose AV slots were requested
       bool ok = true;
       for (int blk = blockIdx.x; ok && blk < blocks; blk += stride, ++it) {
         // the previous block's MMAs have read G
@@ -115,6 +125,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sm.g_loaded, nkb * kSlotBytes);
         for (int kb = 0; kb < nkb; ++kb)
           tma_load_2d(sm.g[kb], &tm_av, &sm.g_loaded, kb * kKB, blk * kRows);
+        ++av_issued;
+        for (int kb = 0; kb < nkb; ++kb, ++gu) {
+          const int su = gu % kUSlots;
+          if (gu >= kUSlots &&
+              !mbar_wait(&sm.u_empty[su], ((gu / kUSlots) - 1) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.u_full[su], kSlotBytes);
+          tma_load_2d(sm.u[su], &tm_u, &sm.u_full[su], kb * kKB, blk * kRows);
+        }
+        if (!ok) break;
         for (int nt = 0; ok && nt < n_tiles; ++nt) {
           for (int kb = 0; kb < nkb; ++kb, ++g) {
             const int st = g % kBStages;
@@ -134,7 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {  // leave no TMA write in flight into shared memory about to be released
         for (int k2 = (g > kBStages ? g - kBStages : 0); k2 < g; ++k2)
           mbar_wait(&sm.b_full[k2 % kBStages], (k2 / kBStages) & 1, nullptr, nullptr);
-        if (it > 0) mbar_wait(&sm.g_loaded, (it - 1) & 1, nullptr, nullptr);
+        for (int k2 = (gu > kUSlots ? gu - kUSlots : 0); k2 < gu; ++k2)
+          mbar_wait(&sm.u_full[k2 % kUSlots], (k2 / kUSlots) & 1, nullptr, nullptr);
+        if (av_issued > 0) mbar_wait(&sm.g_loaded, (av_issued - 1) & 1, nullptr, nullptr);
       }
     }
     __syncwarp();
@@ -187,15 +211,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------------------- Norm(AV) ⊙ U
     const int r = (warp - 2) * 32 + lane;  // row of the block
     const int sw = r & 7;                   // 128-byte swizzle: chunk c sits at c ^ (r & 7)
-    int it = 0;
+    int it = 0, gu = 0;
     bool ok = true;
     for (int blk = blockIdx.x; ok && blk < blocks; blk += stride, ++it) {
       ok = warp_all(lane == 0 ? mbar_wait(&sm.g_loaded, it & 1, abort_flag, status) : true);
       if (!ok) break;
       // (every lane observes the TMA writes: the waiting lane acquired them, the vote orders
       // the warp)
-      const int row = blk * kRows + r;
-      const bool valid = row < M;
       float sum = 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
         const uint8_t* base = sm.g[kb] + r * 128;
@@ -223,21 +245,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const float rstd = rsqrtf(sq / F + eps);
-      const __nv_bfloat16* urow = u + static_cast<int64_t>(valid ? row : 0) * ld_u;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = 0; kb < nkb && ok; ++kb, ++gu) {
+        const int su = gu % kUSlots;
+        ok = warp_all(lane == 0 ? mbar_wait(&sm.u_full[su], (gu / kUSlots) & 1, abort_flag,
+                                            status)
+                                : true);
+        if (!ok) break;
         uint8_t* base = sm.g[kb] + r * 128;
+        const uint8_t* ubase = sm.u[su] + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint4* slot = reinterpret_cast<uint4*>(base + ((c ^ sw) << 4));
           const int col = kb * kKB + c * 8;
           float f[8], fu[8];
           bf16x8_to_f(*slot, f);
-          if (valid) {
-            bf16x8_to_f(*reinterpret_cast<const uint4*>(urow + col), fu);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) fu[e] = 0.f;
-          }
+          // U past the last token is zero (TMA fill), so G is zero there too
+          bf16x8_to_f(*reinterpret_cast<const uint4*>(ubase + ((c ^ sw) << 4)), fu);
           float o[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -253,7 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.w = pack_bf16x2(o[6], o[7]);
           *slot = w;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.u_empty[su]);  // this warp is done with the U slot
       }
+      if (!ok) break;
       fence_async_smem();  // G is read by the MMAs (async proxy)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.g_ready);
@@ -335,8 +361,8 @@ bool f2_fused_supported(int F, int N) {
   return F % kKB == 0 && F >= kKB && F <= kMaxF && N % 8 == 0 && f2_fused_smem() <= 227 * 1024;
 }
 
-cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_w2, int M, int N,
-                            int F, const __nv_bfloat16* u, int64_t ld_u, const float* gamma,
+cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_u,
+                            const CUtensorMap& tm_w2, int M, int N, int F, const float* gamma,
                             const float* beta, float eps, const float* bias,
                             const __nv_bfloat16* x, int64_t ld_x, __nv_bfloat16* y, int64_t ld_y,
                             int* status, int num_sms, cudaStream_t stream) {
@@ -348,7 +374,7 @@ cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_w2, 
   if (e != cudaSuccess) return e;
   const int blocks = (M + kRows - 1) / kRows;
   const int grid = blocks < num_sms ? blocks : num_sms;
-  f2_fused_kernel<<<grid, kThreads, smem, stream>>>(tm_av, tm_w2, M, N, F, u, ld_u, gamma, beta,
+  f2_fused_kernel<<<grid, kThreads, smem, stream>>>(tm_av, tm_u, tm_w2, M, N, F, gamma, beta,
                                                    eps, bias, x, ld_x, y, ld_y, status);
   return cudaGetLastError();
 }

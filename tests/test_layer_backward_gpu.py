@@ -3,7 +3,12 @@
 Gradients of L = Σ dY ⊙ Y through Y = X + f2(Norm(A(X)V(X)) ⊙ U(X)) ("万亿参数推荐大模型：HSTU 架构
 如何超越传统 Self-Attention" §2.1; the training pass of "HSTU：Scaling Law 的首次探索" §7.1.3).
 Same tolerance as the other parity tests: per element |err| <= 2e-2 max|ref row| + 1e-3 and
-relative Frobenius error <= 5e-3 (bias and weight gradients are compared as whole arrays).
+relative Frobenius error <= 5e-3 (bias and weight gradients are compared as whole arrays), except
+the relative Frobenius bound of the two bias-table gradients, 1e-2: in a layer the attention
+backward's tensor-core operands dO = dAV and Q, K, V are bf16 roundings of intermediate results
+(relative error up to 2^-9 each, which the fp64 oracle does not have), and a table entry sums
+dS over up to ~10^5 pairs of both signs, so it keeps the ~3 x 2^-9 relative error of its terms
+instead of averaging it away.
 """
 import numpy as np
 import pytest
@@ -11,9 +16,12 @@ import torch
 
 from oracle import hstu_oracle as O
 from hstu_sequential_transducer_jagged_b200 import workloads as W
+import test_gpu_parity as P
 from test_gpu_parity import B, assert_close, dev  # noqa: F401
 
 pytestmark = pytest.mark.gpu
+
+TABLE_FRO_TOL = 1e-2  # bias-table gradients of the layer backward (module docstring)
 
 NAMES = ("dx", "dw1", "db1", "dw2", "db2", "d_rab_pos", "d_rab_time", "d_ln_gamma", "d_ln_beta")
 
@@ -45,7 +53,15 @@ def _compare(got, ref, what):
     for name in NAMES:
         if ref.get(name) is None or got.get(name) is None:
             continue
-        assert_close(got[name], ref[name], f"{what} {name}")
+        if name in ("d_rab_pos", "d_rab_time"):
+            saved = P.FRO_TOL
+            P.FRO_TOL = TABLE_FRO_TOL
+            try:
+                assert_close(got[name], ref[name], f"{what} {name}")
+            finally:
+                P.FRO_TOL = saved
+        else:
+            assert_close(got[name], ref[name], f"{what} {name}")
 
 
 @pytest.mark.parametrize("mask,m", [(W.MASK_CAUSAL, 0), (W.MASK_MFALCON, 60)])
