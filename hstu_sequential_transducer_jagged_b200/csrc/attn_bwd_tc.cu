@@ -187,22 +187,15 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
   return kChunkConst;
 }
 
-// Position-table index and time bucket of the pair (query i, this thread's key row).
-__device__ __forceinline__ int chunk_pidx(int i, const BwdRow& r, const BwdTabs& t) {
-  return pos_index_direct(i < r.n ? i : r.n, r.pj, t.P);
-}
-
 // One 32-column block of a key row: P and alpha dS (bf16 pairs) from S and dP, and the bias
-// gradients.  i_first: query index of the block's first column; tq_c: its timestamps.  Pass 1
-// computes P and dS of all 32 columns without branches, so their 32 dependency chains can
-// interleave; pass 2 adds dS to the gradient bins (run-length sums, shared-memory atomics when
-// the table index changes).  dS replaces dP in dp (fp32 bits).
+// gradients.  i_first: query index of the block's first column; tq_c: its timestamps.
 template <int V>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], uint32_t (&dp)[32],
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
                                           uint32_t (&pk)[16], uint32_t (&dk)[16], int i_first,
                                           const long long* tq_c, const BwdRow& r,
                                           const BwdTabs& t, float cbias, int cpidx, int ctidx,
                                           BinRun& run_p, BinRun& run_t) {
+  float sum = 0.f;  // constant classes: the block's dS total for the constant bins
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float pv[2], dsa[2];
@@ -210,14 +203,21 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], uint32_t (&dp
     for (int u = 0; u < 2; ++u) {
       const int i = i_first + e + u;
       float bias;
+      int pidx = 0, bidx = 0;
       if (V == kChunkConst) {
         bias = cbias;
       } else {
-        bias = t.use_pos ? t.pos[chunk_pidx(i, r, t)] : 0.f;
+        bias = 0.f;
+        if (t.use_pos) {
+          const int pi = i < r.n ? i : r.n;
+          pidx = pos_index_direct(pi, r.pj, t.P);
+          bias += t.pos[pidx];
+        }
         if (V == kChunkTimeConst) {
           bias += cbias;
         } else if (t.use_time) {
-          bias += t.time[time_bucket64(tq_c[e + u] - r.tj, t.NB)];
+          bidx = time_bucket64(tq_c[e + u] - r.tj, t.NB);
+          bias += t.time[bidx];
         }
       }
       const float x = fmaf(t.alpha, __uint_as_float(s[e + u]), bias);
@@ -228,34 +228,20 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], uint32_t (&dp
         const bool vis = r.jvalid && i < r.L && r.jrow <= i && (r.jrow < r.n || r.jrow == i);
         p = vis ? p : 0.f;
         dsv = vis ? dsv : 0.f;
+        if (vis && t.use_pos) run_p.add(t.bins_pos, pidx, dsv);
+        if (vis && t.use_time) run_t.add(t.bins_time, bidx, dsv);
+      } else {
+        if (V == kChunkTimeConst && t.use_pos) run_p.add(t.bins_pos, pidx, dsv);
+        sum += dsv;
       }
       pv[u] = p;
       dsa[u] = t.alpha * dsv;
-      dp[e + u] = __float_as_uint(dsv);
     }
     pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
     dk[e >> 1] = pack_bf16x2(dsa[0], dsa[1]);
   }
-  // pass 2: bias-table gradients (hidden pairs carry dS = 0 and add nothing)
-  if (V == kChunkGeneral) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float dsv = __uint_as_float(dp[e]);
-      if (t.use_pos) run_p.add(t.bins_pos, chunk_pidx(i_first + e, r, t), dsv);
-      if (t.use_time) run_t.add(t.bins_time, time_bucket64(tq_c[e] - r.tj, t.NB), dsv);
-    }
-  } else {
-    float sum = 0.f;  // the block's dS total for its constant bins
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float dsv = __uint_as_float(dp[e]);
-      sum += dsv;
-      if (V == kChunkTimeConst && t.use_pos)
-        run_p.add(t.bins_pos, chunk_pidx(i_first + e, r, t), dsv);
-    }
-    if (V == kChunkConst && t.use_pos) run_p.add(t.bins_pos, cpidx, sum);
-    if (t.use_time) run_t.add(t.bins_time, ctidx, sum);
-  }
+  if (V == kChunkConst && t.use_pos) run_p.add(t.bins_pos, cpidx, sum);
+  if (V != kChunkGeneral && t.use_time) run_t.add(t.bins_time, ctidx, sum);
 }
 
 // Items: (sequence, 128-row key tile) from the work list built with one tile per item, times heads.
@@ -486,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int z = 0; z < 16; ++z) pk[z] = dk[z] = 0u;
           } else {
-            uint32_t s[32], dp[32];  // dp becomes dS in bwd_chunk
+            uint32_t s[32], dp[32];
             tmem_ld32(lane_addr + kColST + col, s);
             tmem_ld32(lane_addr + kColDPT + col, dp);
             tmem_wait_ld32(s);

@@ -3,19 +3,22 @@
 // ("万亿参数推荐大模型：HSTU 架构如何超越传统 Self-Attention" §2.1, third formula Y = f2(Norm(AV) ⊙ U)
 // and the block diagram's residual edge; "HSTU：Scaling Law 的首次探索" §7.1.4 innovation 3.)
 //
-// Persistent CTAs walk 128-row blocks of tokens.  Per block:
-//   warp 0      TMA: the block's AV rows [128, F] (F = H d_v <= 512) into shared memory, as
-//               F / 64 K-major 128-byte-swizzled slots of [128 rows][64 features] — already the
-//               A operand's layout; the matching U slots (same swizzle) through a 2-slot ring;
-//               then W2 tiles [64 k][256 n] through a 2-stage ring;
-//   warps 2-5   one token row per thread: mean and biased variance of the row from shared memory
-//               (two passes), then, slot by slot as U arrives, G = ((AV - mean) rstd γ + β) ⊙ U
-//               written in place as bf16, fenced for the tensor core's async proxy;
-//   warp 1      tcgen05.mma: for each 256-wide output tile, F / 64 K blocks of four 128x256x16
-//               MMAs into one of two TMEM accumulators (2 x 256 columns);
-//   warps 6-13  epilogue: TMEM -> + b2 + X -> bf16 Y, one row per thread, 128 columns per warp.
-// The next block's AV load waits for this block's last MMA (one G buffer); the accumulators are
-// double-buffered, so the epilogue of one tile overlaps the MMAs of the next.
+// Persistent CTAs walk 128-row blocks of tokens.  The block's AV rows [128, F] (F = H d_v <= 512)
+// sit in F / 64 K-major, 128-byte-swizzled slots of [128 rows][64 features] — already the MMA's
+// A-operand layout — and each slot turns into the matching slot of G in place:
+//   warp 0      TMA: AV slot kb of the next block as soon as this block's MMAs have read slot kb;
+//               U slots (same swizzle) through a 2-slot ring; W2 tiles [64 k][256 n] through a
+//               2-stage ring, interleaved with the U slots in K order;
+//   warps 2-5   one token row per thread: mean and biased variance of the row over all slots
+//               (two passes over shared memory), then slot by slot as U arrives,
+//               G = ((AV - mean) rstd γ + β) ⊙ U written in place as bf16, fenced for the
+//               tensor core's async proxy, and published per slot;
+//   warp 1      tcgen05.mma: K block kb of G against both 256-wide halves of W2 (N <= 512) into
+//               two TMEM accumulators (2 x 256 columns); the slot is released after both;
+//   warps 6-13  epilogue: TMEM -> + b2 + X -> bf16 Y, one row per thread, 128 of every 256
+//               columns per warp; the accumulators are free again for the next block after it.
+// So the next block's AV streams in while this block's MMAs run, and its statistics overlap this
+// block's epilogue.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -26,21 +29,25 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kTileN = 256;
 constexpr int kKB = 64;
-constexpr int kSlotBytes = kRows * kKB * 2;   // 16 KB: one K block of G
-constexpr int kBStageBytes = kKB * kTileN * 2; // 32 KB: four [64 k][64 n] boxes of W2
+constexpr int kSlotBytes = kRows * kKB * 2;     // 16 KB: one K block of AV / G
+constexpr int kBStageBytes = kKB * kTileN * 2;  // 32 KB: four [64 k][64 n] boxes of W2
 constexpr int kBStages = 2;
 constexpr int kUSlots = 2;
-constexpr int kMaxF = 512;                     // 8 slots: 128 KB
-constexpr int kThreads = 448;                  // 14 warps
+constexpr int kMaxF = 512;                      // 8 slots: 128 KB
+constexpr int kMaxSlots = kMaxF / kKB;
+constexpr int kMaxN = 2 * kTileN;               // two TMEM accumulators
+constexpr int kThreads = 448;                   // 14 warps
 
 struct F2Smem {
-  alignas(1024) uint8_t g[kMaxF / kKB][kSlotBytes];
+  alignas(1024) uint8_t g[kMaxSlots][kSlotBytes];
   alignas(1024) uint8_t u[kUSlots][kSlotBytes];
   alignas(1024) uint8_t b[kBStages][kBStageBytes];
-  uint64_t g_loaded, g_ready, g_free;
+  uint64_t av_full[kMaxSlots];    // TMA: slot kb holds the block's AV
+  uint64_t g_ready[kMaxSlots];    // transform warps: slot kb holds G
+  uint64_t slot_free[kMaxSlots];  // MMA: slot kb has been read (both halves)
   uint64_t u_full[kUSlots], u_empty[kUSlots];
   uint64_t b_full[kBStages], b_empty[kBStages];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -60,6 +67,13 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& raw, float (&f)[8]) {
   }
 }
 
+// Lane 0 waits, the warp follows (every lane then sees what the barrier published).
+__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              int* status) {
+  const int lane = threadIdx.x & 31;
+  return warp_all(lane == 0 ? mbar_wait(bar, parity, abort, status) : true);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     f2_fused_kernel(const __grid_constant__ CUtensorMap tm_av,
                     const __grid_constant__ CUtensorMap tm_u,
@@ -73,26 +87,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = F / kKB;
-  const int n_tiles = (N + kTileN - 1) / kTileN;
+  const int n_halves = (N + kTileN - 1) / kTileN;  // 1 or 2
   const int blocks = (M + kRows - 1) / kRows;
   const int stride = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.g_loaded, 1);
-    mbar_init(&sm.g_ready, 4);  // one elected lane per transform warp
-    mbar_init(&sm.g_free, 1);
+    for (int s = 0; s < kMaxSlots; ++s) {
+      mbar_init(&sm.av_full[s], 1);
+      mbar_init(&sm.g_ready[s], 4);  // one elected lane per transform warp
+      mbar_init(&sm.slot_free[s], 1);
+    }
+    for (int s = 0; s < kUSlots; ++s) {
+      mbar_init(&sm.u_full[s], 1);
+      mbar_init(&sm.u_empty[s], 4);
+    }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&sm.b_full[s], 1);
       mbar_init(&sm.b_empty[s], 1);
     }
-    for (int s = 0; s < kUSlots; ++s) {
-      mbar_init(&sm.u_full[s], 1);
-      mbar_init(&sm.u_empty[s], 4);  // one elected lane per transform warp
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&sm.acc_full[a], 1);
-      mbar_init(&sm.acc_empty[a], 8);
-    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.acc_empty, 8);  // one elected lane per epilogue warp
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
@@ -114,19 +128,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_u);
       tma_prefetch_desc(&tm_w2);
       int it = 0, g = 0, gu = 0;  // blocks, W2 stages and U slots issued
-      int av_issued = 0;          // blocks whose AV slots were requested
+      int av_slots = 0;           // AV slot loads issued
       bool ok = true;
       for (int blk = blockIdx.x; ok && blk < blocks; blk += stride, ++it) {
-        // the previous block's MMAs have read G
-        if (it > 0 && !mbar_wait(&sm.g_free, (it - 1) & 1, abort_flag, status)) {
-          ok = false;
-          break;
+        for (int kb = 0; kb < nkb; ++kb) {
+          // the previous block's MMAs have read slot kb
+          if (it > 0 && !mbar_wait(&sm.slot_free[kb], (it - 1) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.av_full[kb], kSlotBytes);
+          tma_load_2d(sm.g[kb], &tm_av, &sm.av_full[kb], kb * kKB, blk * kRows);
+          ++av_slots;
         }
-        mbar_arrive_expect_tx(&sm.g_loaded, nkb * kSlotBytes);
-        for (int kb = 0; kb < nkb; ++kb)
-          tma_load_2d(sm.g[kb], &tm_av, &sm.g_loaded, kb * kKB, blk * kRows);
-        ++av_issued;
-        for (int kb = 0; kb < nkb; ++kb, ++gu) {
+        for (int kb = 0; ok && kb < nkb; ++kb) {
           const int su = gu % kUSlots;
           if (gu >= kUSlots &&
               !mbar_wait(&sm.u_empty[su], ((gu / kUSlots) - 1) & 1, abort_flag, status)) {
@@ -135,10 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&sm.u_full[su], kSlotBytes);
           tma_load_2d(sm.u[su], &tm_u, &sm.u_full[su], kb * kKB, blk * kRows);
-        }
-        if (!ok) break;
-        for (int nt = 0; ok && nt < n_tiles; ++nt) {
-          for (int kb = 0; kb < nkb; ++kb, ++g) {
+          ++gu;
+          for (int h = 0; h < n_halves; ++h, ++g) {
             const int st = g % kBStages;
             if (g >= kBStages &&
                 !mbar_wait(&sm.b_empty[st], ((g / kBStages) - 1) & 1, abort_flag, status)) {
@@ -149,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < kTileN / 64; ++q)
               tma_load_2d(sm.b[st] + q * (kKB * 128), &tm_w2, &sm.b_full[st],
-                          nt * kTileN + 64 * q, kb * kKB);
+                          h * kTileN + 64 * q, kb * kKB);
           }
         }
       }
@@ -158,7 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&sm.b_full[k2 % kBStages], (k2 / kBStages) & 1, nullptr, nullptr);
         for (int k2 = (gu > kUSlots ? gu - kUSlots : 0); k2 < gu; ++k2)
           mbar_wait(&sm.u_full[k2 % kUSlots], (k2 / kUSlots) & 1, nullptr, nullptr);
-        if (av_issued > 0) mbar_wait(&sm.g_loaded, (av_issued - 1) & 1, nullptr, nullptr);
+        // the last load of each slot (loads go to slots 0, 1, .., nkb - 1, 0, 1, ..)
+        for (int s = 0; s < nkb && s < av_slots; ++s) {
+          const int loads = (av_slots - 1 - s) / nkb + 1;
+          mbar_wait(&sm.av_full[s], (loads - 1) & 1, nullptr, nullptr);
+        }
       }
     }
     __syncwarp();
@@ -167,39 +184,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTileN, 0, 1);
       const uint64_t db0 = smem_desc_sw128(smem_u32(sm.b[0]), kKB * 128, 1024);
-      int it = 0, g = 0, j = 0;
+      int it = 0, g = 0;
       bool ok = true;
       for (int blk = blockIdx.x; ok && blk < blocks; blk += stride, ++it) {
-        if (!mbar_wait(&sm.g_ready, it & 1, abort_flag, status)) {
+        // the epilogue has read the accumulators of the previous block
+        if (it > 0 && !mbar_wait(&sm.acc_empty, (it - 1) & 1, abort_flag, status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int nt = 0; ok && nt < n_tiles; ++nt, ++j) {
-          const int ab = j & 1;
-          if (j >= 2 && !mbar_wait(&sm.acc_empty[ab], ((j - 2) >> 1) & 1, abort_flag, status)) {
+        for (int kb = 0; ok && kb < nkb; ++kb) {
+          if (!mbar_wait(&sm.g_ready[kb], it & 1, abort_flag, status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + 256u * ab;
-          for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const uint64_t da = smem_desc_sw128(smem_u32(sm.g[kb]), 16, 1024);
+          for (int h = 0; h < n_halves; ++h, ++g) {
             const int st = g % kBStages;
             if (!mbar_wait(&sm.b_full[st], (g / kBStages) & 1, abort_flag, status)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t da = smem_desc_sw128(smem_u32(sm.g[kb]), 16, 1024);
             const uint64_t db = db0 + static_cast<uint64_t>(st) * (kBStageBytes >> 4);
+            const uint32_t d = tmem + 256u * h;
 #pragma unroll
             for (int kk = 0; kk < kKB / 16; ++kk)
               mma_bf16_ss(d, da + 2 * kk, db + 128 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&sm.b_empty[st]);
           }
-          if (ok) mma_commit(&sm.acc_full[ab]);
+          if (ok) mma_commit(&sm.slot_free[kb]);  // both halves have read G slot kb
         }
-        if (ok) mma_commit(&sm.g_free);
+        if (ok) mma_commit(&sm.acc_full);
       }
       if (!ok) {
         mma_commit(&sm.drain);
@@ -214,12 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0, gu = 0;
     bool ok = true;
     for (int blk = blockIdx.x; ok && blk < blocks; blk += stride, ++it) {
-      ok = warp_all(lane == 0 ? mbar_wait(&sm.g_loaded, it & 1, abort_flag, status) : true);
-      if (!ok) break;
-      // (every lane observes the TMA writes: the waiting lane acquired them, the vote orders
-      // the warp)
       float sum = 0.f;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = 0; ok && kb < nkb; ++kb) {
+        ok = warp_wait_bar(&sm.av_full[kb], it & 1, abort_flag, status);
+        if (!ok) break;
         const uint8_t* base = sm.g[kb] + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -229,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 8; ++e) sum += f[e];
         }
       }
+      if (!ok) break;
       const float mean = sum / F;
       float sq = 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -245,11 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const float rstd = rsqrtf(sq / F + eps);
-      for (int kb = 0; kb < nkb && ok; ++kb, ++gu) {
+      for (int kb = 0; ok && kb < nkb; ++kb, ++gu) {
         const int su = gu % kUSlots;
-        ok = warp_all(lane == 0 ? mbar_wait(&sm.u_full[su], (gu / kUSlots) & 1, abort_flag,
-                                            status)
-                                : true);
+        ok = warp_wait_bar(&sm.u_full[su], (gu / kUSlots) & 1, abort_flag, status);
         if (!ok) break;
         uint8_t* base = sm.g[kb] + r * 128;
         const uint8_t* ubase = sm.u[su] + r * 128;
@@ -276,38 +290,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.w = pack_bf16x2(o[6], o[7]);
           *slot = w;
         }
+        fence_async_smem();  // slot kb of G is read by the MMAs (async proxy)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.u_empty[su]);  // this warp is done with the U slot
+        if (lane == 0) {
+          mbar_arrive(&sm.u_empty[su]);  // this warp is done with the U slot
+          mbar_arrive(&sm.g_ready[kb]);
+        }
       }
-      if (!ok) break;
-      fence_async_smem();  // G is read by the MMAs (async proxy)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.g_ready);
     }
   } else {
     // --------------------------------------------------------------------- epilogue
     const int quad = warp & 3;
-    const int half = (warp - 6) >> 2;  // columns 128 half .. +127 of the 256-wide tile
+    const int half = (warp - 6) >> 2;  // columns 128 half .. +127 of each 256-wide accumulator
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128u * half;
-    int j = 0;
-    for (int blk = blockIdx.x; blk < blocks; blk += stride) {
+    int it = 0;
+    for (int blk = blockIdx.x; blk < blocks; blk += stride, ++it) {
       const int row = blk * kRows + quad * 32 + lane;
-      bool ok = true;
-      for (int nt = 0; nt < n_tiles; ++nt, ++j) {
-        const int ab = j & 1;
-        if (!warp_all(mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, abort_flag, status))) {
-          ok = false;
-          break;
+      const bool row_ok = row < M;
+      if (!warp_all(mbar_wait(&sm.acc_full, it & 1, abort_flag, status))) break;
+      tc_fence_after();
+      for (int h = 0; h < n_halves; ++h) {
+        const int n0 = h * kTileN + 128 * half;
+        // the residual rows of this half, all loads in flight before the first use
+        uint4 xr[16];
+#pragma unroll
+        for (int v = 0; v < 16; ++v) {
+          const int c = n0 + 8 * v;
+          xr[v] = (row_ok && c + 8 <= N)
+                      ? *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(row) * ld_x + c)
+                      : make_uint4(0u, 0u, 0u, 0u);
         }
-        tc_fence_after();
-        const int n0 = nt * kTileN + 128 * half;
-#pragma unroll 1
+#pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t acc[32];
-          tmem_ld32(lane_addr + 256u * ab + ch * 32, acc);
+          tmem_ld32(lane_addr + 256u * h + ch * 32, acc);
           tmem_wait_ld();
           const int c0 = n0 + ch * 32;
-          if (row < M && c0 < N) {
+          if (row_ok && c0 < N) {
             float vals[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -315,13 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (bias != nullptr && c0 + e < N) v += __ldg(bias + c0 + e);
               vals[e] = v;
             }
-            const __nv_bfloat16* xp = x + static_cast<int64_t>(row) * ld_x + c0;
             __nv_bfloat16* yp = y + static_cast<int64_t>(row) * ld_y + c0;
             if (c0 + 32 <= N) {
 #pragma unroll
               for (int w = 0; w < 4; ++w) {
                 float fx[8];
-                bf16x8_to_f(*reinterpret_cast<const uint4*>(xp + 8 * w), fx);
+                bf16x8_to_f(xr[4 * ch + w], fx);
                 uint4 ov;
                 ov.x = pack_bf16x2(vals[8 * w + 0] + fx[0], vals[8 * w + 1] + fx[1]);
                 ov.y = pack_bf16x2(vals[8 * w + 2] + fx[2], vals[8 * w + 3] + fx[3]);
@@ -330,16 +348,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 reinterpret_cast<uint4*>(yp)[w] = ov;
               }
             } else {
+              const __nv_bfloat16* xp = x + static_cast<int64_t>(row) * ld_x + c0;
               for (int e = 0; e < 32; ++e)
                 if (c0 + e < N) yp[e] = __float2bfloat16_rn(vals[e] + __bfloat162float(xp[e]));
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
       }
-      if (!ok) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty);
     }
   }
   tc_fence_before();
@@ -352,13 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-// Shared memory of the fused kernel (F features per token).
+// Shared memory of the fused kernel.
 size_t f2_fused_smem() { return sizeof(F2Smem) + 1024; }
 
-// True when the fused kernel takes a layer: bf16, F a multiple of 64 up to 512, N a multiple of
-// 8 (the caller also checks 16-byte alignment of the operands).
+// True when the fused kernel takes a layer: F a multiple of 64 up to 512, N a multiple of 8 up
+// to 512 (two TMEM accumulators); the caller checks bf16 and 16-byte alignment.
 bool f2_fused_supported(int F, int N) {
-  return F % kKB == 0 && F >= kKB && F <= kMaxF && N % 8 == 0 && f2_fused_smem() <= 227 * 1024;
+  return F % kKB == 0 && F >= kKB && F <= kMaxF && N % 8 == 0 && N >= 8 && N <= kMaxN &&
+         f2_fused_smem() <= 227 * 1024;
 }
 
 cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_u,
