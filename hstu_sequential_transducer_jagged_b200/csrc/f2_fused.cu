@@ -231,7 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0, gu = 0;
     bool ok = true;
     for (int blk = blockIdx.x; ok && blk < blocks; blk += stride, ++it) {
-      float sum = 0.f;
+      // (eight partial sums per pass: the row's 512 additions form eight short dependency
+      // chains instead of one long one)
+      float part[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[e] = 0.f;
       for (int kb = 0; ok && kb < nkb; ++kb) {
         ok = warp_wait_bar(&sm.av_full[kb], it & 1, abort_flag, status);
         if (!ok) break;
@@ -241,12 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           float f[8];
           bf16x8_to_f(*reinterpret_cast<const uint4*>(base + ((c ^ sw) << 4)), f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) sum += f[e];
+          for (int e = 0; e < 8; ++e) part[e] += f[e];
         }
       }
       if (!ok) break;
-      const float mean = sum / F;
-      float sq = 0.f;
+      const float mean =
+          (((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]))) / F;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[e] = 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
         const uint8_t* base = sm.g[kb] + r * 128;
 #pragma unroll
@@ -256,10 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float dl = f[e] - mean;
-            sq += dl * dl;
+            part[e] = fmaf(dl, dl, part[e]);
           }
         }
       }
+      const float sq =
+          ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
       const float rstd = rsqrtf(sq / F + eps);
       for (int kb = 0; ok && kb < nkb; ++kb, ++gu) {
         const int su = gu % kUSlots;
