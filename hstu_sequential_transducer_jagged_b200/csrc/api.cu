@@ -83,10 +83,11 @@ cudaError_t launch_scatter_rows(const void* src, int64_t src_stride, const int32
                                 cudaStream_t stream);
 bool f2_fused_supported(int F, int N);
 cudaError_t launch_f2_fused(const CUtensorMap& tm_av, const CUtensorMap& tm_u,
-                            const CUtensorMap& tm_w2, int M, int N, int F, const float* gamma,
-                            const float* beta, float eps, const float* bias,
-                            const __nv_bfloat16* x, int64_t ld_x, __nv_bfloat16* y, int64_t ld_y,
-                            int* status, int num_sms, cudaStream_t stream);
+                            const CUtensorMap& tm_w2, const CUtensorMap& tm_x,
+                            const CUtensorMap& tm_y, const __nv_bfloat16* av, int64_t ld_av,
+                            int M, int N, int F, const float* gamma, const float* beta, float eps,
+                            const float* bias, float2* stats, int nparts, int* status,
+                            int num_sms, cudaStream_t stream);
 cudaError_t launch_colsum(const __nv_bfloat16* m, int64_t ld, int rows, int cols, float* out,
                           cudaStream_t stream);
 int attn_bwd_tc_ts_box();
@@ -140,9 +141,9 @@ int num_sms_current() {
 }
 
 // 2D bf16 tensor map over a row-major [rows, cols] matrix with row stride ld (elements), box
-// {box_cols, box_rows}, 128-byte swizzle, zero fill out of bounds.
-bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
-                   uint32_t box_cols, uint32_t box_rows) {
+// {box_cols, box_rows}, the given swizzle, zero fill out of bounds.
+bool make_map_bf16_sw(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                      uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -150,9 +151,29 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t col
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The same with 128-byte swizzle (the MMA operand tiles).
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                   uint32_t box_cols, uint32_t box_rows) {
+  return make_map_bf16_sw(map, base, rows, cols, ld, box_cols, box_rows,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Maps of a GEMM's bf16 output C and residual R for the staged TMA epilogue: 32 x 32 boxes,
+// 64-byte swizzle.  Absent matrices get zeroed (unused) maps.
+bool make_epilogue_maps(CUtensorMap* tc, CUtensorMap* tr, const void* C, int64_t ldc,
+                        const void* R, int64_t ldr, int M, int N) {
+  std::memset(tc, 0, sizeof(*tc));
+  std::memset(tr, 0, sizeof(*tr));
+  if (C != nullptr && !make_map_bf16_sw(tc, C, M, N, ldc, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
+  if (R != nullptr && !make_map_bf16_sw(tr, R, M, N, ldr, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
+  return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -239,6 +260,7 @@ AttnGeom make_geom(const void* ws, const WsLayout& w, const int64_t* ts, const f
   g.rab_type = nullptr;
   g.NT = 0;
   g.d_type = nullptr;
+  g.o_stats = nullptr;
   return g;
 }
 
@@ -276,6 +298,16 @@ bool attn_uses_tc(int D, int dtype, const void* q, int64_t ld_q, const void* k, 
          (ld_o % 8 == 0);
 }
 
+// The paired kernel: bf16 tensor cores, head dimension 64, no type term; it keeps the position
+// table in shared memory (it fits for P up to about 1100 next to its tiles: the shared-memory
+// check decides) and loads the timestamps with TMA (16-byte aligned base).
+bool attn_uses_pair(const AttnGeom& g, int D, bool tc) {
+  const bool use_time = g.ts != nullptr && g.rab_time != nullptr;
+  return tc && D == 64 && g.rab_type == nullptr && (g.rab_pos == nullptr || g.P <= 2048) &&
+         (!use_time || aligned16(g.ts)) &&
+         attn_fwd_pair_smem(g.P, g.rab_pos != nullptr) <= 227 * 1024;
+}
+
 // Builds the work list (pairs of query tiles for the head-width-64 tensor-core kernel, single
 // tiles otherwise) and launches the attention forward.
 hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t* offsets,
@@ -284,14 +316,8 @@ hstu_status_t attn_forward_core(const void* ws, const WsLayout& w, const int32_t
                                 const void* v, int64_t ld_v, void* o, int64_t ld_o,
                                 cudaStream_t s, int cand_only = 0) {
   const bool tc = attn_uses_tc(D, dtype, q, ld_q, k, ld_k, v, ld_v, o, ld_o);
-  // the paired kernel keeps the position table in shared memory (it fits for P up to about
-  // 1100 next to its tiles: the shared-memory check below decides) and loads the timestamps
-  // with TMA (16-byte aligned base)
   const bool use_time = g.ts != nullptr && g.rab_time != nullptr;
-  const bool pair = tc && D == 64 && g.rab_type == nullptr &&
-                    (g.rab_pos == nullptr || g.P <= 2048) &&
-                    (!use_time || aligned16(g.ts)) &&
-                    attn_fwd_pair_smem(g.P, g.rab_pos != nullptr) <= 227 * 1024;
+  const bool pair = attn_uses_pair(g, D, tc);
   const int group = pair ? 2 : 1;
   if (build_list(ws, w, offsets, B, T, max_len, g.mask, g.num_candidates, group, s, cand_only) !=
       cudaSuccess)
@@ -334,12 +360,15 @@ hstu_status_t gemm(int dtype, int epi, const void* A, int64_t lda, const void* B
                   aligned16(A) && aligned16(Bm) && aligned16(C) && (R == nullptr || aligned16(R));
   cudaError_t e;
   if (tc) {
-    CUtensorMap ta, tb;
-    if (!make_map_bf16(&ta, A, M, K, lda, 64, 128) || !make_map_bf16(&tb, Bm, K, N, ldb, 64, 64))
+    CUtensorMap ta, tb, tcm, trm;
+    if (!make_map_bf16(&ta, A, M, K, lda, 64, 128) || !make_map_bf16(&tb, Bm, K, N, ldb, 64, 64) ||
+        !make_epilogue_maps(&tcm, &trm, C, ldc, R, ldr, M, N))
       return HSTU_ERR_CUDA;
     GemmArgs ga{};
     ga.ta = &ta;
     ga.tb = &tb;
+    ga.tc = &tcm;
+    ga.tr = &trm;
     ga.M = M;
     ga.N = N;
     ga.K = K;
@@ -360,25 +389,33 @@ hstu_status_t gemm(int dtype, int epi, const void* A, int64_t lda, const void* B
   return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
 }
 
-// Y = X + (Norm(AV) ⊙ U) W2 + b2 over `rows` tokens: one fused tensor-core kernel for bf16 with
-// H d_v <= 512 (G formed in shared memory), else LayerNorm ⊙ U into g_buf and the GEMM.
+// Y = X + (Norm(AV) ⊙ U) W2 + b2 over `rows` tokens: for bf16 with H d_v <= 1024 a row-statistics
+// pass and one fused tensor-core kernel (G formed in shared memory), else LayerNorm ⊙ U into
+// g_buf and the GEMM.
+bool norm_gate_f2_fused(int dtype, const void* av, int64_t ld_av, const void* u, int64_t ld_u,
+                        const void* w2, const void* x, const void* y, int F, int d_model) {
+  return dtype == HSTU_BF16 && f2_fused_supported(F, d_model) && ld_av % 8 == 0 &&
+         ld_u % 8 == 0 && d_model % 8 == 0 && aligned16(av) && aligned16(u) && aligned16(w2) &&
+         aligned16(x) && aligned16(y);
+}
+
+// nparts > 0: g_buf already holds the attention kernel's per-slice statistics of av (F / 32
+// slices a row); else the fused path computes them into g_buf first.
 hstu_status_t norm_gate_f2(int dtype, const void* av, int64_t ld_av, const void* u, int64_t ld_u,
                            const float* gamma, const float* beta, float eps, const void* w2,
                            const float* b2, const void* x, void* y, int rows, int F, int d_model,
-                           void* g_buf, int32_t* status, cudaStream_t s) {
-  const bool fused = dtype == HSTU_BF16 && f2_fused_supported(F, d_model) && ld_av % 8 == 0 &&
-                     ld_u % 8 == 0 && d_model % 8 == 0 && aligned16(av) && aligned16(u) &&
-                     aligned16(w2) && aligned16(x) && aligned16(y);
-  if (fused) {
-    CUtensorMap tav, tu, tw2;
+                           void* g_buf, int32_t* status, cudaStream_t s, int nparts = 0) {
+  if (norm_gate_f2_fused(dtype, av, ld_av, u, ld_u, w2, x, y, F, d_model)) {
+    CUtensorMap tav, tu, tw2, ty, tx;
     if (!make_map_bf16(&tav, av, rows, F, ld_av, 64, 128) ||
         !make_map_bf16(&tu, u, rows, F, ld_u, 64, 128) ||
-        !make_map_bf16(&tw2, w2, F, d_model, d_model, 64, 64))
+        !make_map_bf16(&tw2, w2, F, d_model, d_model, 64, 64) ||
+        !make_epilogue_maps(&ty, &tx, y, d_model, x, d_model, rows, d_model))
       return HSTU_ERR_CUDA;
+    // g_buf (rows x F elements) holds the per-row (mean, rstd) pairs instead of G
     const cudaError_t e = launch_f2_fused(
-        tav, tu, tw2, rows, d_model, F, gamma, beta, eps, b2,
-        static_cast<const __nv_bfloat16*>(x), d_model, static_cast<__nv_bfloat16*>(y), d_model,
-        status, num_sms_current(), s);
+        tav, tu, tw2, tx, ty, static_cast<const __nv_bfloat16*>(av), ld_av, rows, d_model, F,
+        gamma, beta, eps, b2, static_cast<float2*>(g_buf), nparts, status, num_sms_current(), s);
     return e == cudaSuccess ? HSTU_OK : cuda_fail(e);
   }
   if (launch_ln_gate(dtype == HSTU_BF16 ? 0 : 1, av, ld_av, u, ld_u, gamma, beta, eps, g_buf, F,
@@ -400,10 +437,16 @@ hstu_status_t gemm_tc_layout(int epi, int a_mn, int b_mn, const void* A, int64_t
                          : make_map_bf16(&ta, A, M, K, lda, 64, 128);
   const bool ok_b = b_mn ? make_map_bf16(&tb, Bm, K, N, ldb, 64, 64)
                          : make_map_bf16(&tb, Bm, N, K, ldb, 64, 256);
-  if (!ok_a || !ok_b) return HSTU_ERR_CUDA;
+  CUtensorMap tcm, trm;
+  if (!ok_a || !ok_b ||
+      !make_epilogue_maps(&tcm, &trm, epi == 4 ? nullptr : C, ldc, epi == 1 ? R : nullptr, ldr, M,
+                          N))
+    return HSTU_ERR_CUDA;
   GemmArgs ga{};
   ga.ta = &ta;
   ga.tb = &tb;
+  ga.tc = &tcm;
+  ga.tr = &trm;
   ga.M = M;
   ga.N = N;
   ga.K = K;
@@ -721,16 +764,24 @@ hstu_status_t layer_stage(const hstu_layer_desc_t* d, int32_t stage, const void*
     return gemm(d->dtype, 0, x, d->d_model, w1, n1, T, n1, d->d_model, b1, nullptr, 0, uvqk, n1,
                 status, s);
   }
+  AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
+                         d->num_time_buckets, H, T, d->mask, d->num_candidates, d->alpha);
+  set_types(&g, d->token_types, d->rab_type, d->num_types);
+  // With the paired attention kernel and the fused output projection, the attention leaves
+  // the LayerNorm statistics of each 32-column slice of av in gbuf (decided from the
+  // descriptor and the workspace alone, so both stages agree).
+  const bool stats_in_attn =
+      d->dtype == HSTU_BF16 && hv % 32 == 0 && f2_fused_supported(hv, d->d_model) &&
+      aligned16(av) && aligned16(u_ptr) && n1 % 8 == 0 &&
+      attn_uses_pair(g, D, attn_uses_tc(D, d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av, hv));
   if (stage == HSTU_STAGE_ATTENTION) {
-    AttnGeom g = make_geom(ws, w, d->timestamps, d->rab_pos, d->max_pos_dist, d->rab_time,
-                           d->num_time_buckets, H, T, d->mask, d->num_candidates, d->alpha);
-    set_types(&g, d->token_types, d->rab_type, d->num_types);
+    if (stats_in_attn) g.o_stats = reinterpret_cast<float2*>(gbuf);
     return attn_forward_core(ws, w, d->seq_offsets, d->max_seq_len, g, d->num_seqs, T, D,
                              d->dtype, q_ptr, n1, k_ptr, n1, v_ptr, n1, av, hv, s);
   }
   // Norm(AV) ⊙ U, then f2 + residual: Y = X + G W2 + b2
   return norm_gate_f2(d->dtype, av, hv, u_ptr, n1, d->ln_gamma, d->ln_beta, d->ln_eps, w2, b2, x,
-                      y, T, hv, d->d_model, gbuf, status, s);
+                      y, T, hv, d->d_model, gbuf, status, s, stats_in_attn ? hv / 32 : 0);
 }
 }  // namespace
 

@@ -181,8 +181,6 @@ __device__ __forceinline__ float time_term32(const float* time_h, int d) {
   return time_h[log2_small(d)];
 }
 
-__device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_fast(h), h); }
-
 // Per-row constants of one 48-column segment's epilogue.  The mode and the time-term kind are
 // warp-uniform: a warp takes the per-element path for all of its rows when any row needs it
 // (the per-element formulas are exact for every row), so no branch in the epilogue diverges.
@@ -1027,14 +1025,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(it.row0 + i) * ld_o +
                                                 head * kD + 32 * h);
+          uint4 vv[4];
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
-            uint4 vv;
-            vv.x = pack_bf16x2(__uint_as_float(o[8 * w4 + 0]), __uint_as_float(o[8 * w4 + 1]));
-            vv.y = pack_bf16x2(__uint_as_float(o[8 * w4 + 2]), __uint_as_float(o[8 * w4 + 3]));
-            vv.z = pack_bf16x2(__uint_as_float(o[8 * w4 + 4]), __uint_as_float(o[8 * w4 + 5]));
-            vv.w = pack_bf16x2(__uint_as_float(o[8 * w4 + 6]), __uint_as_float(o[8 * w4 + 7]));
-            dst[w4] = vv;
+            vv[w4].x = pack_bf16x2(__uint_as_float(o[8 * w4 + 0]), __uint_as_float(o[8 * w4 + 1]));
+            vv[w4].y = pack_bf16x2(__uint_as_float(o[8 * w4 + 2]), __uint_as_float(o[8 * w4 + 3]));
+            vv[w4].z = pack_bf16x2(__uint_as_float(o[8 * w4 + 4]), __uint_as_float(o[8 * w4 + 5]));
+            vv[w4].w = pack_bf16x2(__uint_as_float(o[8 * w4 + 6]), __uint_as_float(o[8 * w4 + 7]));
+            dst[w4] = vv[w4];
+          }
+          if (g.o_stats != nullptr) {
+            // mean and sum of squared deviations of the 32 stored (bf16) values: two passes
+            float f[32];
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) {
+              const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&vv[w4]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 fv = __bfloat1622float2(p2[e]);
+                f[8 * w4 + 2 * e] = fv.x;
+                f[8 * w4 + 2 * e + 1] = fv.y;
+              }
+            }
+            float sm8[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sm8[e & 3] += f[e];
+            const float mean = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) * (1.f / 32.f);
+            float q8[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float dl = f[e] - mean;
+              q8[e & 3] = fmaf(dl, dl, q8[e & 3]);
+            }
+            g.o_stats[static_cast<int64_t>(it.row0 + i) * (g.H * (kD / 32)) + head * (kD / 32) + h] =
+                make_float2(mean, (q8[0] + q8[1]) + (q8[2] + q8[3]));
           }
         }
         tc_fence_before();

@@ -40,6 +40,10 @@ struct AttnGeom {
   const float* rab_type;
   int32_t NT;
   float* d_type;            // backward: gradient of rab_type [NT*NT] (accumulated), or nullptr
+  // forward (paired kernel): per output row, the mean and the sum of squared deviations of
+  // each 32-column slice of the bf16 output, [T][H d_v / 32] float2, or nullptr (the
+  // LayerNorm statistics of the layer's output projection, combined there)
+  float2* o_stats;
 };
 
 // One launch of the persistent tensor-core GEMM (gemm_tc.cu): C[M, N] = epi(A · B), A and B
@@ -47,6 +51,8 @@ struct AttnGeom {
 struct GemmArgs {
   const CUtensorMap* ta;
   const CUtensorMap* tb;
+  const CUtensorMap* tc;           // epi 0-3: C, box {32, 32}, 64-byte swizzle (TMA store)
+  const CUtensorMap* tr;           // epi 1: the residual, same box and swizzle
   int M, N, K, k_splits;
   int epi, a_mn, b_mn;
   const float* bias;               // [N] or nullptr

@@ -13,6 +13,10 @@
 // of one tile overlaps the main loop of the next.  Warp 0 TMA producer, warp 1 TMEM allocation
 // + single-thread tcgen05.mma issue, warps 2..9 epilogue: warp w reads TMEM lanes 32 (w % 4)
 // .. +31 (one output row per thread) and columns 128 ((w - 2) / 4) .. +127 of the tile.
+// The bf16 epilogues write each 32 x 32 chunk into a swizzled shared-memory staging tile
+// (two per warp) and store it with one TMA store, and the residual arrives the same way, one
+// chunk ahead: a row per thread but whole 64-byte rows per copy, instead of warp-wide
+// accesses that touch 32 cache lines each.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -27,10 +31,14 @@ constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 320;  // 10 warps
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB: [128 rows][64 k], SW128, K-major
 constexpr int kBBytes = kBK * kBN * 2;   // 32 KB: four [64 k][64 n] SW128 boxes, MN-major
+constexpr int kEpiWarps = 8;
+constexpr int kStageTile = 32 * 32 * 2;  // 2 KB: 32 rows x 32 bf16, 64-byte swizzle
 
 struct GemmSmem {
   alignas(1024) uint8_t a[kGemmStages][kABytes];
   alignas(1024) uint8_t b[kGemmStages][kBBytes];
+  alignas(1024) uint8_t stage[kEpiWarps][2][kStageTile];
+  uint64_t rbar[kEpiWarps][2];  // residual chunk landed in stage[w][b]
   uint64_t full[kGemmStages];
   uint64_t empty[kGemmStages];
   uint64_t acc_full[2];
@@ -67,7 +75,9 @@ __device__ __forceinline__ float silu_fast(float x) {
 template <int EPI, int A_MN, int B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tm_a,
-                        const __grid_constant__ CUtensorMap tm_b, int M, int N, int K,
+                        const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_c,
+                        const __grid_constant__ CUtensorMap tm_r, int M, int N, int K,
                         int k_splits, const float* __restrict__ bias,
                         const __nv_bfloat16* __restrict__ resid, int64_t ld_r,
                         __nv_bfloat16* __restrict__ C, int64_t ldc,
@@ -93,7 +103,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
-      mbar_init(&sm.acc_empty[b], 8);  // one elected lane per epilogue warp
+      mbar_init(&sm.acc_empty[b], kEpiWarps);  // one elected lane per epilogue warp
+    }
+    for (int w = 0; w < kEpiWarps; ++w) {
+      mbar_init(&sm.rbar[w][0], 1);
+      mbar_init(&sm.rbar[w][1], 1);
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -203,15 +217,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;  // columns 128 * half .. +127 of the tile
+    const int ew = warp - 2;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 128u * half;
+    const bool bias_vec = bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 15) == 0;
+    uint8_t* stg0 = sm.stage[ew][0];
+    uint8_t* stg1 = sm.stage[ew][1];
+    // residual loads: one wait follows each load of a buffer; bit b of rph is the parity of
+    // buffer b's next completion, bit b of pend marks a load not yet waited for
+    uint32_t rph = 0, pend = 0;
     int j = 0;
-    for (int t = blockIdx.x; t < tiles; t += stride, ++j) {
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < tiles; t += stride, ++j) {
       const int ab = j & 1;
       const int mn = t % mn_tiles, ks = t / mn_tiles;
       const int m0 = (mn / n_tiles) * kBM;
       const int n0 = (mn % n_tiles) * kBN + 128 * half;
-      const int row = m0 + quad * 32 + lane;
-      if (!warp_all(mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, abort_flag, status))) break;
+      const int r0 = m0 + quad * 32;  // first row of this warp's 32
+      const int row = r0 + lane;
+      if constexpr (EPI == 1) {
+        // the first residual chunk: buffer 0's last store (chunk 2 of the previous tile) has
+        // read it
+        if (n0 < N) {
+          if (lane == 0) {
+            bulk_wait_read<1>();
+            mbar_arrive_expect_tx(&sm.rbar[ew][0], kStageTile);
+            tma_load_2d(stg0, &tm_r, &sm.rbar[ew][0], n0, r0);
+          }
+          pend |= 1u;
+        }
+      }
+      if (!warp_all(mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, abort_flag, status))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       // a K range past the end (k_splits not dividing the K blocks) contributed nothing
       const bool empty_range = ks * kb_per >= kblocks;
@@ -221,8 +259,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(lane_addr + 256u * ab + ch * 32, acc);
         tmem_wait_ld();
         const int c0 = n0 + ch * 32;
-        if (row < M && c0 < N && !empty_range) {
-          if constexpr (EPI == 4) {
+        if constexpr (EPI == 4) {
+          if (row < M && c0 < N && !empty_range) {
             float* cp = Cf + static_cast<int64_t>(row) * ldc + c0;
             if (c0 + 32 <= N) {
 #pragma unroll
@@ -234,16 +272,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int e = 0; e < 32; ++e)
                 if (c0 + e < N) atomicAdd(cp + e, __uint_as_float(acc[e]));
             }
-          } else {
+          }
+        } else {
+          if (c0 >= N) continue;  // warp-uniform: nothing of this chunk is stored
+          uint8_t* stg = (ch & 1) ? stg1 : stg0;
           float vals[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = c0 + e;
-            float x = __uint_as_float(acc[e]);
-            if (bias != nullptr && c < N) x += __ldg(bias + c);
-            vals[e] = x;
+          for (int e = 0; e < 32; ++e) vals[e] = __uint_as_float(acc[e]);
+          if (bias != nullptr) {
+            if (bias_vec && c0 + 32 <= N) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + c0 + e));
+                vals[e] += bv.x;
+                vals[e + 1] += bv.y;
+                vals[e + 2] += bv.z;
+                vals[e + 3] += bv.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < N) vals[e] += __ldg(bias + c0 + e);
+            }
           }
-          if (EPI == 3) {  // the fp32 pre-activation, before the SiLU overwrites vals
+          if (EPI == 3 && row < M) {  // the fp32 pre-activation, before the SiLU overwrites vals
             float* pp = C2 + static_cast<int64_t>(row) * ld_c2 + c0;
             if (c0 + 32 <= N) {
 #pragma unroll
@@ -255,53 +307,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (c0 + e < N) pp[e] = vals[e];
             }
           }
-          if (EPI == 1) {
-            const __nv_bfloat16* rp = resid + static_cast<int64_t>(row) * ld_r + c0;
-            if (c0 + 32 <= N) {
+          if constexpr (EPI == 1) {
+            // this chunk's residual rows (TMA, zero past the bounds), then the next chunk's
+            const int rb = ch & 1;
+            ok = warp_all(lane == 0 ? mbar_wait(&sm.rbar[ew][rb], (rph >> rb) & 1u, abort_flag,
+                                                status)
+                                    : true);
+            if (!ok) break;
+            rph ^= 1u << rb;
+            pend &= ~(1u << rb);
 #pragma unroll
-              for (int w = 0; w < 4; ++w) {
-                uint4 rv = *reinterpret_cast<const uint4*>(rp + 8 * w);
-                const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rv);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 rv = *reinterpret_cast<const uint4*>(stg + stage64_offset(lane, q));
+              const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rv);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  float2 f = __bfloat1622float2(r2[e]);
-                  vals[8 * w + 2 * e] += f.x;
-                  vals[8 * w + 2 * e + 1] += f.y;
-                }
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(r2[e]);
+                vals[8 * q + 2 * e] += f.x;
+                vals[8 * q + 2 * e + 1] += f.y;
               }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (c0 + e < N) vals[e] += __bfloat162float(rp[e]);
-            }
-          } else if (EPI == 0 || EPI == 3) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) vals[e] = silu_fast(vals[e]);
-          }
-          __nv_bfloat16* cp = C + static_cast<int64_t>(row) * ldc + c0;
-          if (c0 + 32 <= N) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              uint4 ov;
-              ov.x = pack_bf16x2(vals[8 * w + 0], vals[8 * w + 1]);
-              ov.y = pack_bf16x2(vals[8 * w + 2], vals[8 * w + 3]);
-              ov.z = pack_bf16x2(vals[8 * w + 4], vals[8 * w + 5]);
-              ov.w = pack_bf16x2(vals[8 * w + 6], vals[8 * w + 7]);
-              reinterpret_cast<uint4*>(cp)[w] = ov;
             }
           } else {
+            // the store two chunks back has read this buffer
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            if (EPI == 0 || EPI == 3) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c0 + e < N) cp[e] = __float2bfloat16_rn(vals[e]);
+              for (int e = 0; e < 32; ++e) vals[e] = silu_fast(vals[e]);
+            }
           }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 ov;
+            ov.x = pack_bf16x2(vals[8 * q + 0], vals[8 * q + 1]);
+            ov.y = pack_bf16x2(vals[8 * q + 2], vals[8 * q + 3]);
+            ov.z = pack_bf16x2(vals[8 * q + 4], vals[8 * q + 5]);
+            ov.w = pack_bf16x2(vals[8 * q + 6], vals[8 * q + 7]);
+            *reinterpret_cast<uint4*>(stg + stage64_offset(lane, q)) = ov;
           }
+          fence_proxy_async_smem();  // the staging tile is read by the TMA store
+          __syncwarp();
+          if (lane == 0) {
+            if (r0 < M) {  // rows past M and columns past N are clipped
+              tma_store_2d(&tm_c, stg, c0, r0);
+              bulk_commit();
+            }
+            if constexpr (EPI == 1) {
+              if (ch + 1 < 128 / 32 && c0 + 32 < N) {
+                // the previous chunk's store has read the other buffer: the next residual
+                bulk_wait_read<1>();
+                uint8_t* nxt = (ch & 1) ? stg0 : stg1;
+                mbar_arrive_expect_tx(&sm.rbar[ew][(ch + 1) & 1], kStageTile);
+                tma_load_2d(nxt, &tm_r, &sm.rbar[ew][(ch + 1) & 1], c0 + 32, r0);
+              }
+            }
+          }
+          if (EPI == 1 && ch + 1 < 128 / 32 && c0 + 32 < N) pend |= 1u << ((ch + 1) & 1);
         }
       }
+      if (!ok) break;
       // this warp's part of the accumulator buffer is read: the MMA warp may reuse it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
     }
+    if (lane == 0) {
+      // after a timeout: no residual load still writing into the staging tiles
+      for (int b2 = 0; b2 < 2; ++b2)
+        if (pend & (1u << b2)) mbar_wait(&sm.rbar[ew][b2], (rph >> b2) & 1u, nullptr, nullptr);
+      bulk_wait_all();  // the staging tiles stay valid until the stores are done
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -318,7 +394,8 @@ cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaStream_t
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kGemmThreads, smem, stream>>>(*a.ta, *a.tb, a.M, a.N, a.K, a.k_splits, a.bias,
+  kern<<<grid, kGemmThreads, smem, stream>>>(*a.ta, *a.tb, *a.tc, *a.tr, a.M, a.N, a.K,
+                                             a.k_splits, a.bias,
                                              a.resid, a.ld_r, a.C, a.ldc, a.C2, a.ld_c2, a.Cf,
                                              a.status);
   return cudaGetLastError();

@@ -287,6 +287,61 @@ def attention_backward(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time,
     return out if d_type is None else out + (d_type,)
 
 
+def bias_grad_entries(q, k, v, d_o, seq_offsets, timestamps, rab_pos, rab_time, *, num_heads,
+                      d_qk, d_v, max_pos_dist, num_time_buckets, alpha=1.0, max_delta=31,
+                      max_bucket=5):
+    """Selected entries of the causal attention's bias-table gradients, exactly as
+    attention_backward defines them, by enumerating only the pairs that reach those entries.
+
+    Returns (d_rab_pos[P .. P + max_delta], d_rab_time[0 .. max_bucket]) (fp64).
+      * position entry P + Δ (Δ < P, so not clamped) collects the pairs (i, i - Δ);
+      * time bucket b <= max_bucket collects the pairs with ts_i - ts_j < 2^(max_bucket + 1)
+        (bucket(dt) <= max_bucket exactly there), found per row by a search over the
+        sequence's non-decreasing timestamps.
+    Each pair contributes dS = (dO_i · V_j) φ2'(α q_i·k_j + rab) summed over heads, as in
+    attention_backward (causal mask, no type term).
+    """
+    H, P = num_heads, max_pos_dist
+    assert 0 <= max_delta < P and 0 <= max_bucket < num_time_buckets - 1
+    Q, K, V = _heads(q, H, d_qk), _heads(k, H, d_qk), _heads(v, H, d_v)
+    dO = _heads(d_o, H, d_v)
+    d_pos = np.zeros(max_delta + 1, dtype=np.float64)
+    d_time = np.zeros(max_bucket + 1, dtype=np.float64)
+    rp = np.asarray(rab_pos, dtype=np.float64)
+    rt = np.asarray(rab_time, dtype=np.float64)
+
+    def d_s(s, I, J):
+        """dS of the pairs (s + I, s + J) summed over heads."""
+        dt = np.asarray(timestamps[s + I], dtype=np.int64) - np.asarray(timestamps[s + J],
+                                                                         dtype=np.int64)
+        bias = rp[position_index(I - J, P)] + rt[time_bucket(dt, num_time_buckets)]
+        sc = alpha * np.einsum("phd,phd->ph", Q[s + I], K[s + J]) + bias[:, None]
+        da = np.einsum("phd,phd->ph", dO[s + I], V[s + J])
+        return (da * silu_grad(sc)).sum(axis=1), dt
+
+    for b in range(len(seq_offsets) - 1):
+        s, e = int(seq_offsets[b]), int(seq_offsets[b + 1])
+        L = e - s
+        if L == 0:
+            continue
+        ts = np.asarray(timestamps[s:e], dtype=np.int64)
+        assert np.all(np.diff(ts) >= 0), "timestamps must not decrease within a sequence"
+        for delta in range(min(max_delta, L - 1) + 1):
+            I = np.arange(delta, L)
+            ds, _ = d_s(s, I, I - delta)
+            d_pos[delta] += ds.sum()
+        # rows i and the first key j with ts_i - ts_j < 2^(max_bucket + 1)
+        lim = np.int64(1) << np.int64(max_bucket + 1)
+        first = np.searchsorted(ts, ts - lim, side="right")
+        counts = np.arange(L) - first + 1
+        I = np.repeat(np.arange(L), counts)
+        J = np.concatenate([np.arange(f, i + 1) for i, f in enumerate(first)]) if L else I
+        ds, dt = d_s(s, I, J)
+        bk = time_bucket(dt, num_time_buckets)
+        d_time += np.bincount(bk, weights=ds, minlength=max_bucket + 1)[:max_bucket + 1]
+    return d_pos, d_time
+
+
 # --------------------------------------------------------------------------------------------
 # the layer: U,V,Q,K = Split(φ1(f1(X)));  Y = X + f2(Norm(A(X)V(X)) ⊙ U(X))
 # ([Review §2.1] first and third formula + the block diagram's residual edge;

@@ -236,10 +236,9 @@ def test_attention_forward_fp32(B):
 
 
 def test_attention_forward_full_size_sampled_rows(B):
-    """The 4-layer stack's attention shape (B=8, L~U{2048..8192}, H=8, d=64) at full size."""
+    """The 4-layer stack's attention shape (B=8, L~U{2048..8192}, H=8, d=64) at full size, with
+    the attention workload's own score distribution (unit-variance Q, K, V)."""
     case = W.make_attn_fwdbwd_bf16_b64(seed=3, B=8, lo=2048, hi=8192)
-    case.q = W.round_to_bf16(case.q * 0.25)
-    case.k = W.round_to_bf16(case.k * 0.25)
     out = gpu_attention(B, case).float().cpu().numpy()
     off = case.seq_offsets
     rng = np.random.default_rng(5)
@@ -280,6 +279,18 @@ def test_layer_forward_small(B, bf16):
     y = gpu_layer(B, case)
     torch.cuda.synchronize()
     assert_close(y, oracle_layer(case), f"layer bf16={bf16}")
+
+
+@pytest.mark.parametrize("d_model,H,d", [(264, 3, 32), (200, 2, 64), (128, 8, 128)])
+def test_layer_forward_f2_shapes(B, d_model, H, d):
+    # the fused output projection at its edges: a partial second 256-column unit (264), a
+    # single partial unit (200), F = H d_v not a multiple of 64 (96) and the largest F (1024);
+    # 507 tokens leave a partial 128-row block
+    case = W.random_layer_case(22, [300, 1, 129, 0, 77], d_model=d_model, H=H, d=d, P=30,
+                               NB=16, w_std=0.05)
+    y = gpu_layer(B, case)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_layer(case), f"layer f2 d_model={d_model} H={H} d={d}")
 
 
 def test_layer_forward_mfalcon_small(B):
@@ -334,10 +345,11 @@ def test_mfalcon_workload_sampled_sequence(B):
         x = gpu_layer(B, case, l, x=x)
     torch.cuda.synchronize()
     y = x.float().cpu().numpy()
-    s, e, off = _sequence_subcase(case, 5)
-    ref = O.stack_forward(case.x[s:e], case.layers, off, case.timestamps[s:e],
-                          round_between=W.round_to_bf16, **attn_kw(case))
-    assert_close(y[s:e], ref, "mfalcon sequence 5")
+    for b in (0, 5, case.num_seqs - 1):
+        s, e, off = _sequence_subcase(case, b)
+        ref = O.stack_forward(case.x[s:e], case.layers, off, case.timestamps[s:e],
+                              round_between=W.round_to_bf16, **attn_kw(case))
+        assert_close(y[s:e], ref, f"mfalcon sequence {b}")
 
 
 # ----------------------------------------------------------------------- attention backward
@@ -391,6 +403,21 @@ def test_attention_backward_full_size_sampled(B):
             assert_close(g, r, f"full backward seq {b} {name}")
     tp, tt = float(dp.double().sum()), float(dtm.double().sum())
     assert abs(tp - tt) <= 1e-3 * max(abs(tp), abs(tt), 1.0)
+    # table entries compared element by element, each summed over every sequence: offsets
+    # 0..31 of the position table and the time buckets of differences below 512 s
+    P = case.max_pos_dist
+    ref_p, ref_t = O.bias_grad_entries(case.q, case.k, case.v, case.d_o, case.seq_offsets,
+                                       case.timestamps, case.rab_pos, case.rab_time,
+                                       max_delta=31, max_bucket=8, **_attn_kw_causal(case))
+    assert_close(dp[P:P + 32], ref_p, "full backward d_rab_pos entries P..P+31")
+    assert_close(dtm[:9], ref_t, "full backward d_rab_time buckets 0..8")
+
+
+def _attn_kw_causal(case):
+    assert case.mask == W.MASK_CAUSAL
+    kw = attn_kw(case)
+    del kw["mask"], kw["num_candidates"]
+    return kw
 
 
 # ---------------------------------------------------------------------------- misc kernels

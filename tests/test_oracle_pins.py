@@ -659,3 +659,24 @@ def test_type_bias_gradient_finite_differences():
         assert abs(fd - d_type[c]) <= 1e-6 * max(1.0, abs(fd))
     assert abs(d_type.sum() - res[3].sum()) <= 1e-9 * max(1.0, abs(res[3].sum()))
     assert abs(d_type.sum() - res[4].sum()) <= 1e-9 * max(1.0, abs(res[4].sum()))
+
+
+def test_bias_grad_entries_match_full_backward():
+    # the pair-enumerating restatement of the bias-table gradient entries agrees with the full
+    # backward (itself pinned by finite differences) on a small causal case whose timestamps
+    # repeat and step by a few seconds, so that every selected bucket and offset is populated
+    rng = np.random.default_rng(17)
+    lengths = [37, 1, 90, 64]
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T, H, d, P, NB = int(off[-1]), 2, 8, 12, 10
+    q, k, v, d_o = (rng.normal(0, 0.7, (T, H * d)) for _ in range(4))
+    ts = np.concatenate([np.cumsum(rng.integers(0, 9, size=n)) for n in lengths]).astype(np.int64)
+    rab_pos = rng.normal(0, 0.5, 2 * P + 1)
+    rab_time = rng.normal(0, 0.5, NB)
+    kw = dict(num_heads=H, d_qk=d, d_v=d, max_pos_dist=P, num_time_buckets=NB, alpha=0.6)
+    full = O.attention_backward(q, k, v, d_o, off, ts, rab_pos, rab_time, **kw)
+    dp, dt = O.bias_grad_entries(q, k, v, d_o, off, ts, rab_pos, rab_time, max_delta=7,
+                                 max_bucket=4, **kw)
+    assert np.abs(dt).min() > 0  # every selected bucket has pairs
+    np.testing.assert_allclose(dp, full[3][P:P + 8], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dt, full[4][:5], rtol=1e-10, atol=1e-12)
