@@ -858,9 +858,10 @@ def main():
         "e2e": e2e,
         "configs": configs,
         "clocks": clocks,
-        # per layer: f1 GEMM, work list, attention, and the fused Norm(AV) * U + f2 kernel (bf16
-        # with H d_v <= 512) or LayerNorm * U and the f2 GEMM
-        "gpu_launches": (4 if wl.num_heads * wl.d_v <= 512 else 5) * L * K,
+        # per layer: f1 GEMM, work list, attention (which also leaves the LayerNorm statistics),
+        # and the fused Norm(AV) * U + f2 kernel (bf16 with H d_v and d_model <= 512), or
+        # LayerNorm * U and the f2 GEMM
+        "gpu_launches": (4 if wl.num_heads * wl.d_v <= 512 and wl.d_model <= 512 else 5) * L * K,
         "wall_s_timed_region": wall,
     }
     print(json.dumps(line), flush=True)
