@@ -284,7 +284,8 @@ def attention_backward(q, k, v, d_o, seq_offsets, max_seq_len, timestamps=None, 
     dv = torch.empty_like(v)
     d_pos = None if rab_pos is None else torch.empty_like(rab_pos)
     d_time = None if rab_time is None else torch.empty_like(rab_time)
-    if dq.stride(0) != q.stride(0) or dk.stride(0) != k.stride(0) or dv.stride(0) != v.stride(0):
+    if T > 0 and (dq.stride(0) != q.stride(0) or dk.stride(0) != k.stride(0)
+                  or dv.stride(0) != v.stride(0)):
         raise ValueError("q, k, v must be contiguous for the backward binding")
     desc = attn_desc(seq_offsets=seq_offsets, total_tokens=T, max_seq_len=max_seq_len,
                      timestamps=timestamps, num_heads=num_heads, d_qk=d, d_v=v.shape[1] // num_heads,

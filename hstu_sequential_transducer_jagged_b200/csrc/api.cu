@@ -569,7 +569,9 @@ hstu_status_t hstu_attention_forward(const hstu_attn_desc_t* d, const void* q, c
   if (st != HSTU_OK) return st;
   const int D = d->d_qk;
   const int64_t cols = static_cast<int64_t>(d->num_heads) * D;
-  if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
+  // (row strides mean nothing for an empty batch: views of zero rows may report any stride)
+  if (d->total_tokens > 0 &&
+      (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols))
     return HSTU_ERR_INVALID_ARG;
   const WsLayout w = attn_layout(d->total_tokens, d->num_seqs, d->max_seq_len);
   st = check_ws(ws, ws_bytes, w.total_attn);
@@ -630,7 +632,9 @@ hstu_status_t attn_backward_impl(const hstu_attn_desc_t* d, const void* q, const
   if (st != HSTU_OK) return st;
   const int D = d->d_qk;
   const int64_t cols = static_cast<int64_t>(d->num_heads) * D;
-  if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
+  // (row strides mean nothing for an empty batch: views of zero rows may report any stride)
+  if (d->total_tokens > 0 &&
+      (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols))
     return HSTU_ERR_INVALID_ARG;
   if (d->rab_pos != nullptr && d_rab_pos == nullptr) return HSTU_ERR_INVALID_ARG;
   if (d->rab_time != nullptr && d->timestamps != nullptr && d_rab_time == nullptr)
@@ -1243,7 +1247,9 @@ extern "C" hstu_status_t hstu_attention_forward_static_ws(const hstu_attn_desc_t
   // the checks hstu_attention_forward makes before it touches the workspace, made here before
   // the status word of the shared array is cleared
   const int64_t cols = static_cast<int64_t>(d->num_heads) * d->d_qk;
-  if (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols)
+  // (row strides mean nothing for an empty batch: views of zero rows may report any stride)
+  if (d->total_tokens > 0 &&
+      (d->ld_q < cols || d->ld_k < cols || d->ld_v < cols || d->ld_o < cols))
     return HSTU_ERR_INVALID_ARG;
   if (d->num_seqs > 0 && d->total_tokens > 0 &&
       (q == nullptr || k == nullptr || v == nullptr || o == nullptr))

@@ -78,7 +78,7 @@ typedef struct {
   int32_t num_heads;          /* H >= 1 */
   int32_t d_qk;               /* per-head query/key width */
   int32_t d_v;                /* per-head value width */
-  int64_t ld_q, ld_k, ld_v, ld_o;  /* row strides in elements */
+  int64_t ld_q, ld_k, ld_v, ld_o;  /* row strides in elements (not checked when total_tokens is 0) */
   int32_t mask;               /* hstu_mask_t */
   int32_t num_candidates;     /* M-FALCON: the last m tokens of every sequence are candidates */
   int32_t mfalcon_microbatch; /* b_m >= 1 (M-FALCON only); the output does not depend on it */

@@ -87,6 +87,19 @@ def test_attention_workspace_checks(lib):
     assert lib.hstu_attention_forward(None, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 1
 
 
+def test_empty_batch_accepts_any_row_strides(lib):
+    # zero tokens: nothing to compute, and zero-row views report arbitrary strides (0 for an
+    # empty torch tensor); the call succeeds without touching any buffer
+    d = _desc(total_tokens=0, max_seq_len=0, ld_q=0, ld_k=0, ld_v=0, ld_o=0)
+    need = lib.hstu_attention_workspace_size(ctypes.byref(d))
+    assert lib.hstu_attention_forward(ctypes.byref(d), None, None, None, None, FAKE, need,
+                                      None) == 0
+    # with tokens the same strides are rejected
+    d = _desc(ld_q=0)
+    assert lib.hstu_attention_forward(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                      None) == 1
+
+
 def test_workspace_size_grows_with_batch(lib):
     small = lib.hstu_attention_workspace_size(ctypes.byref(_desc()))
     big = lib.hstu_attention_workspace_size(ctypes.byref(_desc(num_seqs=64, total_tokens=81920,

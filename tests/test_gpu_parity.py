@@ -230,6 +230,57 @@ def test_attention_forward_mfalcon_microbatch_invariance(B):
     assert_close(outs[0], ref, "mfalcon microbatched oracle")
 
 
+def _wide_timestamps(case, seed, gap_mean, base=1_700_000_000_000):
+    """Epoch-millisecond-scale timestamps with exponential gaps (30 % of them zero, so equal
+    timestamps still occur)."""
+    rng = np.random.default_rng(seed)
+    ts = np.empty(int(case.seq_offsets[-1]), np.int64)
+    for b in range(case.num_seqs):
+        s, e = int(case.seq_offsets[b]), int(case.seq_offsets[b + 1])
+        g = rng.exponential(gap_mean, size=e - s)
+        g[rng.random(e - s) < 0.3] = 0.0
+        ts[s:e] = base + np.floor(np.cumsum(g)).astype(np.int64)
+    case.timestamps = ts
+
+
+@pytest.mark.parametrize("gap_mean,d", [(3.0e4, 64), (2.0e8, 64), (2.0e8, 128)])
+def test_attention_forward_wide_timestamps(B, gap_mean, d):
+    # time differences past 2^23 (the limit of the 32-bit per-element forms) and past 2^30 (the
+    # classifier's 32-bit reductions) on epoch-scale absolute values; NB = 128 reaches the
+    # high buckets
+    case = W.random_attention_case(14, [700, 129, 300], H=2, d=d, P=64, NB=128)
+    _wide_timestamps(case, 14, gap_mean)
+    assert_close(gpu_attention(B, case), oracle_attention(case), f"wide timestamps {gap_mean:g}")
+
+
+def test_attention_forward_long_sequence_sampled_rows(B):
+    # one 20000-token sequence beside short ones: over 200 KV tiles per late query tile, and the
+    # longest work items first
+    case = W.random_attention_case(15, [20000, 3, 700], H=2, d=64, P=1024, NB=128)
+    out = gpu_attention(B, case).float().cpu().numpy()
+    rng = np.random.default_rng(15)
+    rows = [0, 1, 127, 128, 129, 9999, 10000, 19871, 19998, 19999, 20000, 20002, 20003, 20702]
+    rows = np.unique(np.array(rows + list(rng.integers(0, 20000, size=24))))
+    ref = oracle_attention(case, rows=rows)
+    assert_close(out[rows], ref[rows], "long sequence sampled rows")
+
+
+def test_attention_forward_empty_batch(B):
+    # sequences that are all empty: nothing to compute, and zero-row views (whatever strides
+    # they report) are accepted
+    case = W.random_attention_case(16, [0, 0, 0], H=2, d=64, P=8, NB=8)
+    out = gpu_attention(B, case)
+    assert out.shape[0] == 0
+    dq, dk, dv, dp, dt = gpu_backward(B, case)
+    assert dq.shape[0] == 0 and float(dp.abs().sum()) == 0.0 and float(dt.abs().sum()) == 0.0
+
+
+def test_layer_forward_empty_batch(B):
+    case = W.random_layer_case(17, [0, 0], d_model=128, H=2, d=64, P=8, NB=8)
+    y = gpu_layer(B, case)
+    assert y.shape[0] == 0
+
+
 def test_attention_forward_fp32(B):
     case = W.random_attention_case(13, [100, 17, 130], H=2, d=32, P=20, NB=16, bf16=False)
     assert_close(gpu_attention(B, case), oracle_attention(case), "fp32")
@@ -379,6 +430,16 @@ def test_attention_backward_small(B, mask, m):
     ref = oracle_backward(case)
     for name, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got, ref):
         assert_close(g, r, f"backward {name}")
+
+
+def test_attention_backward_wide_timestamps(B):
+    # the backward's time buckets from 64-bit differences past 2^30, epoch-scale values
+    case = W.random_attention_case(31, [300, 129, 1], H=2, d=64, P=20, NB=64, qkv_std=0.5)
+    _wide_timestamps(case, 31, 2.0e8)
+    got = gpu_backward(B, case)
+    ref = oracle_backward(case)
+    for name, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got, ref):
+        assert_close(g, r, f"backward wide timestamps {name}")
 
 
 def test_attention_backward_mid_size(B):
