@@ -12,8 +12,10 @@
 // (TMA, 5-stage ring, the tile's timestamps with them) that both query tiles use.  Each query
 // tile owns two 96-column score buffers in tensor memory and its epilogue writes P (bf16) over
 // the S it has just read, so 2 x 2 x 96 + 2 x 64 (O) columns fit the 512 of an SM: while the
-// epilogue turns S(k) into P(k), the tensor core already holds S(k+1), and S(k+2) goes into the
-// buffer of S(k) once the PV that read P(k) from it has completed.
+// epilogue turns S(k) into P(k), the tensor core already holds S(k+1), and S(k+2) is issued into
+// the buffer of S(k) right after the PV that reads P(k) from it: tcgen05.mma instructions issued
+// by one thread execute in order, so its writes follow that PV's reads without a wait (the
+// pattern of the vendor's Blackwell attention, where each S buffer also holds P).
 //
 // Warpgroup 0: warp 0 TMA producer; warps 1 and 3 issue the tcgen05.mma of query tile 0 and 1
 // (one thread each; warp 1 also owns the TMEM allocation); warp 2 classifies each KV tile (bias
@@ -76,7 +78,6 @@ struct PairSmem {
   uint64_t cls_ready[kStages];           // the tile's classification and timestamps
   uint64_t s_full[2][2];
   uint64_t p_full[2][2];
-  uint64_t pv_done[2][2];                // the PV that read P from score buffer [a][b]
   uint64_t o_full[2];
   uint64_t o_empty[2];
   uint64_t drain[2];
@@ -466,7 +467,6 @@ struct IssuerCtx {
   uint32_t buf0, o_col;            // score buffer 1 lies 96 columns after buffer 0
   uint64_t* s_full0;               // buffer 1's barriers follow buffer 0's
   uint64_t* p_full0;
-  uint64_t* pv_done0;
   uint64_t* o_full;
   uint64_t* o_empty;
   uint64_t* kv_full;
@@ -495,7 +495,6 @@ __device__ __forceinline__ void issue_pv(const IssuerCtx& c, int b, int st, bool
   for (int kk = 0; kk < kKV / 16; ++kk)
     mma_bf16_ts(c.o_col, pb + (kk < 3 ? 8 * kk : 48 + 8 * (kk - 3)), dv + 128 * kk, idesc,
                 (acc || kk > 0) ? 1u : 0u);
-  mma_commit(c.pv_done0 + b);
 }
 
 // 20 warps launch with 96 registers each (5 warps per SM sub-partition); after set-up
@@ -546,7 +545,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sm.s_full[a][b], 1);
         mbar_init(&sm.p_full[a][b], 8);  // one elected lane per epilogue warp of tile a
-        mbar_init(&sm.pv_done[a][b], 1);
       }
       mbar_init(&sm.o_full[a], 1);
       mbar_init(&sm.o_empty[a], 8);
@@ -636,7 +634,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         c.buf0 = tmem + col_buf(a, 0);
         c.s_full0 = &sm.s_full[a][0];
         c.p_full0 = &sm.p_full[a][0];
-        c.pv_done0 = &sm.pv_done[a][0];
         c.o_col = tmem + col_o(a);
         c.o_full = &sm.o_full[a];
         c.o_empty = &sm.o_empty[a];
@@ -658,15 +655,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sl = qi & 1;
           const uint64_t dq = sl ? c.dq[1] : c.dq[0];
           ok = mbar_wait(&sm.q_full[sl], (qi >> 1) & 1, abort_flag, g.status);
-          // prologue: the first two S (the epilogue read their buffers' previous contents
-          // before the P that this thread has already consumed)
+          // prologue: the first two S (the buffers' previous P, of the last item, went to PVs
+          // this thread has already issued, so in-order execution keeps them intact)
           const int first = ok ? min(2, cnt) : 0;
           for (int kk = 0; kk < first; ++kk) {
             const int u = gu + (kk < nh ? kk : cb + (kk - nh));
             // cls_ready follows kv_full: the classifier waited for the tile's load
             ok = mbar_wait(&sm.cls_ready[u % kStages], (u / kStages) & 1, abort_flag, g.status);
-            // the buffer's previous P has been read by its PV
-            if (ok && gs >= 2) ok = mbar_wait(c.pv_done0 + (gs & 1), ((gs - 2) >> 1) & 1, abort_flag, g.status);
             if (!ok) break;
             tc_fence_after();
             issue_s(c, dq, gs & 1, u % kStages);
@@ -691,8 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   st2 -= kStages;
                   ph2 ^= 1;
                 }
-                ok = mbar_wait(&sm.cls_ready[st2], ph2, abort_flag, g.status) &&
-                     mbar_wait(c.pv_done0 + (gs & 1), ((gs - 2) >> 1) & 1, abort_flag, g.status);
+                // into the buffer whose P the PV just issued reads: issued after it by this
+                // thread, so executed after it
+                ok = mbar_wait(&sm.cls_ready[st2], ph2, abort_flag, g.status);
                 if (!ok) break;
                 tc_fence_after();
                 issue_s(c, dq, gs & 1, st2);
@@ -963,8 +959,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         rc = segment_ctx(rc, sm.cls[st][8 * a + 2 * quad + h], c0t, h, ti, row_valid, use_time,
                          g.NB, &sm.tmin[st][h], &sm.tmax[st][h], sm.rab_time_h);
-        // S(k) was issued after PV(k-2) had completed (same buffer), and all eight warps of
-        // tile a finished tile k-2 (its P preceded that PV): tile k-2's stage is free
+        // S(k) is complete, and so is every MMA this tile's issuer issued before it, PV(k-2)
+        // among them: tile k-2's stage is free for this query tile
         if (k >= 2 && lead) mbar_arrive(&sm.kv_empty[(gu + plan.uidx(a, k - 2)) % kStages]);
         tc_fence_after();
         const uint32_t seg_addr = lane_addr + col_buf(a, b) + kSeg * h;
