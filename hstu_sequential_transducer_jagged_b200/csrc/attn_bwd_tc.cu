@@ -52,7 +52,7 @@ struct BwdSmem {
   alignas(128) long long tq[kQStages][kTsStride];  // timestamps of the query tile
   uint64_t kv_full, kv_empty;
   uint64_t qd_full[kQStages], qd_empty[kQStages];
-  uint64_t s_full, p_full, mm_done, dq_full, dq_empty, acc_full, acc_empty, drain;
+  uint64_t s_full, p_full, dq_full, dq_empty, acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
   // followed by float bins[2P+1 + NB]
@@ -286,7 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.p_full, 8);
-    mbar_init(&sm.mm_done, 1);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_empty, 4);
     mbar_init(&sm.acc_full, 1);
@@ -361,8 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = gs % kQStages;
           const bool first = qt == kt;
           ok = mbar_wait(&sm.qd_full[st], (gs / kQStages) & 1, abort_flag, g.status);
-          // the previous step's MMAs read P^T / dS^T (aliased with S^T / dP^T) and the dS tile
-          if (ok && gs > 0) ok = mbar_wait(&sm.mm_done, (gs - 1) & 1, abort_flag, g.status);
+          // The previous step's dV, dK and dQ MMAs read P^T / dS^T (aliased with S^T / dP^T)
+          // and the dS tile.  This thread issued them before the S^T / dP^T MMAs below, and one
+          // thread's MMAs execute in order, so no wait is needed; the epilogue writes the next
+          // dS tile only after s_full, whose commit follows those MMAs too.
           if (!ok) break;
           tc_fence_after();
           const uint32_t qb = smem_u32(sm.q[st]), ob = smem_u32(sm.dO[st]);
@@ -394,7 +395,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ss(tmem + kColDQ, smem_desc_sw128(dsb + kk * 2048, kTileBytes, 1024),
                         smem_desc_sw128(kb + kk * 2048, kTileBytes, 1024), id_q, kk > 0 ? 1u : 0u);
           mma_commit(&sm.dq_full);
-          mma_commit(&sm.mm_done);
           mma_commit(&sm.qd_empty[st]);
         }
         if (!ok) break;
