@@ -14,15 +14,17 @@
 //   Sᵀ = K Qᵀ and dPᵀ = V dOᵀ                       (smem x smem MMAs, M = keys, N = queries)
 //   epilogue (one key row per thread): x = alpha s + bias, σ = 1/2 + tanh(x/2)/2, P = x σ,
 //     dS = dP σ (1 + x (1 - σ)), 0 where the mask hides the pair; Pᵀ and (alpha dS)ᵀ as bf16
-//     over the first halves of the Sᵀ / dPᵀ columns, (alpha dS)ᵀ also to shared memory (the
+//     over the first half of each 32-query chunk's own Sᵀ / dPᵀ columns (a chunk is one warp's,
+//     so no warp writes columns another still reads), (alpha dS)ᵀ also to shared memory (the
 //     MN-major A operand of dQ); bias-table gradients summed in registers along runs of one
 //     table index and added to shared-memory bins when the index changes
 //   dV += Pᵀ dO,  dK += (alpha dS)ᵀ Q                 (tensor-memory A operand)
 //   dQ  = (alpha dS) K -> tensor memory -> 4 drain warps add it (16-byte vector atomics) to an
 //     fp32 accumulator in global memory, converted to bf16 after the kernel.
 // TMEM columns: Sᵀ 0..127, dPᵀ 128..255, dV 256..319, dK 320..383, dQ 384..447.
-// Warps: 0 TMA producer, 1 MMA issuer (and the TMEM allocation), 2-3 idle, 4-11 epilogue (lane
-// quarter w % 4, query half (w - 4) / 4), 12-15 dQ drain (lane quarter w % 4).
+// Warps: 0 TMA producer, 1 MMA issuer (and the TMEM allocation), 2-17 epilogue (lane quarter
+// w % 4, 32-query chunk (w - 2) / 4: four warps per SM sub-partition to hide the latency of the
+// per-element chain), 18-21 dQ drain (lane quarter w % 4).
 // Items are visited in the reverse of the forward's longest-first order (which sorts by the
 // number of key tiles a query tile visits), so that key tiles near the start of long sequences,
 // which walk the most query tiles, start first.
@@ -37,7 +39,9 @@ namespace {
 constexpr int kD = 64;
 constexpr int kT = 128;
 constexpr int kQStages = 2;
-constexpr int kThreads = 512;
+constexpr int kThreads = 704;   // 22 warps
+constexpr int kEpiWarps = 16;
+constexpr int kEpiFirst = 2;
 constexpr int kTileBytes = kT * kD * 2;   // 16 KB
 constexpr int kTsStride = 144;            // 1152 bytes per stage (TMA destination 128-aligned)
 constexpr int kTsBox = 130;
@@ -68,6 +72,26 @@ __device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
         "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
         "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
       :
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  __syncwarp();
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+
+// Each thread of a warp writes 8 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 
@@ -187,17 +211,17 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
   return kChunkConst;
 }
 
-// One 32-column block of a key row: P and alpha dS (bf16 pairs) from S and dP, and the bias
-// gradients.  i_first: query index of the block's first column; tq_c: its timestamps.
-template <int V>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
-                                          uint32_t (&pk)[16], uint32_t (&dk)[16], int i_first,
+// W columns of a key row (half of a 32-query block): P and alpha dS (bf16 pairs) from S and dP,
+// and the bias gradients.  i_first: query index of the first column; tq_c: its timestamps.
+template <int V, int W>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[W], const uint32_t (&dp)[W],
+                                          uint32_t (&pk)[W / 2], uint32_t (&dk)[W / 2], int i_first,
                                           const long long* tq_c, const BwdRow& r,
                                           const BwdTabs& t, float cbias, int cpidx, int ctidx,
                                           BinRun& run_p, BinRun& run_t) {
   float sum = 0.f;  // constant classes: the block's dS total for the constant bins
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
+  for (int e = 0; e < W; e += 2) {
     float pv[2], dsa[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -285,11 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.qd_empty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full, 8);
+    mbar_init(&sm.p_full, kEpiWarps);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_empty, 4);
     mbar_init(&sm.acc_full, 1);
-    mbar_init(&sm.acc_empty, 8);
+    mbar_init(&sm.acc_empty, kEpiWarps);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbarrier_init();
@@ -381,7 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk) {  // 16 queries per step; P^T / dS^T columns
-            const uint32_t pc = kk < 4 ? 8 * kk : 64 + 8 * (kk - 4);
+            // queries 16 kk..: chunk kk / 2 keeps its 32 queries' pairs in its first 16 columns
+            const uint32_t pc = 32 * (kk >> 1) + 8 * (kk & 1);
             mma_bf16_ts(tmem + kColDV, tmem + kColST + pc, smem_desc_sw128(ob + kk * 2048, kTileBytes, 1024),
                         id_kv, (!first || kk > 0) ? 1u : 0u);
             mma_bf16_ts(tmem + kColDK, tmem + kColDPT + pc, smem_desc_sw128(qb + kk * 2048, kTileBytes, 1024),
@@ -407,9 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= kEpiFirst && warp < kEpiFirst + kEpiWarps) {
     // ---------------------------------------------------------------- epilogue
-    const int quad = warp & 3, hq = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int qc = (warp - kEpiFirst) >> 2;  // 32-query chunk of every query tile
+    const int hq = qc >> 1, ch = qc & 1;     // its half of the dS tile and place in it
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float alpha = g.alpha;
     // Bias-gradient runs: along one key row the table index changes only where the clamped
@@ -457,46 +484,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const long long* tq = sm.tq[st] + ((it.row0 + qt * kT) & 1);
         uint8_t* ds_row = sm.ds + hq * kTileBytes + (quad * 32 + lane) * 128;
+        const int rr = quad * 32 + lane;
+        const uint32_t col = 32 * qc;
+        const int i0 = qt * kT + static_cast<int>(col);
+        const long long* tq_c = tq + col;
+        float cbias = 0.f;
+        int cpidx = 0, ctidx = 0;
+        const int cls = kFast ? chunk_class(i0, j0, L, n, tabs, tq_c, tj_lo, tj_hi, cbias, cpidx,
+                                            ctidx)
+                              : kChunkGeneral;
 #pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {  // 32 query columns per chunk
-          const uint32_t col = 64 * hq + 32 * ch;
-          const int i0 = qt * kT + static_cast<int>(col);
-          const long long* tq_c = tq + col;
-          float cbias = 0.f;
-          int cpidx = 0, ctidx = 0;
-          const int cls = kFast ? chunk_class(i0, j0, L, n, tabs, tq_c, tj_lo, tj_hi, cbias,
-                                              cpidx, ctidx)
-                                : kChunkGeneral;
-          uint32_t pk[16], dk[16];
+        for (int hf = 0; hf < 2; ++hf) {  // 16 queries at a time (fewer live registers)
+          const uint32_t c16 = col + 16 * hf;
+          uint32_t pk[8], dk[8];
           if (cls == kChunkZero) {
 #pragma unroll
-            for (int z = 0; z < 16; ++z) pk[z] = dk[z] = 0u;
+            for (int z = 0; z < 8; ++z) pk[z] = dk[z] = 0u;
           } else {
-            uint32_t s[32], dp[32];
-            tmem_ld32(lane_addr + kColST + col, s);
-            tmem_ld32(lane_addr + kColDPT + col, dp);
-            tmem_wait_ld32(s);
-            tmem_wait_ld32(dp);
+            uint32_t sv[16], dp[16];
+            tmem_ld16(lane_addr + kColST + c16, sv);
+            tmem_ld16(lane_addr + kColDPT + c16, dp);
+            tmem_wait_ld16(sv);
+            tmem_wait_ld16(dp);
             if (cls == kChunkConst)
-              bwd_chunk<kChunkConst>(s, dp, pk, dk, i0, tq_c, row, tabs, cbias, cpidx, ctidx,
-                                     run_p, run_t);
+              bwd_chunk<kChunkConst, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row, tabs,
+                                         cbias, cpidx, ctidx, run_p, run_t);
             else if (cls == kChunkTimeConst)
-              bwd_chunk<kChunkTimeConst>(s, dp, pk, dk, i0, tq_c, row, tabs, cbias, cpidx,
-                                         ctidx, run_p, run_t);
+              bwd_chunk<kChunkTimeConst, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row,
+                                             tabs, cbias, cpidx, ctidx, run_p, run_t);
             else
-              bwd_chunk<kChunkGeneral>(s, dp, pk, dk, i0, tq_c, row, tabs, cbias, cpidx, ctidx,
-                                       run_p, run_t);
+              bwd_chunk<kChunkGeneral, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row,
+                                           tabs, cbias, cpidx, ctidx, run_p, run_t);
           }
-          // P^T / (a dS)^T over the already-read first half of this warp's 64 columns
-          tmem_st16(lane_addr + kColST + 64 * hq + 16 * ch, pk);
-          tmem_st16(lane_addr + kColDPT + 64 * hq + 16 * ch, dk);
-          // (a dS)^T row to shared memory: chunk cc (8 queries) of this half at cc ^ (row & 7)
-          const int rr = quad * 32 + lane;
+          // P^T / (a dS)^T over the chunk's own first 16 columns, already read by this warp
+          tmem_st8(lane_addr + kColST + col + 8 * hf, pk);
+          tmem_st8(lane_addr + kColDPT + col + 8 * hf, dk);
+          // (a dS)^T row to shared memory: 8-query block cb of this half at cb ^ (row & 7)
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int chunk = 4 * ch + cc;
-            uint4 val = make_uint4(dk[4 * cc], dk[4 * cc + 1], dk[4 * cc + 2], dk[4 * cc + 3]);
-            *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (rr & 7)) * 16)) = val;
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int cb = 4 * ch + 2 * hf + c2;
+            const uint4 val = make_uint4(dk[4 * c2], dk[4 * c2 + 1], dk[4 * c2 + 2], dk[4 * c2 + 3]);
+            *reinterpret_cast<uint4*>(ds_row + ((cb ^ (rr & 7)) * 16)) = val;
           }
         }
         tmem_wait_st();
@@ -506,22 +534,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm.p_full);
       }
       if (!ok) break;
-      // the item's dV, dK: this warp's 32 of the 64 columns of each
+      // the item's dV, dK: this warp's 16 of the 64 columns of each
       ok = warp_wait(&sm.acc_full, jj & 1, abort_flag, g.status);
       if (!ok) break;
       tc_fence_after();
-      uint32_t a[32];
+      uint32_t a[16];
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
-        tmem_ld32(lane_addr + (which ? kColDK : kColDV) + 32 * hq, a);
-        tmem_wait_ld32(a);
+        tmem_ld16(lane_addr + (which ? kColDK : kColDV) + 16 * qc, a);
+        tmem_wait_ld16(a);
         if (jvalid) {
           // a layer's backward: dpre = dK (dV) ⊙ SiLU'(Z) before the one rounding to bf16
           const float* zrow = which ? zg.k : zg.v;
           if (zrow != nullptr) {
-            zrow += static_cast<int64_t>(it.row0 + jrow) * zg.ld + head * kD + 32 * hq;
+            zrow += static_cast<int64_t>(it.row0 + jrow) * zg.ld + head * kD + 16 * qc;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
+            for (int e = 0; e < 16; e += 4) {
               const float4 z4 = *reinterpret_cast<const float4*>(zrow + e);
               a[e] = __float_as_uint(__uint_as_float(a[e]) * silu_grad_z(z4.x));
               a[e + 1] = __float_as_uint(__uint_as_float(a[e + 1]) * silu_grad_z(z4.y));
@@ -531,9 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __nv_bfloat16* dst = (which ? dk_out : dv_out) +
                                static_cast<int64_t>(it.row0 + jrow) * (which ? ld_dk : ld_dv) +
-                               head * kD + 32 * hq;
+                               head * kD + 16 * qc;
 #pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) {
+          for (int w4 = 0; w4 < 2; ++w4) {
             uint4 vv;
             vv.x = pack_bf16x2(__uint_as_float(a[8 * w4 + 0]), __uint_as_float(a[8 * w4 + 1]));
             vv.y = pack_bf16x2(__uint_as_float(a[8 * w4 + 2]), __uint_as_float(a[8 * w4 + 3]));
@@ -549,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     run_p.flush(tabs.bins_pos);
     run_t.flush(tabs.bins_time);
-  } else if (warp >= 12) {
+  } else if (warp >= kEpiFirst + kEpiWarps) {
     // ---------------------------------------------------------------- dQ drain
     const int quad = warp & 3;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);

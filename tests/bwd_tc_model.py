@@ -134,7 +134,7 @@ def chunk_class(i0, j0, L, n, P, NB, tq_c, tj, jvalid, tabp, tabt, use_pos=True,
     return "const", np.float32(tterm), 0, ctidx
 
 
-DEFAULT_KNOBS = dict(ds_swizzle=True, dq_lbo=kTileBytes, split_pc=True, p_col_step=16)
+DEFAULT_KNOBS = dict(ds_swizzle=True, dq_lbo=kTileBytes, split_pc=True, p_col_step=32)
 
 
 def run(case, fast, knobs=None):
@@ -275,10 +275,10 @@ def run(case, fast, knobs=None):
                                         run_add("t", npos, ctidx, csum[l])
                                 pk = pack(pv[:, 0::2], pv[:, 1::2])
                                 dk_ = pack(dsa[:, 0::2], dsa[:, 1::2])
-                            # TMEM stores: 16 columns at 64 hq + 16 ch
+                            # TMEM stores: 16 columns at the chunk's own first columns, 64 hq + 32 ch
                             pcol = kColST + 64 * hq + kn['p_col_step'] * ch
                             tm.w[lanes, pcol:pcol + 16] = pk
-                            tm.w[lanes, kColDPT + 64 * hq + 16 * ch:kColDPT + 64 * hq + 16 * ch + 16] = dk_
+                            tm.w[lanes, kColDPT + 64 * hq + 32 * ch:kColDPT + 64 * hq + 32 * ch + 16] = dk_
                             # dS row to shared memory: chunk (4 ch + cc) at (chunk ^ (rr & 7)) * 16
                             rr = quad * 32 + np.arange(32)
                             ds_row = DS_B + hq * kTileBytes + rr * 128
@@ -291,7 +291,7 @@ def run(case, fast, knobs=None):
                                 sm.write_u16(addr, halves)
                 # dV += P^T dO, dK += (a dS)^T Q  (TS; B MN-major, LBO = tile bytes)
                 for kk in range(8):
-                    pc = (8 * kk if kk < 4 else 64 + 8 * (kk - 4)) if kn['split_pc'] else 8 * kk
+                    pc = (32 * (kk >> 1) + 8 * (kk & 1)) if kn['split_pc'] else 8 * kk
                     acc = (not first_item_step) or kk > 0
                     mma(tm, kColDV, tmem_a(tm, kColST + pc),
                         decode_mnmajor(sm, DO_B + kk * 2048, 64, kTileBytes, 1024), acc)

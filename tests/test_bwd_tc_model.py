@@ -58,7 +58,7 @@ def test_model_matches_oracle(name, fast):
 
 
 @pytest.mark.parametrize("knob", [dict(ds_swizzle=False), dict(dq_lbo=8192),
-                                  dict(split_pc=False), dict(p_col_step=32)])
+                                  dict(split_pc=False), dict(p_col_step=16)])
 def test_planted_layout_mistakes_fail(knob):
     case = CASES["causal"]()
     with np.errstate(all="ignore"):  # misplaced operands read garbage
