@@ -32,3 +32,23 @@ def test_attention_forward_alibi_bias(B, d, mask, m):
                                     m_p, m_t, num_heads=2, d_qk=d, d_v=d, num_time_buckets=NB,
                                     alpha=case.alpha, mask=mask, num_candidates=m)
     assert_close(out, ref, f"alibi d={d} m={m}")
+
+
+def test_attention_forward_alibi_bias_long_sequences(B):
+    # tables spanning P = 2599 >= the longest sequence: too wide for the paired kernel's shared
+    # copy, so the single-tile tensor-core forward reads the table from global memory
+    case = W.random_attention_case(29, [2600, 700, 1], H=2, d=64, P=8, NB=32, gap_mean=600.0,
+                                   qkv_std=0.5)
+    m_p, m_t, NB = 0.002, 0.05, 32
+    P = int(case.max_seq_len) - 1
+    pos, tim = B.alibi_tables(m_p, m_t, P, NB)
+    bf = torch.bfloat16
+    out = B.attention_forward(dev(case.q, bf), dev(case.k, bf), dev(case.v, bf),
+                              dev(case.seq_offsets), case.max_seq_len, dev(case.timestamps),
+                              dev(pos), dev(tim), num_heads=2, max_pos_dist=P,
+                              num_time_buckets=NB, alpha=case.alpha)
+    torch.cuda.synchronize()
+    ref = O.attention_forward_alibi(case.q, case.k, case.v, case.seq_offsets, case.timestamps,
+                                    m_p, m_t, num_heads=2, d_qk=64, d_v=64, num_time_buckets=NB,
+                                    alpha=case.alpha)
+    assert_close(out, ref, "alibi long sequences")
