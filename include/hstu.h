@@ -55,7 +55,7 @@ typedef struct CUstream_st* hstu_stream_t; /* a cudaStream_t; NULL = the legacy 
 typedef enum {
   HSTU_OK = 0,
   HSTU_ERR_INVALID_ARG = 1,   /* a host-side argument check failed; nothing was launched */
-  HSTU_ERR_UNSUPPORTED = 2,   /* a valid combination this build does not implement */
+  HSTU_ERR_UNSUPPORTED = 2,   /* a valid combination the library does not implement */
   HSTU_ERR_WORKSPACE = 3,     /* ws is NULL, misaligned or smaller than *_workspace_size() */
   HSTU_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
   HSTU_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (reported via the status word) */
