@@ -279,11 +279,6 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// bar.sync on a named barrier shared by `count` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // True in every lane iff pred holds in every lane of the (converged) warp.  Branches that enclose
 // .sync.aligned tcgen05 instructions are taken on warp-uniform conditions only.
 __device__ __forceinline__ bool warp_all(bool pred) { return __all_sync(0xffffffffu, pred); }
