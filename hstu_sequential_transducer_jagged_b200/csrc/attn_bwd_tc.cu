@@ -153,8 +153,31 @@ struct BwdTabs {
 
 // Classes of a 32-query x 32-key block of one warp (warp-uniform): every pair hidden; every pair
 // visible with one position bin and one time bucket; every pair visible with one time bucket;
-// anything else (per-element mask, bias and bins).
-constexpr int kChunkGeneral = 0, kChunkTimeConst = 1, kChunkConst = 2, kChunkZero = 3;
+// the same two with every distance inside the position band (diagonal bin sums, see DiagBins),
+// the second also with per-element time buckets from 32-bit differences; anything else
+// (per-element mask, bias and bins).
+constexpr int kChunkGeneral = 0, kChunkTimeConst = 1, kChunkConst = 2, kChunkZero = 3,
+              kChunkBandTC = 4, kChunkBandT32 = 5;
+
+// Position-bin sums of a fully visible 32 x 32 block whose distances all lie inside the band:
+// the pair (key j0 + l, query i0 + e) falls in diagonal e - l + 31 (0..62), i.e. bin
+// i0 - j0 - 31 + P + (e - l + 31).  Lane m keeps diagonals m and m + 32: at column e the value of
+// lane (e + 31 - m) mod 32 belongs to diagonal m when m >= e and to m + 32 otherwise, so one
+// shuffle per column replaces a shared-memory atomic per element; 63 atomics close the block.
+struct DiagBins {
+  float lo, hi;
+  __device__ __forceinline__ void add(int e, float v) {
+    const int m = threadIdx.x & 31;
+    const float w = __shfl_sync(0xffffffffu, v, (e - 1 - m) & 31);
+    if (m >= e) lo += w; else hi += w;
+  }
+  __device__ __forceinline__ void flush(float* bins, int first_bin) {
+    const int m = threadIdx.x & 31;
+    atomicAdd(&bins[first_bin + m], lo);
+    if (m < 31) atomicAdd(&bins[first_bin + 32 + m], hi);
+    lo = hi = 0.f;
+  }
+};
 
 __device__ __forceinline__ long long warp_min64(long long v) {
 #pragma unroll
@@ -185,6 +208,9 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
   const int j1 = j0 + 31;
   if (i0 >= L || j0 >= L || i0 + 31 < j0) return kChunkZero;
   if (!(i0 >= j1 && i0 + 31 < L && j1 < n)) return kChunkGeneral;  // not every pair visible
+  // every distance i - j of the block in [0, P] and every query a history token: the position
+  // index is i - j + P, no clamp
+  const bool band = t.use_pos && i0 + 31 < n && i0 + 31 - j0 <= t.P;
   float tterm = 0.f;
   ctidx = 0;
   if (t.use_time) {
@@ -192,7 +218,11 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
     const long long tq_lo = warp_min64(tq), tq_hi = warp_max64(tq);
     const int b_lo = time_bucket64(tq_lo - tj_hi, t.NB);
     const int b_hi = time_bucket64(tq_hi - tj_lo, t.NB);
-    if (b_lo != b_hi) return kChunkGeneral;
+    if (b_lo != b_hi) {
+      // per-element buckets: from the 32-bit differences when all of them lie in (-2^23, 2^23)
+      const bool small = tq_hi - tj_lo < (1ll << 23) && tq_lo - tj_hi > -(1ll << 23);
+      return (small && (band || !t.use_pos)) ? kChunkBandT32 : kChunkGeneral;
+    }
     ctidx = b_lo;
     tterm = t.time[b_lo];
   }
@@ -201,7 +231,7 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
     // keys are history tokens (position = index); queries past the history sit at n
     if (!pos_segment_beyond_clamp(i0 < n ? i0 : n, j1, t.P)) {
       cbias = tterm;
-      return kChunkTimeConst;
+      return band ? kChunkBandTC : kChunkTimeConst;
     }
     cpidx = 2 * t.P;  // every distance at or beyond the clamp
     cbias = t.pos[cpidx] + tterm;
@@ -266,6 +296,50 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[W], const uint32_t
   }
   if (V == kChunkConst && t.use_pos) run_p.add(t.bins_pos, cpidx, sum);
   if (V != kChunkGeneral && t.use_time) run_t.add(t.bins_time, ctidx, sum);
+}
+
+// W columns of a fully visible band block (classes kChunkBandTC and kChunkBandT32): the same P and
+// alpha dS as bwd_chunk, with the position bins summed by diagonal (dg) and, for kChunkBandT32,
+// the time bucket of each pair from the low 32 bits of the two timestamps (every difference of
+// the block lies in (-2^23, 2^23)).  eg0: block column of the first of the W queries; pb: this
+// key row's position index for that query (i - j + P); tq_lo: the queries' timestamps as pairs
+// of 32-bit words, low word first.
+template <int V, int W>
+__device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uint32_t (&dp)[W],
+                                               uint32_t (&pk)[W / 2], uint32_t (&dk)[W / 2],
+                                               int eg0, int pb, const unsigned* tq_lo,
+                                               unsigned tj_lo, const BwdTabs& t, float cbias,
+                                               int ctidx, DiagBins& dg, BinRun& run_t) {
+  float sum = 0.f;  // kChunkBandTC: the block's dS total for its one time bin
+#pragma unroll
+  for (int e = 0; e < W; e += 2) {
+    float pv[2], dsa[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float bias = V == kChunkBandTC ? cbias : 0.f;
+      if (t.use_pos) bias += t.pos[pb + e + u];
+      int bidx = 0;
+      if (V == kChunkBandT32) {
+        bidx = bucket_small(static_cast<int>(tq_lo[2 * (e + u)] - tj_lo), t.NB - 1);
+        bias += t.time[bidx];
+      }
+      const float x = fmaf(t.alpha, __uint_as_float(s[e + u]), bias);
+      const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
+      const float p = x * sg;
+      const float dsv = __uint_as_float(dp[e + u]) * sg * fmaf(x, 1.f - sg, 1.f);
+      if (t.use_pos) dg.add(eg0 + e + u, dsv);
+      if (V == kChunkBandT32) {
+        run_t.add(t.bins_time, bidx, dsv);
+      } else {
+        sum += dsv;
+      }
+      pv[u] = p;
+      dsa[u] = t.alpha * dsv;
+    }
+    pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+    dk[e >> 1] = pack_bf16x2(dsa[0], dsa[1]);
+  }
+  if (V == kChunkBandTC && t.use_time) run_t.add(t.bins_time, ctidx, sum);
 }
 
 // Items: (sequence, 128-row key tile) from the work list built with one tile per item, times heads.
@@ -493,6 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cls = kFast ? chunk_class(i0, j0, L, n, tabs, tq_c, tj_lo, tj_hi, cbias, cpidx,
                                             ctidx)
                               : kChunkGeneral;
+        DiagBins dg{0.f, 0.f};
+        const unsigned* tq_lo = reinterpret_cast<const unsigned*>(tq_c);
+        const unsigned tj_lo32 = static_cast<unsigned>(row.tj);
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {  // 16 queries at a time (fewer live registers)
           const uint32_t c16 = col + 16 * hf;
@@ -509,6 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (cls == kChunkConst)
               bwd_chunk<kChunkConst, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row, tabs,
                                          cbias, cpidx, ctidx, run_p, run_t);
+            else if (cls == kChunkBandTC)
+              bwd_chunk_band<kChunkBandTC, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
+                                               tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
+                                               run_t);
+            else if (cls == kChunkBandT32)
+              bwd_chunk_band<kChunkBandT32, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
+                                                tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
+                                                run_t);
             else if (cls == kChunkTimeConst)
               bwd_chunk<kChunkTimeConst, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row,
                                              tabs, cbias, cpidx, ctidx, run_p, run_t);
@@ -527,6 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(ds_row + ((cb ^ (rr & 7)) * 16)) = val;
           }
         }
+        if ((cls == kChunkBandTC || cls == kChunkBandT32) && use_pos)
+          dg.flush(tabs.bins_pos, i0 - j0 - 31 + g.P);
         tmem_wait_st();
         fence_async_smem();  // the dS tile is read by the dQ MMA (async proxy)
         tc_fence_before();

@@ -404,11 +404,12 @@ def test_mfalcon_workload_sampled_sequence(B):
 
 
 # ----------------------------------------------------------------------- attention backward
-def gpu_backward(B, case):
+def gpu_backward(B, case, use_time=True, use_pos=True):
     dt = act(case)
     q, k, v, d_o = (dev(case.q, dt), dev(case.k, dt), dev(case.v, dt), dev(case.d_o, dt))
     res = B.attention_backward(q, k, v, d_o, dev(case.seq_offsets), case.max_seq_len,
-                               dev(case.timestamps), dev(case.rab_pos), dev(case.rab_time),
+                               dev(case.timestamps), dev(case.rab_pos) if use_pos else None,
+                               dev(case.rab_time) if use_time else None,
                                num_heads=case.num_heads, max_pos_dist=case.max_pos_dist,
                                num_time_buckets=case.num_time_buckets, alpha=case.alpha,
                                mask=case.mask, num_candidates=case.num_candidates,
@@ -417,9 +418,10 @@ def gpu_backward(B, case):
     return res
 
 
-def oracle_backward(case):
+def oracle_backward(case, use_time=True, use_pos=True):
     return O.attention_backward(case.q, case.k, case.v, case.d_o, case.seq_offsets,
-                                case.timestamps, case.rab_pos, case.rab_time, **attn_kw(case))
+                                case.timestamps, case.rab_pos if use_pos else None,
+                                case.rab_time if use_time else None, **attn_kw(case))
 
 
 @pytest.mark.parametrize("mask,m", [(W.MASK_CAUSAL, 0), (W.MASK_MFALCON, 50)])
@@ -440,6 +442,34 @@ def test_attention_backward_wide_timestamps(B):
     ref = oracle_backward(case)
     for name, g, r in zip(("dq", "dk", "dv", "d_rab_pos", "d_rab_time"), got, ref):
         assert_close(g, r, f"backward wide timestamps {name}")
+
+
+@pytest.mark.parametrize("use_time,use_pos,mask,m,wide", [
+    (True, True, W.MASK_CAUSAL, 0, False),
+    (False, True, W.MASK_CAUSAL, 0, False),
+    (True, False, W.MASK_CAUSAL, 0, False),
+    (True, True, W.MASK_MFALCON, 40, False),
+    (True, True, W.MASK_CAUSAL, 0, True),
+    (True, False, W.MASK_CAUSAL, 0, True),
+])
+def test_attention_backward_band_blocks(B, use_time, use_pos, mask, m, wide):
+    # P = 160 over sequences of up to 740 tokens: 32 x 32 blocks whose distances all lie in the
+    # position band sum the position bins by diagonal, with one time bucket or per-element
+    # buckets from 32-bit differences; blocks past the band, with candidates, on the diagonal or
+    # (wide) with differences past 2^23 take the other paths
+    case = W.random_attention_case(33 + m, [700 + m, 300 + m, 65 + m, 1], H=2, d=64, P=160,
+                                   NB=32, mask=mask, num_candidates=m, gap_mean=20.0,
+                                   qkv_std=0.5)
+    if wide:
+        _wide_timestamps(case, 33, 2.0e4)
+    got = gpu_backward(B, case, use_time, use_pos)
+    ref = oracle_backward(case, use_time, use_pos)
+    names = ("dq", "dk", "dv", "d_rab_pos", "d_rab_time")
+    for name, g, r in zip(names, got, ref):
+        if g is None:
+            assert (name == "d_rab_pos" and not use_pos) or (name == "d_rab_time" and not use_time)
+            continue
+        assert_close(g, r, f"backward band blocks {name}")
 
 
 def test_attention_backward_mid_size(B):
