@@ -53,7 +53,7 @@ cudaError_t launch_attn_bwd_simt(int dtype, int D, const AttnGeom& g, const void
                                  float* d_pos, float* d_time, int grid, cudaStream_t stream);
 cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdo,
-                               const CUtensorMap& tts, const AttnGeom& g, __nv_bfloat16* dq,
+                               const CUtensorMap& tts, const CUtensorMap& tdq, const AttnGeom& g, __nv_bfloat16* dq,
                                int64_t ld_dq, __nv_bfloat16* dk, int64_t ld_dk,
                                __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc, float* d_pos,
                                float* d_time, int grid, bool fast, const SiluGradZ& zg,
@@ -174,6 +174,22 @@ bool make_epilogue_maps(CUtensorMap* tc, CUtensorMap* tr, const void* C, int64_t
   if (R != nullptr && !make_map_bf16_sw(tr, R, M, N, ldr, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return false;
   return true;
+}
+
+// 2D fp32 tensor map over a row-major [rows, cols] matrix with row stride ld (elements), box
+// {box_cols, box_rows}, 128-byte swizzle (the attention backward's dQ reduction target).
+bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                  uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -688,8 +704,10 @@ hstu_status_t attn_backward_impl(const hstu_attn_desc_t* d, const void* q, const
         (use_time && !make_map_i64_1d(&tts, d->timestamps, T, attn_bwd_tc_ts_box())))
       return HSTU_ERR_CUDA;
     float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.total_attn);
+    CUtensorMap tdq;
+    if (!make_map_f32(&tdq, dq_acc, T, cols, cols, 32, 32)) return HSTU_ERR_CUDA;
     const int pgrid = grid < num_sms_current() ? grid : num_sms_current();
-    e = launch_attn_bwd_tc(tq, tk, tv, tdo, tts, g, static_cast<__nv_bfloat16*>(dq), d->ld_q,
+    e = launch_attn_bwd_tc(tq, tk, tv, tdo, tts, tdq, g, static_cast<__nv_bfloat16*>(dq), d->ld_q,
                            static_cast<__nv_bfloat16*>(dk), d->ld_k,
                            static_cast<__nv_bfloat16*>(dv), d->ld_v, dq_acc, d_rab_pos,
                            d_rab_time, pgrid, true, zg, s);

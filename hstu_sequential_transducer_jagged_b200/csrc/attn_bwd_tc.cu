@@ -19,8 +19,11 @@
 //     MN-major A operand of dQ); bias-table gradients summed in registers along runs of one
 //     table index and added to shared-memory bins when the index changes
 //   dV += Pᵀ dO,  dK += (alpha dS)ᵀ Q                 (tensor-memory A operand)
-//   dQ  = (alpha dS) K -> tensor memory -> 4 drain warps add it (16-byte vector atomics) to an
-//     fp32 accumulator in global memory, converted to bf16 after the kernel.
+//   dQ  = (alpha dS) K -> tensor memory -> 4 drain warps stage their 32 rows in shared memory and
+//     add them to an fp32 accumulator in global memory with TMA reductions (kept off the
+//     load/store path that the epilogue's shared-memory reads share), converted to bf16 after
+//     the kernel.  Rows of a ragged last query tile hold exact zeros (their dS is zero), so the
+//     reduction may cover rows of the next sequence.
 // TMEM columns: Sᵀ 0..127, dPᵀ 128..255, dV 256..319, dK 320..383, dQ 384..447.
 // Warps: 0 TMA producer, 1 MMA issuer (and the TMEM allocation), 2-17 epilogue (lane quarter
 // w % 4, 32-query chunk (w - 2) / 4: four warps per SM sub-partition to hide the latency of the
@@ -53,6 +56,7 @@ struct BwdSmem {
   alignas(1024) uint8_t q[kQStages][kTileBytes];
   alignas(1024) uint8_t dO[kQStages][kTileBytes];
   alignas(1024) uint8_t ds[2 * kTileBytes];      // [query half][key row][64 queries] SW128
+  alignas(1024) uint8_t dqs[4][2][32 * 128];     // dQ staging: [drain warp][32 columns][32 rows] fp32 SW128
   alignas(128) long long tq[kQStages][kTsStride];  // timestamps of the query tile
   uint64_t kv_full, kv_empty;
   uint64_t qd_full[kQStages], qd_empty[kQStages];
@@ -349,10 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_ts, AttnGeom g,
+                       const __grid_constant__ CUtensorMap tm_ts,
+                       const __grid_constant__ CUtensorMap tm_dq, AttnGeom g,
                        __nv_bfloat16* __restrict__ dk_out, int64_t ld_dk,
                        __nv_bfloat16* __restrict__ dv_out, int64_t ld_dv,
-                       float* __restrict__ dq_acc, int64_t ld_acc,
                        float* __restrict__ d_pos, float* __restrict__ d_time, SiluGradZ zg) {
   const int nitems = *g.item_count;
   const int total = nitems * g.H;
@@ -678,26 +682,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = warp_wait(&sm.dq_full, gs & 1, abort_flag, g.status);
         if (!ok) break;
         tc_fence_after();
-        const int i = qt * kT + quad * 32 + lane;
+        // the previous reduction from this warp's staging rows has finished reading them
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
         uint32_t a[32];
 #pragma unroll 1
         for (int ch = 0; ch < 2; ++ch) {
           tmem_ld32(lane_addr + kColDQ + 32 * ch, a);
           tmem_wait_ld32(a);
-          if (i < L) {
-            float* dst = dq_acc + static_cast<int64_t>(it.row0 + i) * ld_acc + head * kD + 32 * ch;
+          // row `lane` of the 32 x 32 box, 16-byte chunk c at c ^ (row & 7) (128-byte swizzle)
+          uint8_t* row = sm.dqs[quad][ch] + lane * 128;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              atomicAdd(reinterpret_cast<float4*>(dst + e),
-                        make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]),
-                                    __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3])));
-          }
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
         }
         tc_fence_before();
+        fence_proxy_async_smem();  // the staged rows are read by the TMA (async proxy)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.dq_empty);
+        if (lane == 0) {
+          mbar_arrive(&sm.dq_empty);
+          const int r0 = it.row0 + qt * kT + quad * 32;
+          tma_reduce_add_2d(&tm_dq, sm.dqs[quad][0], head * kD, r0);
+          tma_reduce_add_2d(&tm_dq, sm.dqs[quad][1], head * kD + 32, r0);
+          bulk_commit();
+        }
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -755,7 +767,8 @@ size_t attn_bwd_tc_smem(int P, int NB) {
 
 // Launches the backward over the work list in g (one 128-row tile per item): tq / tk / tv / tdo
 // are 64 x 128 boxes (128-byte swizzle) over Q, K, V, dO; tts a 130-element int64 box over the
-// timestamps (used when g.ts and g.rab_time are set).  dq_acc: fp32 [T, H*64], zeroed here.
+// timestamps (used when g.ts and g.rab_time are set); tdq 32 x 32 boxes (128-byte swizzle) over
+// dq_acc, fp32 [T, H*64], zeroed here and accumulated by TMA reductions.
 // grid: at most one CTA per SM (persistent).  fast: classify each 32 x 32 block of a warp
 // (hidden, visible with constant bias terms, visible with a constant time term) and skip the
 // per-element work these make unnecessary; otherwise every element takes the per-element path.
@@ -763,7 +776,7 @@ size_t attn_bwd_tc_smem(int P, int NB) {
 // not fit in shared memory.
 cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdo,
-                               const CUtensorMap& tts, const AttnGeom& g,
+                               const CUtensorMap& tts, const CUtensorMap& tdq, const AttnGeom& g,
                                __nv_bfloat16* dq, int64_t ld_dq, __nv_bfloat16* dk,
                                int64_t ld_dk, __nv_bfloat16* dv, int64_t ld_dv, float* dq_acc,
                                float* d_pos, float* d_time, int grid, bool fast,
@@ -777,8 +790,8 @@ cudaError_t launch_attn_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tk,
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, g, dk, ld_dk, dv, ld_dv, dq_acc,
-                                           static_cast<int64_t>(g.H) * 64, d_pos, d_time, zg);
+  kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tts, tdq, g, dk, ld_dk, dv, ld_dv,
+                                           d_pos, d_time, zg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(g.T) * g.H * 8;  // 8 columns per thread
