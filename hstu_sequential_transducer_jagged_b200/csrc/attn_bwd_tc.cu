@@ -200,6 +200,24 @@ __device__ __forceinline__ long long warp_max64(long long v) {
   return v;
 }
 
+// Range of the 32 query timestamps tq_c[0..31] of a block (lane l holds entry l): offsets from
+// entry 0 (one broadcast load) reduced with redux.sync when they all fit in 32 bits, else the
+// 64-bit shuffle reductions.
+__device__ __forceinline__ void query_time_range(const long long* tq_c, long long& lo,
+                                                 long long& hi) {
+  const long long v = tq_c[threadIdx.x & 31];
+  const long long base = tq_c[0];
+  const long long d = v - base;
+  if (__all_sync(0xffffffffu, d >= INT_MIN && d <= INT_MAX)) {
+    const int di = static_cast<int>(d);
+    lo = base + __reduce_min_sync(0xffffffffu, di);
+    hi = base + __reduce_max_sync(0xffffffffu, di);
+  } else {
+    lo = warp_min64(v);
+    hi = warp_max64(v);
+  }
+}
+
 // Class of the block of queries i0 .. i0+31 and keys j0 .. j0+31.  tq_c: the block's query
 // timestamps (lane l reads entry l); tj_lo / tj_hi: the warp's key timestamp range.  For the two
 // constant classes it returns the constant bias terms (summed in the per-element path's order:
@@ -218,8 +236,8 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
   float tterm = 0.f;
   ctidx = 0;
   if (t.use_time) {
-    const long long tq = tq_c[threadIdx.x & 31];
-    const long long tq_lo = warp_min64(tq), tq_hi = warp_max64(tq);
+    long long tq_lo, tq_hi;
+    query_time_range(tq_c, tq_lo, tq_hi);
     const int b_lo = time_bucket64(tq_lo - tj_hi, t.NB);
     const int b_hi = time_bucket64(tq_hi - tj_lo, t.NB);
     if (b_lo != b_hi) {
