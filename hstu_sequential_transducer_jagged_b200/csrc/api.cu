@@ -177,7 +177,8 @@ bool make_epilogue_maps(CUtensorMap* tc, CUtensorMap* tr, const void* C, int64_t
 }
 
 // 2D fp32 tensor map over a row-major [rows, cols] matrix with row stride ld (elements), box
-// {box_cols, box_rows}, 128-byte swizzle (the attention backward's dQ reduction target).
+// {box_cols, box_rows}, 64-byte swizzle (the attention backward's dQ reduction target: 16 x 32
+// boxes).
 bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
                   uint32_t box_cols, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -187,7 +188,7 @@ bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -705,7 +706,7 @@ hstu_status_t attn_backward_impl(const hstu_attn_desc_t* d, const void* q, const
       return HSTU_ERR_CUDA;
     float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.total_attn);
     CUtensorMap tdq;
-    if (!make_map_f32(&tdq, dq_acc, T, cols, cols, 32, 32)) return HSTU_ERR_CUDA;
+    if (!make_map_f32(&tdq, dq_acc, T, cols, cols, 16, 32)) return HSTU_ERR_CUDA;
     const int pgrid = grid < num_sms_current() ? grid : num_sms_current();
     e = launch_attn_bwd_tc(tq, tk, tv, tdo, tts, tdq, g, static_cast<__nv_bfloat16*>(dq), d->ld_q,
                            static_cast<__nv_bfloat16*>(dk), d->ld_k,

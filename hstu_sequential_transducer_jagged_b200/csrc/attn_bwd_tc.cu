@@ -19,15 +19,17 @@
 //     MN-major A operand of dQ); bias-table gradients summed in registers along runs of one
 //     table index and added to shared-memory bins when the index changes
 //   dV += Pᵀ dO,  dK += (alpha dS)ᵀ Q                 (tensor-memory A operand)
-//   dQ  = (alpha dS) K -> tensor memory -> 4 drain warps stage their 32 rows in shared memory and
-//     add them to an fp32 accumulator in global memory with TMA reductions (kept off the
-//     load/store path that the epilogue's shared-memory reads share), converted to bf16 after
-//     the kernel.  Rows of a ragged last query tile hold exact zeros (their dS is zero), so the
-//     reduction may cover rows of the next sequence.
+//   dQ  = (alpha dS) K -> tensor memory; at the next step each epilogue warp stages its 32 rows
+//     x 16 columns in shared memory and adds them to an fp32 accumulator in global memory with a
+//     TMA reduction (the tile is complete by then: its MMAs were issued before the next step's
+//     Sᵀ / dPᵀ, and one thread's MMAs execute in order; the next dQ is issued only after every
+//     warp's p_full, which follows its drain).  Converted to bf16 after the kernel.  Rows of a
+//     ragged last query tile hold exact zeros (their dS is zero), so the reduction may cover
+//     rows of the next sequence.
 // TMEM columns: Sᵀ 0..127, dPᵀ 128..255, dV 256..319, dK 320..383, dQ 384..447.
 // Warps: 0 TMA producer, 1 MMA issuer (and the TMEM allocation), 2-17 epilogue (lane quarter
 // w % 4, 32-query chunk (w - 2) / 4: four warps per SM sub-partition to hide the latency of the
-// per-element chain), 18-21 dQ drain (lane quarter w % 4).
+// per-element chain).  18 warps, at most 5 on a sub-partition: 96 registers a thread.
 // Items are visited in the reverse of the forward's longest-first order (which sorts by the
 // number of key tiles a query tile visits), so that key tiles near the start of long sequences,
 // which walk the most query tiles, start first.
@@ -42,7 +44,7 @@ namespace {
 constexpr int kD = 64;
 constexpr int kT = 128;
 constexpr int kQStages = 2;
-constexpr int kThreads = 704;   // 22 warps
+constexpr int kThreads = 576;   // 18 warps
 constexpr int kEpiWarps = 16;
 constexpr int kEpiFirst = 2;
 constexpr int kTileBytes = kT * kD * 2;   // 16 KB
@@ -56,28 +58,15 @@ struct BwdSmem {
   alignas(1024) uint8_t q[kQStages][kTileBytes];
   alignas(1024) uint8_t dO[kQStages][kTileBytes];
   alignas(1024) uint8_t ds[2 * kTileBytes];      // [query half][key row][64 queries] SW128
-  alignas(1024) uint8_t dqs[4][2][32 * 128];     // dQ staging: [drain warp][32 columns][32 rows] fp32 SW128
+  alignas(1024) uint8_t dqs[16][32 * 64];        // dQ staging: [epilogue warp][32 rows][16 fp32] SW64
   alignas(128) long long tq[kQStages][kTsStride];  // timestamps of the query tile
   uint64_t kv_full, kv_empty;
   uint64_t qd_full[kQStages], qd_empty[kQStages];
-  uint64_t s_full, p_full, dq_full, dq_empty, acc_full, acc_empty, drain;
+  uint64_t s_full, p_full, dq_last, acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
   // followed by float bins[2P+1 + NB]
 };
-
-__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
-  __syncwarp();
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
-        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
-        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-      :
-      : "memory");
-}
 
 __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
   __syncwarp();
@@ -406,8 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.p_full, kEpiWarps);
-    mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, 4);
+    mbar_init(&sm.dq_last, 1);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.acc_empty, kEpiWarps);
     mbar_init(&sm.drain, 1);
@@ -508,20 +496,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ts(tmem + kColDK, tmem + kColDPT + pc, smem_desc_sw128(qb + kk * 2048, kTileBytes, 1024),
                         id_kv, (!first || kk > 0) ? 1u : 0u);
           }
-          if (gs > 0) ok = mbar_wait(&sm.dq_empty, (gs - 1) & 1, abort_flag, g.status);
-          if (!ok) break;
-          tc_fence_after();
+          // dQ overwrites the previous step's tile: every epilogue warp drained it before its
+          // p_full arrival above
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk)  // 16 keys per step
             mma_bf16_ss(tmem + kColDQ, smem_desc_sw128(dsb + kk * 2048, kTileBytes, 1024),
                         smem_desc_sw128(kb + kk * 2048, kTileBytes, 1024), id_q, kk > 0 ? 1u : 0u);
-          mma_commit(&sm.dq_full);
           mma_commit(&sm.qd_empty[st]);
         }
         if (!ok) break;
         mma_commit(&sm.acc_full);
         mma_commit(&sm.kv_empty);
       }
+      if (ok && gs > 0) mma_commit(&sm.dq_last);  // the last dQ tile, drained after the loop
       if (!ok) {
         mma_commit(&sm.drain);
         mbar_wait(&sm.drain, 0, nullptr, nullptr);
@@ -549,6 +536,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tabs.NB = g.NB;
     tabs.use_pos = use_pos;
     tabs.use_time = use_time;
+    // this warp's 32 rows x 16 columns of the dQ tile in TMEM, added to dq_acc at (x, y) by a
+    // TMA reduction from this warp's staging rows (64-byte swizzle)
+    uint8_t* dq_stage = sm.dqs[warp - kEpiFirst];
+    auto drain_dq = [&](int x, int y) {
+      uint32_t a[16];
+      tmem_ld16(lane_addr + kColDQ + 16 * qc, a);
+      tmem_wait_ld16(a);
+      if (lane == 0) bulk_wait_read<0>();  // the previous reduction has read the staging rows
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(dq_stage + stage64_offset(lane, c)) =
+            make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+      fence_async_smem();  // read by the TMA (async proxy)
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_2d(&tm_dq, dq_stage, x, y);
+        bulk_commit();
+      }
+    };
+    int dq_x = 0, dq_y = 0;  // where the previous step's dQ tile goes
     int gs = 0, jj = 0;
     bool ok = true;
     for (int w = blockIdx.x; ok && w < total; w += stride, ++jj) {
@@ -578,6 +586,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && use_time) ok = warp_wait(&sm.qd_full[st], (gs / kQStages) & 1, abort_flag, g.status);
         if (!ok) break;
         tc_fence_after();
+        // the previous step's dQ (complete: issued before this step's S^T / dP^T)
+        if (gs > 0) drain_dq(dq_x, dq_y);
+        dq_x = head * kD + 16 * qc;
+        dq_y = it.row0 + qt * kT + quad * 32;
         const long long* tq = sm.tq[st] + ((it.row0 + qt * kT) & 1);
         uint8_t* ds_row = sm.ds + hq * kTileBytes + (quad * 32 + lane) * 128;
         const int rr = quad * 32 + lane;
@@ -684,50 +696,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty);
     }
-    run_p.flush(tabs.bins_pos);
-    run_t.flush(tabs.bins_time);
-  } else if (warp >= kEpiFirst + kEpiWarps) {
-    // ---------------------------------------------------------------- dQ drain
-    const int quad = warp & 3;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    int gs = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; ok && w < total; w += stride) {
-      const WorkItem it = g.items[nitems - 1 - w / g.H];
-      const int head = w % g.H, kt = it.qtile, L = it.len;
-      const int nt = (L + kT - 1) / kT;
-      for (int qt = kt; ok && qt < nt; ++qt, ++gs) {
-        ok = warp_wait(&sm.dq_full, gs & 1, abort_flag, g.status);
-        if (!ok) break;
+    if (ok && gs > 0) {  // the last dQ tile
+      ok = warp_wait(&sm.dq_last, 0, abort_flag, g.status);
+      if (ok) {
         tc_fence_after();
-        // the previous reduction from this warp's staging rows has finished reading them
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-        uint32_t a[32];
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          tmem_ld32(lane_addr + kColDQ + 32 * ch, a);
-          tmem_wait_ld32(a);
-          // row `lane` of the 32 x 32 box, 16-byte chunk c at c ^ (row & 7) (128-byte swizzle)
-          uint8_t* row = sm.dqs[quad][ch] + lane * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();  // the staged rows are read by the TMA (async proxy)
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sm.dq_empty);
-          const int r0 = it.row0 + qt * kT + quad * 32;
-          tma_reduce_add_2d(&tm_dq, sm.dqs[quad][0], head * kD, r0);
-          tma_reduce_add_2d(&tm_dq, sm.dqs[quad][1], head * kD + 32, r0);
-          bulk_commit();
-        }
+        drain_dq(dq_x, dq_y);
       }
     }
     if (lane == 0) bulk_wait_all();
+    run_p.flush(tabs.bins_pos);
+    run_t.flush(tabs.bins_time);
   }
   tc_fence_before();
   __syncthreads();
@@ -785,7 +763,7 @@ size_t attn_bwd_tc_smem(int P, int NB) {
 
 // Launches the backward over the work list in g (one 128-row tile per item): tq / tk / tv / tdo
 // are 64 x 128 boxes (128-byte swizzle) over Q, K, V, dO; tts a 130-element int64 box over the
-// timestamps (used when g.ts and g.rab_time are set); tdq 32 x 32 boxes (128-byte swizzle) over
+// timestamps (used when g.ts and g.rab_time are set); tdq 16 x 32 boxes (64-byte swizzle) over
 // dq_acc, fp32 [T, H*64], zeroed here and accumulated by TMA reductions.
 // grid: at most one CTA per SM (persistent).  fast: classify each 32 x 32 block of a warp
 // (hidden, visible with constant bias terms, visible with a constant time term) and skip the
