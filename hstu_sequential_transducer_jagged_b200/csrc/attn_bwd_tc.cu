@@ -109,20 +109,24 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // Bias-gradient run: sums dS in registers while the table index stays the same and adds the
-// sum to the shared-memory bin when the index moves on.
+// sum to the shared-memory bin when the index moves on.  Bin i sits at bins[i * stride]: the
+// time table's bins are spread one copy per lane (stride 32, bins offset by the lane), so that
+// the 32 lanes of a warp, which often end runs of the same index together, add to 32 banks
+// instead of one address.
 struct BinRun {
   int idx;
   float acc;
+  int stride;
   __device__ __forceinline__ void add(float* bins, int i, float v) {
     if (i != idx) {
-      if (idx >= 0) atomicAdd(&bins[idx], acc);
+      if (idx >= 0) atomicAdd(&bins[idx * stride], acc);
       idx = i;
       acc = 0.f;
     }
     acc += v;
   }
   __device__ __forceinline__ void flush(float* bins) {
-    if (idx >= 0) atomicAdd(&bins[idx], acc);
+    if (idx >= 0) atomicAdd(&bins[idx * stride], acc);
     idx = -1;
     acc = 0.f;
   }
@@ -379,13 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int stride = static_cast<int>(gridDim.x);
 
-  // bins[0, nbins): gradient bins; then copies of the two bias tables
+  // bins[0, nbins): gradient bins (the time entries unused); then copies of the two bias
+  // tables; then the time table's bins, 32 copies (entry b of lane l at b * 32 + l)
   float* tab_pos = bins + nbins;
   float* tab_time = tab_pos + npos;
+  float* tbins = tab_pos + nbins;
+  const int ntime = nbins - npos;
   for (int e = threadIdx.x; e < nbins; e += kThreads) {
     bins[e] = 0.f;
     tab_pos[e] = e < npos ? g.rab_pos[e] : g.rab_time[e - npos];
   }
+  for (int e = threadIdx.x; e < 32 * ntime; e += kThreads) tbins[e] = 0.f;
   if (threadIdx.x == 0) {
     mbar_init(&sm.kv_full, 1);
     mbar_init(&sm.kv_empty, 1);
@@ -525,12 +533,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Bias-gradient runs: along one key row the table index changes only where the clamped
     // distance or the time bucket changes, so each thread sums a run in registers and adds it
     // to the shared-memory bin when the index moves on.
-    BinRun run_p{-1, 0.f}, run_t{-1, 0.f};
+    BinRun run_p{-1, 0.f, 1}, run_t{-1, 0.f, 32};
     BwdTabs tabs;
     tabs.pos = tab_pos;
     tabs.time = tab_time;
     tabs.bins_pos = bins;
-    tabs.bins_time = bins + npos;
+    tabs.bins_time = tbins + lane;
     tabs.alpha = alpha;
     tabs.P = g.P;
     tabs.NB = g.NB;
@@ -710,7 +718,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   for (int e = threadIdx.x; e < nbins; e += kThreads) {
-    const float v = bins[e];
+    float v = 0.f;
+    if (e < npos) {
+      v = bins[e];
+    } else {
+      const float* c = tbins + 32 * (e - npos);
+#pragma unroll 4
+      for (int l = 0; l < 32; ++l) v += c[l];
+    }
     if (v != 0.f) atomicAdd(e < npos ? &d_pos[e] : &d_time[e - npos], v);
   }
   if (warp == 1) {
@@ -758,7 +773,7 @@ __global__ void f32_to_bf16_rows(const float* __restrict__ src, int64_t ld_src,
 int attn_bwd_tc_ts_box() { return kTsBox; }
 
 size_t attn_bwd_tc_smem(int P, int NB) {
-  return sizeof(BwdSmem) + 1024 + 2 * sizeof(float) * (2 * P + 1 + NB);
+  return sizeof(BwdSmem) + 1024 + 2 * sizeof(float) * (2 * P + 1 + NB) + 32 * sizeof(float) * NB;
 }
 
 // Launches the backward over the work list in g (one 128-row tile per item): tq / tk / tv / tdo
