@@ -154,7 +154,9 @@ struct BwdTabs {
 // the second also with per-element time buckets from 32-bit differences; anything else
 // (per-element mask, bias and bins).
 constexpr int kChunkGeneral = 0, kChunkTimeConst = 1, kChunkConst = 2, kChunkZero = 3,
-              kChunkBandTC = 4, kChunkBandT32 = 5;
+              kChunkBandTC = 4, kChunkBandT32 = 5, kChunkBandTH = 6;
+// kChunkBandTH: as kChunkBandT32 with every pair in bucket b or b + 1 (ctidx = b): the bucket is
+// b + 1 iff the difference is at least 2^(b+1), one compare per pair.
 
 // Position-bin sums of a fully visible 32 x 32 block whose distances all lie inside the band:
 // the pair (key j0 + l, query i0 + e) falls in diagonal e - l + 31 (0..62), i.e. bin
@@ -236,7 +238,9 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
     if (b_lo != b_hi) {
       // per-element buckets: from the 32-bit differences when all of them lie in (-2^23, 2^23)
       const bool small = tq_hi - tj_lo < (1ll << 23) && tq_lo - tj_hi > -(1ll << 23);
-      return (small && (band || !t.use_pos)) ? kChunkBandT32 : kChunkGeneral;
+      if (!(small && (band || !t.use_pos))) return kChunkGeneral;
+      ctidx = b_lo;
+      return b_hi == b_lo + 1 ? kChunkBandTH : kChunkBandT32;
     }
     ctidx = b_lo;
     tterm = t.time[b_lo];
@@ -313,10 +317,11 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[W], const uint32_t
   if (V != kChunkGeneral && t.use_time) run_t.add(t.bins_time, ctidx, sum);
 }
 
-// W columns of a fully visible band block (classes kChunkBandTC and kChunkBandT32): the same P and
-// alpha dS as bwd_chunk, with the position bins summed by diagonal (dg) and, for kChunkBandT32,
-// the time bucket of each pair from the low 32 bits of the two timestamps (every difference of
-// the block lies in (-2^23, 2^23)).  eg0: block column of the first of the W queries; pb: this
+// W columns of a fully visible band block (classes kChunkBandTC, kChunkBandT32, kChunkBandTH): the
+// same P and alpha dS as bwd_chunk, with the position bins summed by diagonal (dg) and, for
+// kChunkBandT32 / kChunkBandTH, the time bucket of each pair from the low 32 bits of the two
+// timestamps (every difference of the block lies in (-2^23, 2^23)); kChunkBandTH sums its two
+// time bins in registers and adds them to two runs (run_t, run_t2).  eg0: block column of the first of the W queries; pb: this
 // key row's position index for that query (i - j + P); tq_lo: the queries' timestamps as pairs
 // of 32-bit words, low word first.
 template <int V, int W>
@@ -324,8 +329,13 @@ __device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uin
                                                uint32_t (&pk)[W / 2], uint32_t (&dk)[W / 2],
                                                int eg0, int pb, const unsigned* tq_lo,
                                                unsigned tj_lo, const BwdTabs& t, float cbias,
-                                               int ctidx, DiagBins& dg, BinRun& run_t) {
-  float sum = 0.f;  // kChunkBandTC: the block's dS total for its one time bin
+                                               int ctidx, DiagBins& dg, BinRun& run_t,
+                                               BinRun& run_t2) {
+  float sum = 0.f;     // kChunkBandTC: the block's dS total for its one time bin
+  float sum_hi = 0.f;  // kChunkBandTH: the dS total of bucket ctidx + 1 (sum: of ctidx)
+  const int thr = V == kChunkBandTH ? threshold_of(ctidx) : 0;
+  const float t_lo = V == kChunkBandTH ? t.time[ctidx] : 0.f;
+  const float t_hi = V == kChunkBandTH ? t.time[ctidx + 1] : 0.f;
 #pragma unroll
   for (int e = 0; e < W; e += 2) {
     float pv[2], dsa[2];
@@ -334,9 +344,13 @@ __device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uin
       float bias = V == kChunkBandTC ? cbias : 0.f;
       if (t.use_pos) bias += t.pos[pb + e + u];
       int bidx = 0;
+      bool upper = false;
       if (V == kChunkBandT32) {
         bidx = bucket_small(static_cast<int>(tq_lo[2 * (e + u)] - tj_lo), t.NB - 1);
         bias += t.time[bidx];
+      } else if (V == kChunkBandTH) {
+        upper = threshold_takes_hi(static_cast<int>(tq_lo[2 * (e + u)] - tj_lo), thr);
+        bias += upper ? t_hi : t_lo;
       }
       const float x = fmaf(t.alpha, __uint_as_float(s[e + u]), bias);
       const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
@@ -345,6 +359,9 @@ __device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uin
       if (t.use_pos) dg.add(eg0 + e + u, dsv);
       if (V == kChunkBandT32) {
         run_t.add(t.bins_time, bidx, dsv);
+      } else if (V == kChunkBandTH) {
+        sum += upper ? 0.f : dsv;
+        sum_hi += upper ? dsv : 0.f;
       } else {
         sum += dsv;
       }
@@ -355,6 +372,10 @@ __device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uin
     dk[e >> 1] = pack_bf16x2(dsa[0], dsa[1]);
   }
   if (V == kChunkBandTC && t.use_time) run_t.add(t.bins_time, ctidx, sum);
+  if (V == kChunkBandTH) {  // two runs, so that neither ends at every block
+    run_t.add(t.bins_time, ctidx, sum);
+    run_t2.add(t.bins_time, ctidx + 1, sum_hi);
+  }
 }
 
 // Items: (sequence, 128-row key tile) from the work list built with one tile per item, times heads.
@@ -533,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Bias-gradient runs: along one key row the table index changes only where the clamped
     // distance or the time bucket changes, so each thread sums a run in registers and adds it
     // to the shared-memory bin when the index moves on.
-    BinRun run_p{-1, 0.f, 1}, run_t{-1, 0.f, 32};
+    BinRun run_p{-1, 0.f, 1}, run_t{-1, 0.f, 32}, run_t2{-1, 0.f, 32};
     BwdTabs tabs;
     tabs.pos = tab_pos;
     tabs.time = tab_time;
@@ -631,11 +652,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             else if (cls == kChunkBandTC)
               bwd_chunk_band<kChunkBandTC, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
                                                tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
-                                               run_t);
+                                               run_t, run_t2);
             else if (cls == kChunkBandT32)
               bwd_chunk_band<kChunkBandT32, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
                                                 tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
-                                                run_t);
+                                                run_t, run_t2);
+            else if (cls == kChunkBandTH)
+              bwd_chunk_band<kChunkBandTH, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
+                                               tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
+                                               run_t, run_t2);
             else if (cls == kChunkTimeConst)
               bwd_chunk<kChunkTimeConst, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row,
                                              tabs, cbias, cpidx, ctidx, run_p, run_t);
@@ -654,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(ds_row + ((cb ^ (rr & 7)) * 16)) = val;
           }
         }
-        if ((cls == kChunkBandTC || cls == kChunkBandT32) && use_pos)
+        if (cls >= kChunkBandTC && use_pos)
           dg.flush(tabs.bins_pos, i0 - j0 - 31 + g.P);
         tmem_wait_st();
         fence_async_smem();  // the dS tile is read by the dQ MMA (async proxy)
@@ -714,6 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) bulk_wait_all();
     run_p.flush(tabs.bins_pos);
     run_t.flush(tabs.bins_time);
+    run_t2.flush(tabs.bins_time);
   }
   tc_fence_before();
   __syncthreads();
