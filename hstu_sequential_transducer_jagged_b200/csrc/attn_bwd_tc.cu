@@ -154,9 +154,11 @@ struct BwdTabs {
 // the second also with per-element time buckets from 32-bit differences; anything else
 // (per-element mask, bias and bins).
 constexpr int kChunkGeneral = 0, kChunkTimeConst = 1, kChunkConst = 2, kChunkZero = 3,
-              kChunkBandTC = 4, kChunkBandT32 = 5, kChunkBandTH = 6;
+              kChunkBandTC = 4, kChunkBandT32 = 5, kChunkBandTH = 6, kChunkBandT32M = 7;
 // kChunkBandTH: as kChunkBandT32 with every pair in bucket b or b + 1 (ctidx = b): the bucket is
 // b + 1 iff the difference is at least 2^(b+1), one compare per pair.
+// kChunkBandT32M: the causal diagonal block of two history tiles (i0 == j0), pair (j, i) visible
+// iff j <= i, otherwise as kChunkBandT32.
 
 // Position-bin sums of a fully visible 32 x 32 block whose distances all lie inside the band:
 // the pair (key j0 + l, query i0 + e) falls in diagonal e - l + 31 (0..62), i.e. bin
@@ -224,10 +226,13 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
                                            int& ctidx) {
   const int j1 = j0 + 31;
   if (i0 >= L || j0 >= L || i0 + 31 < j0) return kChunkZero;
-  if (!(i0 >= j1 && i0 + 31 < L && j1 < n)) return kChunkGeneral;  // not every pair visible
-  // every distance i - j of the block in [0, P] and every query a history token: the position
+  // the diagonal block inside the history (both masks reduce to j <= i there)
+  const bool diag = i0 == j0 && i0 + 31 < n && t.use_time;
+  if (!(i0 >= j1 && i0 + 31 < L && j1 < n) && !diag) return kChunkGeneral;
+  // every distance i - j of the block in [-P, P] and every query a history token: the position
   // index is i - j + P, no clamp
-  const bool band = t.use_pos && i0 + 31 < n && i0 + 31 - j0 <= t.P;
+  const bool band =
+      t.use_pos && i0 + 31 < n && i0 + 31 - j0 <= t.P && (!diag || j1 - i0 <= t.P);
   float tterm = 0.f;
   ctidx = 0;
   if (t.use_time) {
@@ -240,8 +245,10 @@ __device__ __forceinline__ int chunk_class(int i0, int j0, int L, int n, const B
       const bool small = tq_hi - tj_lo < (1ll << 23) && tq_lo - tj_hi > -(1ll << 23);
       if (!(small && (band || !t.use_pos))) return kChunkGeneral;
       ctidx = b_lo;
+      if (diag) return kChunkBandT32M;
       return b_hi == b_lo + 1 ? kChunkBandTH : kChunkBandT32;
     }
+    if (diag) return kChunkGeneral;
     ctidx = b_lo;
     tterm = t.time[b_lo];
   }
@@ -324,10 +331,10 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[W], const uint32_t
 // time bins in registers and adds them to two runs (run_t, run_t2).  eg0: block column of the first of the W queries; pb: this
 // key row's position index for that query (i - j + P); tq_lo: the queries' timestamps as pairs
 // of 32-bit words, low word first.
-template <int V, int W>
+template <int V, int W, bool MASKED = false>
 __device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uint32_t (&dp)[W],
                                                uint32_t (&pk)[W / 2], uint32_t (&dk)[W / 2],
-                                               int eg0, int pb, const unsigned* tq_lo,
+                                               int eg0, int pb, int jmi, const unsigned* tq_lo,
                                                unsigned tj_lo, const BwdTabs& t, float cbias,
                                                int ctidx, DiagBins& dg, BinRun& run_t,
                                                BinRun& run_t2) {
@@ -354,8 +361,13 @@ __device__ __forceinline__ void bwd_chunk_band(const uint32_t (&s)[W], const uin
       }
       const float x = fmaf(t.alpha, __uint_as_float(s[e + u]), bias);
       const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
-      const float p = x * sg;
-      const float dsv = __uint_as_float(dp[e + u]) * sg * fmaf(x, 1.f - sg, 1.f);
+      float p = x * sg;
+      float dsv = __uint_as_float(dp[e + u]) * sg * fmaf(x, 1.f - sg, 1.f);
+      if (MASKED) {  // column e + u visible iff it is at least jmi (the key row's own query)
+        const bool vis = e + u >= jmi;
+        p = vis ? p : 0.f;
+        dsv = vis ? dsv : 0.f;
+      }
       if (t.use_pos) dg.add(eg0 + e + u, dsv);
       if (V == kChunkBandT32) {
         run_t.add(t.bins_time, bidx, dsv);
@@ -650,15 +662,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               bwd_chunk<kChunkConst, 16>(sv, dp, pk, dk, i0 + 16 * hf, tq_c + 16 * hf, row, tabs,
                                          cbias, cpidx, ctidx, run_p, run_t);
             else if (cls == kChunkBandTC)
-              bwd_chunk_band<kChunkBandTC, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
+              bwd_chunk_band<kChunkBandTC, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P, 0,
                                                tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
                                                run_t, run_t2);
             else if (cls == kChunkBandT32)
-              bwd_chunk_band<kChunkBandT32, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
+              bwd_chunk_band<kChunkBandT32, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P, 0,
                                                 tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
                                                 run_t, run_t2);
+            else if (cls == kChunkBandT32M)
+              bwd_chunk_band<kChunkBandT32, 16, true>(sv, dp, pk, dk, 16 * hf,
+                                                      i0 + 16 * hf - jrow + g.P,
+                                                      jrow - (i0 + 16 * hf), tq_lo + 32 * hf,
+                                                      tj_lo32, tabs, cbias, ctidx, dg, run_t,
+                                                      run_t2);
             else if (cls == kChunkBandTH)
-              bwd_chunk_band<kChunkBandTH, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P,
+              bwd_chunk_band<kChunkBandTH, 16>(sv, dp, pk, dk, 16 * hf, i0 + 16 * hf - jrow + g.P, 0,
                                                tq_lo + 32 * hf, tj_lo32, tabs, cbias, ctidx, dg,
                                                run_t, run_t2);
             else if (cls == kChunkTimeConst)
