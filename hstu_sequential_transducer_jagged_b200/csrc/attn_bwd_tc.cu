@@ -16,8 +16,10 @@
 //     dS = dP σ (1 + x (1 - σ)), 0 where the mask hides the pair; Pᵀ and (alpha dS)ᵀ as bf16
 //     over the first half of each 32-query chunk's own Sᵀ / dPᵀ columns (a chunk is one warp's,
 //     so no warp writes columns another still reads), (alpha dS)ᵀ also to shared memory (the
-//     MN-major A operand of dQ); bias-table gradients summed in registers along runs of one
-//     table index and added to shared-memory bins when the index changes
+//     MN-major A operand of dQ); bias-table gradients: position bins of band blocks summed by
+//     diagonal (DiagBins), otherwise summed in registers along runs of one table index and
+//     added to shared-memory bins when the index changes (the time table's bins one copy per
+//     lane, so that lanes ending runs of the same index together hit different banks)
 //   dV += Pᵀ dO,  dK += (alpha dS)ᵀ Q                 (tensor-memory A operand)
 //   dQ  = (alpha dS) K -> tensor memory; at the next step each epilogue warp stages its 32 rows
 //     x 16 columns in shared memory and adds them to an fp32 accumulator in global memory with a
