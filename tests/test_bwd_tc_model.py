@@ -117,3 +117,36 @@ def test_block_classes_exact():
                 if cls == "const":
                     assert (pidx[ii, jj] == cp).all()
     assert seen == {"zero", "general", "const", "timeconst"}
+
+
+# ------------------------------------------------------------ diagonal position-bin sums
+def diag_bins_by_shuffle(v, src_offset=-1):
+    """The band blocks' position-bin sums as the kernel forms them (DiagBins in attn_bwd_tc.cu):
+    lane m keeps diagonals m (lo) and m + 32 (hi); at block column e it takes the value of lane
+    (e + src_offset - m) mod 32 from the warp shuffle and adds it to lo when m >= e, else to hi.
+    v[l, e] is the dS of key row l (lane) and block column e.  Returns the 63 diagonal sums,
+    diagonal k = e - l + 31."""
+    lo = np.zeros(32)
+    hi = np.zeros(32)
+    lanes = np.arange(32)
+    for e in range(v.shape[1]):
+        src = (e + src_offset - lanes) & 31
+        w = v[src, e]
+        lo += np.where(lanes >= e, w, 0.0)
+        hi += np.where(lanes >= e, 0.0, w)
+    return np.concatenate([lo, hi[:31]])
+
+
+@pytest.mark.parametrize("width", [16, 32])
+def test_diag_bins_shuffle_mapping(width):
+    """Brute force: every pair (l, e) lands on diagonal e - l + 31; the kernel's mapping gives
+    the same 63 sums for a full block and for the first 16 columns (one half)."""
+    rng = np.random.default_rng(7 + width)
+    v = rng.standard_normal((32, width))
+    ref = np.zeros(63)
+    for l in range(32):
+        for e in range(width):
+            ref[e - l + 31] += v[l, e]
+    np.testing.assert_allclose(diag_bins_by_shuffle(v), ref, rtol=0, atol=1e-12)
+    # the planted mistake: a source lane off by one must not reproduce the sums
+    assert not np.allclose(diag_bins_by_shuffle(v, src_offset=0), ref)
